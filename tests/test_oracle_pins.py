@@ -1,0 +1,301 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks one oracle function against a closed form, an independent
+library routine (scipy / numpy / Python's math), brute force, or the
+hand-derived worked example in tests/golden/.  tests/test_oracle_mutations.py
+plants plausible mistakes in a copy of the oracle's C source and checks that
+these pins catch every one of them.
+
+Passages pinned (all on page "十亿参数的三维重建模型，能塞进手机吗？"):
+  训练后量化（PTQ）              symmetric quantizer, rounding, clamp range
+  预全局旋转（Pre-Global-Rotation） Hadamard, H H^T = I, product invariance, outlier spreading
+  后局部平滑（Post-Local-Smooth）  smoothing factors, alpha, rotate-then-scale
+  细粒度量化粒度                  per-token / per-channel steps (reading)
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle
+from w4a4_post_quantized_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _popcount_parity_matrix(d):
+    """Closed form of the Sylvester Hadamard entry: (-1)^popcount(i & j)."""
+    i = np.arange(d, dtype=np.uint32)[:, None]
+    j = np.arange(d, dtype=np.uint32)[None, :]
+    par = np.bitwise_count(i & j) & 1
+    return np.where(par == 1, -1.0, 1.0)
+
+
+# ------------------------------------------------------------------ Hadamard
+@pytest.mark.parametrize("d", [1, 2, 4, 8, 16, 64, 256, 1024, 4096])
+def test_hadamard_closed_form(d):
+    H = oracle.hadamard(d)
+    assert np.array_equal(H, _popcount_parity_matrix(d))
+    if d >= 2:
+        assert np.array_equal(H, scipy.linalg.hadamard(d).astype(np.float64))
+
+
+@pytest.mark.parametrize("d", [2, 16, 1024, 2048])
+def test_hadamard_orthogonal(d):
+    H = oracle.hadamard(d)
+    G = H @ H.T  # exact in fp64: +-1 entries, sums <= d
+    assert np.array_equal(G, d * np.eye(d))
+
+
+def test_hadamard_rejects_non_power_of_two():
+    with pytest.raises(ValueError):
+        oracle.hadamard(12)
+
+
+# ------------------------------------------------------------------ rotation
+@pytest.mark.parametrize("d", [4, 64, 1024])
+def test_rotate_matches_library_product(d):
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((7, d))
+    ref = X @ scipy.linalg.hadamard(d).astype(np.float64) / math.sqrt(d)
+    got = oracle.rotate(X)
+    assert np.max(np.abs(got - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+@pytest.mark.parametrize("d", [8, 1024])
+def test_rotate_is_an_involution_and_preserves_norm(d):
+    # H/sqrt(d) is symmetric and orthonormal, so applying it twice is the identity
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((5, d)) * 10
+    Y = oracle.rotate(X)
+    np.testing.assert_allclose(np.linalg.norm(Y, axis=1), np.linalg.norm(X, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(oracle.rotate(Y), X, rtol=0, atol=1e-12 * np.max(np.abs(X)))
+
+
+@pytest.mark.parametrize("d", [64, 1024])
+def test_rotation_keeps_matmul_invariant(d):
+    # (X H)(W H)^T = X H H^T W^T = X W^T   [pre-global rotation, product invariance]
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((6, d))
+    W = rng.standard_normal((5, d)) * 0.02
+    lhs = oracle.rotate(X) @ oracle.rotate(W).T
+    rhs = X @ W.T
+    assert np.max(np.abs(lhs - rhs)) <= 1e-12 * np.max(np.abs(X)) * np.max(np.abs(W)) * d
+
+
+@pytest.mark.parametrize("d", [16, 1024])
+def test_one_hot_outlier_is_spread_evenly(d):
+    # the lemma: an outlier on one channel lands on every channel with equal magnitude
+    for j in [0, 1, d // 2 + 3, d - 1]:
+        e = np.zeros((1, d))
+        e[0, j] = 1.0
+        r = oracle.rotate(e)[0]
+        assert np.allclose(np.abs(r), 1.0 / math.sqrt(d), rtol=0, atol=1e-15)
+        assert np.array_equal(np.sign(r), _popcount_parity_matrix(d)[j])
+
+
+def test_rotation_reduces_heavy_tails():
+    X = synth.bf16_bits_to_f32(synth.activations(1374, 1024, seed=5)).astype(np.float64)
+    Xt = oracle.rotate(X)
+    ratio_before = np.max(np.abs(X)) / np.sqrt(np.mean(X * X))
+    ratio_after = np.max(np.abs(Xt)) / np.sqrt(np.mean(Xt * Xt))
+    assert ratio_after < 0.5 * ratio_before
+
+
+# ----------------------------------------------------------------- smoothing
+def test_smooth_factors_hand_values():
+    Xt = np.array([[5.0, -1.0, -2.0, 0.0], [-4.0, 0.5, 1.0, 0.0]])
+    Wt = np.array([[2.0, 0.0, 0.0, 0.0], [0.0, -2.0, 0.0, 3.0]])
+    s = oracle.smooth_factors(Xt, Wt, 0.5)
+    np.testing.assert_allclose(s, [math.sqrt(5 / 2), math.sqrt(1 / 2), 1.0, 1.0], rtol=1e-15)
+    s25 = oracle.smooth_factors(Xt, Wt, 0.25)
+    np.testing.assert_allclose(s25[:2], [5 ** 0.25 / 2 ** 0.75, 1.0 / 2 ** 0.75], rtol=1e-15)
+
+
+def test_smoothing_identity_and_balance():
+    rng = np.random.default_rng(4)
+    Xt = rng.standard_normal((30, 64)) * rng.uniform(0.1, 30, 64)
+    Wt = rng.standard_normal((20, 64)) * 0.02
+    s = oracle.smooth_factors(Xt, Wt, 0.5)
+    Xh, Wh = Xt / s, Wt * s
+    # SmoothQuant identity: (X diag(s)^-1)(diag(s) W^T) = X W^T
+    np.testing.assert_allclose(Xh @ Wh.T, Xt @ Wt.T, rtol=1e-12, atol=1e-12)
+    # alpha = 0.5 equalises the per-channel maxima of both operands
+    np.testing.assert_allclose(np.max(np.abs(Xh), 0), np.max(np.abs(Wh), 0), rtol=1e-12)
+
+
+# ----------------------------------------------------------------- quantizer
+def test_quantizer_hand_values_and_ties():
+    y = np.array([[1.0, -3.5, 7.0, 0.5, 2.5, -7.0, 0.0, 3.49, -0.5, 1.5]])
+    q, d = oracle.quantize_rows(y, 4)
+    assert d[0] == 1.0
+    # round half to even: -3.5 -> -4, 0.5 -> 0, 2.5 -> 2, -0.5 -> 0, 1.5 -> 2
+    assert q.tolist() == [[1, -4, 7, 0, 2, -7, 0, 3, 0, 2]]
+
+
+@pytest.mark.parametrize("decision", ["f64", "f32"])
+def test_quantizer_range_error_and_extremes(decision):
+    rng = np.random.default_rng(6)
+    Y = rng.standard_normal((50, 256)) * rng.uniform(1e-3, 1e3, (50, 1))
+    Y[3] = 0.0
+    q, d = oracle.quantize_rows(Y, 4, decision)
+    assert q.min() >= -8 and q.max() <= 7
+    assert d[3] == 0 and np.all(q[3] == 0)
+    nz = d > 0
+    err = np.abs(Y[nz] - q[nz] * d[nz, None])
+    assert np.all(err <= d[nz, None] * (0.5 + 1e-6))
+    amax_idx = np.argmax(np.abs(Y[nz]), axis=1)
+    picked = q[nz][np.arange(nz.sum()), amax_idx]
+    assert np.all(np.abs(picked) == 7)
+    np.testing.assert_allclose(d[nz], np.max(np.abs(Y[nz]), 1) / 7, rtol=1e-6)
+
+
+def test_quantizer_other_bit_width():
+    y = np.array([[127.0, -63.5, 1.0]])
+    q, d = oracle.quantize_rows(y, 8)
+    assert d[0] == 1.0 and q.tolist() == [[127, -64, 1]]
+
+
+def test_quantizer_decisions_agree_away_from_ties():
+    rng = np.random.default_rng(7)
+    Y = rng.standard_normal((40, 1024))
+    q64, d64 = oracle.quantize_rows(Y, 4, "f64")
+    q32, d32 = oracle.quantize_rows(Y, 4, "f32")
+    ratio = Y / d64[:, None]
+    frac = np.abs(ratio - np.floor(ratio) - 0.5)
+    far = frac > 1e-5
+    assert np.array_equal(q64[far], q32[far])
+    np.testing.assert_allclose(d32, d64, rtol=1e-6)
+
+
+# --------------------------------------------------------------------- int4 packing
+def test_pack_nibble_order():
+    q = np.array([[1, -1, -8, 7, 0, -8, 3, 4]], np.int8)
+    p = oracle.pack_int4(q)
+    assert p.tolist() == [[0xF1, 0x78, 0x80, 0x43]]
+    assert np.array_equal(oracle.unpack_int4(p, 8), q)
+
+
+def test_pack_roundtrip_all_codes():
+    rng = np.random.default_rng(8)
+    q = rng.integers(-8, 8, (9, 64)).astype(np.int8)
+    assert np.array_equal(oracle.unpack_int4(oracle.pack_int4(q), 64), q)
+    b = synth.random_packed_codes(5, 32, seed=3)
+    assert np.array_equal(oracle.pack_int4(oracle.unpack_int4(b, 32)), b)
+
+
+def test_pack_rejects_out_of_range():
+    with pytest.raises(ValueError):
+        oracle.pack_int4(np.array([[8, 0]], np.int8))
+
+
+# ----------------------------------------------------------------- integer GEMM
+def test_int_gemm_brute_force_4x8x8():
+    rng = np.random.default_rng(9)
+    A = rng.integers(-8, 8, (4, 8)).astype(np.int8)
+    B = rng.integers(-8, 8, (8, 8)).astype(np.int8)
+    acc = oracle.int_gemm(A, B)
+    for m in range(4):
+        for n in range(8):
+            s = 0
+            for k in range(8):
+                s += int(A[m, k]) * int(B[n, k])
+            assert acc[m, n] == s
+
+
+def test_int_gemm_matches_numpy_rectangular():
+    rng = np.random.default_rng(10)
+    A = rng.integers(-8, 8, (13, 96)).astype(np.int8)
+    B = rng.integers(-8, 8, (40, 96)).astype(np.int8)
+    assert np.array_equal(oracle.int_gemm(A, B), A.astype(np.int64) @ B.astype(np.int64).T)
+    # extremes: every product (-8)(-8) = 64 accumulates to 64*K without overflow
+    A = np.full((2, 4096), -8, np.int8)
+    assert np.all(oracle.int_gemm(A, A) == 64 * 4096)
+
+
+def test_dequant_hand_values():
+    acc = np.array([[49, -21], [0, 7]], np.int64)
+    Y = oracle.dequant(acc, [0.5, 2.0], [0.25, 4.0], [1.0, -1.0])
+    assert Y.tolist() == [[49 * 0.125 + 1.0, -21 * 2.0 - 1.0], [1.0, 7 * 8.0 - 1.0]]
+    Y0 = oracle.dequant(acc, [1.0, 1.0], [1.0, 1.0], None)
+    assert np.array_equal(Y0, acc.astype(np.float64))
+
+
+def test_matmul_nt_matches_numpy():
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((5, 33))
+    W = rng.standard_normal((7, 33))
+    b = rng.standard_normal(7)
+    np.testing.assert_allclose(oracle.matmul_nt(X, W, b), X @ W.T + b, rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------------------------------ bf16 helpers
+def _py_bf16_round(v: float) -> float:
+    """Independent nearest-even rounding of a double to 8 significant bits."""
+    if v == 0.0:
+        return v
+    m, e = math.frexp(v)
+    return math.ldexp(round(m * 256.0), e - 8)   # Python's round() is half-to-even
+
+
+def test_bf16_conversions_exact_and_rne():
+    vals = np.array([1.0, -2.5, 3.140625, 1e-3, 65504.0, -7.25])
+    bits = synth.to_bf16_bits(vals.astype(np.float32))
+    back = oracle.bf16_to_f64(bits)
+    assert np.array_equal(back, synth.bf16_bits_to_f32(bits).astype(np.float64))
+    # ties: 1 + 2^-8 is halfway between 1 and 1 + 2^-7 -> even (1.0); 1 + 3*2^-8 -> 1 + 2^-6
+    t = oracle.bf16_to_f64(oracle.f64_to_bf16(np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8)])))
+    assert t.tolist() == [1.0, 1 + 2 ** -6, -1.0]
+    rng = np.random.default_rng(12)
+    v = rng.standard_normal(2000) * 10 ** rng.uniform(-3, 3, 2000)
+    got = oracle.bf16_to_f64(oracle.f64_to_bf16(v))
+    assert got.tolist() == [_py_bf16_round(float(x)) for x in v]
+
+
+def test_gelu_against_math_erf():
+    x = synth.to_bf16_bits(np.linspace(-6, 6, 777).astype(np.float32))
+    xs = oracle.bf16_to_f64(x)
+    got = oracle.bf16_to_f64(oracle.gelu_bf16(x))
+    ref = [_py_bf16_round(0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0)))) for v in xs]
+    assert got.tolist() == ref
+    one = oracle.bf16_to_f64(oracle.gelu_bf16(synth.to_bf16_bits(np.array([1.0, 0.0], np.float32))))
+    assert one[1] == 0.0 and abs(one[0] - 0.8413447460685429) < 2 ** -8
+
+
+# ------------------------------------------------------------------ worked example
+def test_worked_example_k4():
+    g = json.load(open(os.path.join(GOLDEN, "worked_example_k4.json")))
+    X = synth.to_bf16_bits(np.array(g["inputs"]["X"], np.float32))
+    W = synth.to_bf16_bits(np.array(g["inputs"]["W"], np.float32))
+    b = synth.to_bf16_bits(np.array(g["inputs"]["bias"], np.float32))
+    pw = oracle.prepare_weights(W, b, X, alpha=g["inputs"]["alpha"])
+    ev = {k: (np.array([[eval(e, {"sqrt": math.sqrt}) if isinstance(e, str) else e for e in row]
+                        for row in v]) if isinstance(v[0], list)
+              else np.array([eval(e, {"sqrt": math.sqrt}) for e in v]))
+          for k, v in g["expected"].items()}
+    np.testing.assert_allclose(oracle.rotate(oracle.bf16_to_f64(X)), ev["X_rot"], atol=1e-14)
+    np.testing.assert_allclose(pw.Wt, ev["W_rot"], atol=1e-14)
+    np.testing.assert_allclose(pw.s, ev["s"], rtol=1e-14)
+    assert pw.qw.tolist() == ev["qw"].astype(int).tolist()
+    np.testing.assert_allclose(pw.delta_ch, ev["delta_ch"], rtol=1e-14)
+    Y, qx, dt, acc = oracle.linear(X, pw)
+    assert qx.tolist() == ev["qx"].astype(int).tolist()
+    np.testing.assert_allclose(dt, ev["delta_tok"], rtol=1e-14)
+    assert acc.tolist() == ev["acc"].astype(int).tolist()
+    np.testing.assert_allclose(Y[0], ev["Y"], rtol=1e-13)
+    np.testing.assert_allclose(oracle.reference_fp(X, W, b)[0], ev["Y_unquantized"], rtol=1e-14)
+
+
+def test_dsfq_beats_single_steps_on_heavy_tails():
+    """Ablation the pages report (rotation + scaling beat either alone); on the
+    heavy-tailed generator the oracle's SQNR orders the same way."""
+    X = synth.activations(1374, 256, seed=21)
+    W = synth.weights(128, 256, seed=22)
+    b = synth.bias(128, seed=23)
+    ref = oracle.reference_fp(X, W, b)
+    full = oracle.linear(X, oracle.prepare_weights(W, b, X))[0]
+    plain = oracle.linear(X, oracle.prepare_weights(W, b, X, plain=True), plain=True)[0]
+    assert oracle.sqnr_db(ref, full) > oracle.sqnr_db(ref, plain) + 3.0
