@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark of the DSFQ W4A4 linear (libw4a4) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Workload (default): the frame-attention QKV linear of a VGGT-style 1024-wide
+transformer at 8 frames: X [10992, 1024] bf16 -> Y [10992, 3072] bf16, one
+"step" = the whole hot path on one batch: rotate + smooth + per-token int4
+quantize + pack (kernel 1), integer GEMM on the tensor cores + dequant/bias
+epilogue (kernel 2).  Weight preparation is offline and untimed.
+
+Metric: W4A4 linear throughput in TOPS (2*M*N*K integer ops per step), with
+tokens/s alongside; roofline fractions against the measured peaks.
+
+Under torchrun each rank runs an independent replica on its own GPU (token
+batches are independent: weak scaling, no data-path collective); the timed
+region is bracketed by barrier + synchronize and the max over ranks is used.
+
+--impl reference times the CPU oracle (the only reference this build has: the
+pages hold no code) on a bounded sample of the same workload, on the host
+cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w4a4_post_quantized_b200 import synth  # noqa: E402
+
+WORKLOADS = {
+    "c2_frame_qkv": dict(frames=8, K=1024, N=3072,
+                         desc="VGGT frame-attention QKV linear, 8 frames: M=10992, K=1024, N=3072"),
+    "c1_single_linear": dict(frames=1, K=1024, N=1024,
+                             desc="single linear, 1 frame: M=1374, K=1024, N=1024"),
+    "c3_fc2": dict(frames=8, K=4096, N=1024,
+                   desc="VGGT MLP fc2 (GELU on input), 8 frames: M=10992, K=4096, N=1024", gelu=True),
+}
+METRIC = "W4A4 linear TOPS & tokens/s on VGGT shapes, % of INT8 TC peak / HBM BW"
+NSETS = 4          # input/output buffer sets rotated so no step finds its inputs in L2
+INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput ratio (4.5 / 2.25 POPS)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained"),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def profile_traffic(kernel_file: str, key: str):
+    """Per-launch DRAM bytes from the committed ncu summary, or None when the
+    kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(key)
+    if not d:
+        return None
+    src = os.path.join(ROOT, "w4a4_post_quantized_b200", "csrc", kernel_file)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d["bytes_per_launch"] if d.get("source_sha") == h else None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                rows.append((float(f[0]), float(f[1]), f[3:7]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(wl, rows_per_step: int, seed: int = 0):
+    """Prepare (untimed) and return a closure that runs the oracle's hot path
+    (rotate, smooth, quantize, integer GEMM, dequantize) on `rows_per_step`
+    rows of the workload."""
+    import oracle
+    K, N = wl["K"], wl["N"]
+    M = wl["frames"] * synth.FRAME_TOKENS
+    X = synth.activations(M, K, seed=seed)
+    W = synth.weights(N, K, seed=seed + 1)
+    b = synth.bias(N, seed=seed + 2)
+    pw = oracle.prepare_weights(W, b, X[:synth.calibration_rows(M)])
+    rows = np.concatenate([synth.special_rows(min(M, rows_per_step)),
+                           np.arange(5, M, max(1, M // rows_per_step))])[:rows_per_step]
+    Xs = X[np.sort(rows)]
+    gelu = wl.get("gelu", False)
+
+    def run():
+        return oracle.linear(Xs, pw, gelu=gelu)[0]
+    return run, len(Xs), oracle.max_threads()
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    rows = args.cpu_rows
+    run, r, cores = cpu_oracle_sample(wl, rows)
+    K, N = wl["K"], wl["N"]
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    tops = 2.0 * r * N * K / dt / 1e12
+    sample = f"{r} of {wl['frames'] * synth.FRAME_TOKENS} token rows per step (special tokens included)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/int64",
+        "data": "synthetic", "tokens_per_s": r / dt,
+        "config": {"workload": wl["desc"], "M_sampled": r, "N": N, "K": K},
+        "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, wl, world, rank, local):
+    import torch
+    from w4a4_post_quantized_b200 import w4a4
+    K, N = wl["K"], wl["N"]
+    gelu = wl.get("gelu", False)
+    flags = w4a4.W4A4_FLAG_GELU if gelu else 0
+    M = wl["frames"] * synth.FRAME_TOKENS
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    # ------------------------------------------------------------ inputs (untimed)
+    seed = 1000 * rank
+    W = bf16(synth.weights(N, K, seed=seed + 1))
+    b = bf16(synth.bias(N, seed=seed + 2))
+    Xs = [bf16(synth.activations(M, K, seed=seed + 10 + i)) for i in range(NSETS)]
+    pw = w4a4.w4a4_prepare_weights(W, b, Xs[0][:synth.calibration_rows(M)])
+    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(NSETS)]
+    wsb = w4a4.w4a4_workspace_bytes(M, K)
+    WSs = [torch.empty(wsb, dtype=torch.uint8, device=dev) for _ in range(NSETS)]
+    st_off = ((M * K // 2 + 255) // 256) * 256
+    QX = [ws[:M * K // 2].view(M, K // 2) for ws in WSs]
+    ST = [ws[st_off:st_off + 4 * M].view(torch.float32) for ws in WSs]
+    torch.cuda.synchronize()
+
+    def step(i):
+        w4a4.w4a4_linear_fused(Xs[i % NSETS], pw, Y=Ys[i % NSETS], workspace=WSs[i % NSETS], flags=flags)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    w4a4.w4a4_clear_device_status()
+
+    # ---------------------------------------------------------------- timed region
+    # each step: quantize kernel [event] GEMM kernel [event]: the same two
+    # launches w4a4_linear_fused makes, with events between them so that each
+    # kernel's duration is measured inside the timed region
+    evq = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            j = i % NSETS
+            e0, e1, e2 = evq[i]
+            e0.record(stream)
+            w4a4.w4a4_quantize_act(Xs[j], pw.inv_smooth, flags, qx=QX[j], scale_tok=ST[j])
+            e1.record(stream)
+            w4a4.w4a4_linear(QX[j], ST[j], pw, Y=Ys[j])
+            e2.record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    status = w4a4.w4a4_get_device_status()
+    elapsed_ms = max_over_ranks(world, t0.elapsed_time(t1))
+    q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evq)
+    g_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evq)
+    ms_step = elapsed_ms / args.steps
+    ops = 2.0 * M * N * K
+    value = world * ops * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    # ------------------------------------------------------------- end to end
+    Xh = [torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    for x, src in zip(Xh, Xs):
+        x.copy_(src.cpu())
+    Yh = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    for i in range(2):
+        Xs[0].copy_(Xh[i], non_blocking=True)
+        step(0)
+        Yh.copy_(Ys[0], non_blocking=True)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a0.record(stream)
+    for i in range(e2e_steps):
+        Xs[0].copy_(Xh[i % 2], non_blocking=True)
+        step(0)
+        Yh.copy_(Ys[0], non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / e2e_steps
+    e2e_value = world * ops / (e2e_ms * 1e-3) / 1e12
+
+    # ------------------------------------------------------------- roofline
+    peaks = load_peaks()
+    int8_peak = peaks["bf16"] * INT8_PER_BF16
+    gemm_tops = ops / (g_ms * 1e-3) / 1e12
+    q_bytes = 2.0 * M * K + M * K / 2 + 4.0 * M
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    roofline = {"bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": gemm_tops,
+                "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
+                "traffic": profile_traffic("gemm.cu", f"gemm_{args.workload}"),
+                "peak_note": f"int8 = {INT8_PER_BF16:g} x {peaks['src']} bf16 burst {peaks['bf16']} TFLOP/s",
+                "ms_per_launch": g_ms, "algorithmic_ops_per_launch": ops}
+    roofline_q = {"bound": "hbm", "kernel": "quantize_rows_kernel", "achieved": q_gbs,
+                  "peak": peaks["hbm"], "unit": "GB/s", "frac": q_gbs / peaks["hbm"],
+                  "traffic": profile_traffic("quant.cu", f"quant_{args.workload}"),
+                  "ms_per_launch": q_ms, "algorithmic_bytes_per_launch": q_bytes}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s4xs4->s32 (bf16 in/out, fp32 transform)", "data": "synthetic",
+        "tokens_per_s": world * M * args.steps / (elapsed_ms * 1e-3),
+        "config": {"workload": wl["desc"], "M": M, "N": N, "K": K, "per_rank_batch": M,
+                   "parallelism": f"dp{world} (independent replicas)",
+                   "l2": f"inputs/outputs rotated over {NSETS} buffer sets (~{(2*M*K+2*M*N+M*K//2)*NSETS/1e6:.0f} MB > L2)"},
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_value, "unit": "TOPS", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
+                "api": "w4a4_linear_fused with pinned-host X/Y copies on the same stream"},
+        "gpu_launches": 2 * args.steps,
+        "roofline": roofline,
+        "roofline_quantize": roofline_q,
+        "device_status": status,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        run, r, cores = cpu_oracle_sample(wl, args.cpu_rows)
+        run()
+        t = time.perf_counter()
+        run()
+        dt = time.perf_counter() - t
+        line["cpu_baseline"] = {"value": 2.0 * r * N * K / dt / 1e12, "unit": "TOPS", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{r} of {M} token rows, one pass ({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c2_frame_qkv")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    wl = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, wl, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

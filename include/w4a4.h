@@ -1,0 +1,166 @@
+/*
+ * w4a4.h -- C ABI of libw4a4, the DSFQ W4A4 quantized linear layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * DSFQ = Dual-Smoothed Fine-Grained Quantization, the quantizer of QuantVGGT.
+ * Sources (page "十亿参数的三维重建模型，能塞进手机吗？", a translation of the
+ * QuantVGGT paper):
+ *   [PTQ]    section 训练后量化（PTQ）: symmetric N-bit quantizer,
+ *            q = clamp(round(x / delta), -2^(N-1), 2^(N-1) - 1); here N = 4.
+ *   [ROT]    section 预全局旋转（Pre-Global-Rotation）: Hadamard rotation of
+ *            activations and weights along the input features, H H^T = I.
+ *   [SMOOTH] section 后局部平滑（Post-Local-Smooth）: per-channel smoothing
+ *            factors computed in the rotated space, alpha = 0.5, applied
+ *            after the rotation and folded into the weights.
+ *   [GRAN]   section 细粒度量化粒度: read as one step per token for
+ *            activations and one step per output channel for weights.
+ *
+ * Per layer, with X [M, K] bf16 activations and W [N, K] bf16 weights:
+ *   offline : Wt = W H/sqrt(K); s_j = max|Xt_calib[:,j]|^a / max|Wt[:,j]|^(1-a);
+ *             W^ = Wt diag(s); qw[n,:] = int4(W^[n,:]), delta_ch[n] = max|W^[n,:]|/7
+ *   online  : X^ = (X H/sqrt(K)) diag(s)^-1; qx[m,:] = int4(X^[m,:]),
+ *             delta_tok[m] = max|X^[m,:]|/7;
+ *             Y[m,n] = bf16( (sum_k qx[m,k] qw[n,k]) * delta_tok[m] * delta_ch[n] + b[n] )
+ *   int4(v) = round-half-even(v / delta) with delta = max|v| / 7 (codes in [-7, 7];
+ *   an all-zero row has delta = 0 and zero codes).  H is the Sylvester
+ *   Hadamard matrix in natural order, K in {1024, 4096}.
+ *
+ * Conventions for every call:
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     allocates nothing and keeps no pointer after a call returns.
+ *   - Arrays are row-major and contiguous.  bf16 values are passed as their
+ *     raw 16-bit patterns (uint16_t).
+ *   - Packed int4 codes: two per byte, element 2i in the low nibble, element
+ *     2i+1 in the high nibble, each nibble the 4-bit two's complement code.
+ *   - Alignment: every array pointer and the workspace must be 16-byte
+ *     aligned (the kernels use 16-byte vector accesses and TMA).  Violations
+ *     return W4A4_ERR_ALIGN.
+ *   - Shapes: K must be 1024 or 4096 (W4A4_ERR_UNSUPPORTED otherwise); N must
+ *     be a positive multiple of 256 (W4A4_ERR_SHAPE); M >= 0, and M = 0 is a
+ *     no-op that returns W4A4_OK.  M must stay below 2^31.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns without synchronizing, except
+ *     w4a4_get_device_status.  Launch failures return W4A4_ERR_CUDA.
+ *   - Argument checks happen on the host before anything is enqueued; a call
+ *     that returns an error enqueued nothing.
+ *   - Kernels never trap.  Every wait inside a kernel is bounded; a wait that
+ *     runs out sets W4A4_DEV_TIMEOUT in the device status word (read it with
+ *     w4a4_get_device_status) and the kernel returns early, leaving its output
+ *     undefined.
+ *   - Calls on the same stream are ordered; the library holds no state
+ *     between calls except the device status word.
+ */
+#ifndef W4A4_H_
+#define W4A4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4A4_OK = 0,
+    W4A4_ERR_ARG = 1,          /* null pointer or invalid scalar argument */
+    W4A4_ERR_SHAPE = 2,        /* M, N or workspace size not accepted */
+    W4A4_ERR_ALIGN = 3,        /* pointer not aligned as required */
+    W4A4_ERR_UNSUPPORTED = 4,  /* K not in {1024, 4096}, or unknown flag */
+    W4A4_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed */
+    W4A4_ERR_TIMEOUT = 6       /* a kernel reported a bounded wait running out */
+} w4a4_status;
+
+/* Bits of the device status word (w4a4_get_device_status). */
+#define W4A4_DEV_TIMEOUT 0x1u
+
+/* Flags. */
+#define W4A4_FLAG_GELU  0x1u  /* quantize_act / linear_fused: apply exact-erf GELU
+                                 to X (rounded to bf16) before the rotation; the
+                                 input of an MLP's second linear */
+#define W4A4_FLAG_PLAIN 0x2u  /* no rotation and no smoothing: plain per-token /
+                                 per-channel int4 quantization (the baseline that
+                                 DSFQ is measured against); must match between
+                                 prepare_weights and the activation calls */
+
+/* Prepared weights of one linear layer.  The caller allocates every array
+ * (device memory) with the sizes given and keeps ownership. */
+typedef struct {
+    int32_t N;            /* output features, multiple of 256 */
+    int32_t K;            /* input features, 1024 or 4096 */
+    uint8_t *qw;          /* [N, K/2] packed int4 codes of W^ */
+    float *scale_ch;      /* [N] delta_ch */
+    float *bias;          /* [N] fp32 bias (zeros when the layer has none) */
+    float *smooth;        /* [K] s */
+    float *inv_smooth;    /* [K] 1/s (what the activation quantizer multiplies by) */
+    uint32_t flags;       /* W4A4_FLAG_PLAIN when prepared without DSFQ */
+} w4a4_weights_t;
+
+/* Bytes of workspace w4a4_linear_fused needs for M tokens of width K:
+ * the packed activation codes (M*K/2, rounded up to 256) followed by the
+ * per-token steps (4*M).  Returns 0 for an unsupported K. */
+size_t w4a4_workspace_bytes(int64_t M, int32_t K);
+
+/* Offline weight preparation [ROT][SMOOTH][PTQ][GRAN].
+ *   W       [N, K] bf16 weights; bias [N] bf16 or NULL;
+ *   X_calib [M_calib, K] bf16 calibration activations (M_calib >= 1), used
+ *           only for the per-channel activation maxima of the smoothing step;
+ *   alpha   smoothing exponent in [0, 1] (the page uses 0.5);
+ *   flags   0 or W4A4_FLAG_PLAIN (then s = 1 and no rotation; X_calib may be NULL);
+ *   out     caller-allocated arrays to fill; out->N and out->K must equal N
+ *           and K; out->flags is set to (flags & W4A4_FLAG_PLAIN).
+ * Rounding decisions are taken in binary32.  A channel whose activation or
+ * weight maximum is zero gets s_j = 1. */
+w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_t N, int32_t K,
+                                 const uint16_t *X_calib, int64_t M_calib, float alpha,
+                                 uint32_t flags, w4a4_weights_t *out, void *stream);
+
+/* Online activation quantizer [ROT][SMOOTH][PTQ][GRAN]: for each of the M
+ * rows of X [M, K] bf16: optional GELU (W4A4_FLAG_GELU), rotation X H/sqrt(K),
+ * multiplication by inv_smooth [K], per-token step delta = absmax/7 written to
+ * scale_tok [M] (fp32), codes round-half-even(x / delta) packed into qx
+ * [M, K/2].  With W4A4_FLAG_PLAIN the rotation and smoothing are skipped
+ * (inv_smooth may then be NULL).  Inputs must be finite. */
+w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const float *inv_smooth,
+                              uint8_t *qx, float *scale_tok, uint32_t flags, void *stream);
+
+/* Quantized linear from codes: Y [M, N] bf16 =
+ *   round-to-nearest-even( (qx qw^T)[m,n] * scale_tok[m] * w->scale_ch[n] + w->bias[n] ).
+ * The integer product is exact (int32 accumulation on the tensor cores); the
+ * epilogue is fp32. */
+w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
+                        const w4a4_weights_t *w, uint16_t *Y, void *stream);
+
+/* Quantized linear from bf16 activations: w4a4_quantize_act (with
+ * w->inv_smooth and the given flags) into `workspace`, then w4a4_linear.
+ * workspace must hold w4a4_workspace_bytes(M, w->K) bytes (workspace_bytes
+ * says how many it holds); its contents afterwards are the codes and steps. */
+w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t *w, uint16_t *Y,
+                              void *workspace, size_t workspace_bytes, uint32_t flags,
+                              void *stream);
+
+/* Integer product only: acc [M, N] int32 = qx [M, K/2] times qw [N, K/2]
+ * transposed, both packed int4.  Same tensor-core path as w4a4_linear, with
+ * the raw accumulators written out; used to check that the integer product is
+ * exact. */
+w4a4_status w4a4_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int32_t N, int32_t K,
+                          int32_t *acc, void *stream);
+
+/* Synchronizes `stream`, then copies the device status word (bits
+ * W4A4_DEV_*) of the current device into *status.  Returns W4A4_ERR_TIMEOUT
+ * when a bit is set, W4A4_OK otherwise. */
+w4a4_status w4a4_get_device_status(void *stream, uint32_t *status);
+
+/* Clears the device status word of the current device (enqueued on stream). */
+w4a4_status w4a4_clear_device_status(void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *w4a4_status_string(w4a4_status s);
+
+/* Library version string. */
+const char *w4a4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A4_H_ */

@@ -1,0 +1,58 @@
+"""Comparison rules shared by the GPU parity tests.
+
+Integer codes.  Both sides take the rounding decision in binary32 (the
+oracle's decision="f32" quantizer), but the CUDA path reaches its binary32
+values through an fp32 fast Walsh-Hadamard transform while the oracle rounds
+its exact fp64 values once.  Where the exact ratio value/step lies within the
+fp32 error bound of a rounding boundary (x.5), both codes are correct.  So a
+code may differ from the oracle's only
+  * by +-1,
+  * at an element whose fp64 ratio is within `tie_bound` of a half-integer,
+  * on at most 1e-4 of the elements (checked on the large cases).
+Everything else must be bit-exact.
+
+tie_bound: each rotated value is a +-sum of K inputs formed through log2(K)
+rounding levels, so its absolute error is at most log2(K) * u * sum_i |x_i| /
+sqrt(K) (u = 2^-24); the smoothing multiply, the reciprocal step and the
+absmax add a few relative u.  The bound below takes that, times the
+multiplier and 7/absmax, with a factor 4 of margin.
+"""
+import numpy as np
+
+U = 2.0 ** -24
+
+
+def tie_bound(x_in: np.ndarray, mult: np.ndarray, ratio: np.ndarray, amax: np.ndarray, K: int) -> np.ndarray:
+    """Per-row bound on |ratio_cuda - ratio_exact| (rows of x_in are the
+    transform's inputs, mult the per-channel multipliers)."""
+    l1 = np.sum(np.abs(x_in), axis=1)
+    e_val = np.log2(K) * U * l1 / np.sqrt(K) * np.max(np.abs(mult))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        e_ratio = np.where(amax > 0, 7.0 * e_val / amax, 0.0)
+    return 4.0 * (e_ratio + 8 * U * 7.0 * (1 + np.max(np.abs(ratio), axis=1) / 7.0))
+
+
+def compare_codes(got: np.ndarray, want: np.ndarray, ratio: np.ndarray, bound_row: np.ndarray,
+                  max_frac: float | None = 1e-4):
+    """got, want: int codes [rows, K]; ratio: fp64 value/step [rows, K];
+    bound_row: tie_bound per row.  Returns the number of flips."""
+    diff = got.astype(np.int32) - want.astype(np.int32)
+    bad = np.nonzero(diff)
+    n = len(bad[0])
+    if n:
+        assert np.all(np.abs(diff[bad]) == 1), f"code differs by more than 1: {np.unique(diff[bad])}"
+        r = ratio[bad]
+        dist = np.abs(np.abs(r - np.floor(r)) - 0.5)
+        allowed = bound_row[bad[0]]
+        assert np.all(dist <= allowed), (
+            f"{int(np.sum(dist > allowed))} of {n} flips are not at rounding ties "
+            f"(worst distance {dist.max():.3e}, bound {allowed.min():.3e})")
+    if max_frac is not None:
+        assert n <= max_frac * got.size, f"{n} flips > {max_frac} of {got.size}"
+    return n
+
+
+def rel_fro(got, want) -> float:
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))

@@ -1,0 +1,149 @@
+"""C-ABI checks that need no GPU: libw4a4.so loads, exports every function
+include/w4a4.h declares, and rejects bad arguments on the host (before any
+CUDA call) with the documented status codes."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a4.h")
+LIB = os.path.join(ROOT, "w4a4_post_quantized_b200", "libw4a4.so")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from w4a4_post_quantized_b200 import build
+        build.build()
+    return ctypes.CDLL(LIB)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["w4a4_prepare_weights", "w4a4_quantize_act", "w4a4_linear", "w4a4_linear_fused",
+              "w4a4_workspace_bytes", "w4a4_gemm_s32", "w4a4_get_device_status"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in w4a4.h but not exported by libw4a4.so"
+
+
+def test_status_codes_match_binding():
+    text = open(HEADER).read()
+    codes = dict((k, int(v)) for k, v in re.findall(r"(W4A4_(?:OK|ERR_[A-Z]+))\s*=\s*(\d+)", text))
+    assert codes == {"W4A4_OK": 0, "W4A4_ERR_ARG": 1, "W4A4_ERR_SHAPE": 2, "W4A4_ERR_ALIGN": 3,
+                     "W4A4_ERR_UNSUPPORTED": 4, "W4A4_ERR_CUDA": 5, "W4A4_ERR_TIMEOUT": 6}
+
+
+class WeightsT(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("qw", ctypes.c_void_p),
+                ("scale_ch", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("smooth", ctypes.c_void_p), ("inv_smooth", ctypes.c_void_p),
+                ("flags", ctypes.c_uint32)]
+
+
+A = 0x10000  # fake, 16-byte aligned device addresses: never dereferenced on the host
+
+
+def _setup(lib):
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    lib.w4a4_workspace_bytes.restype = ctypes.c_size_t
+    lib.w4a4_workspace_bytes.argtypes = [i64, i32]
+    lib.w4a4_quantize_act.argtypes = [vp, i64, i32, vp, vp, vp, ctypes.c_uint32, vp]
+    lib.w4a4_linear.argtypes = [vp, vp, i64, ctypes.POINTER(WeightsT), vp, vp]
+    lib.w4a4_linear_fused.argtypes = [vp, i64, ctypes.POINTER(WeightsT), vp, vp, ctypes.c_size_t,
+                                      ctypes.c_uint32, vp]
+    lib.w4a4_prepare_weights.argtypes = [vp, vp, i32, i32, vp, i64, ctypes.c_float, ctypes.c_uint32,
+                                         ctypes.POINTER(WeightsT), vp]
+    lib.w4a4_gemm_s32.argtypes = [vp, vp, i64, i32, i32, vp, vp]
+    lib.w4a4_status_string.restype = ctypes.c_char_p
+    lib.w4a4_version.restype = ctypes.c_char_p
+
+
+def _weights(N=1024, K=1024, base=A, flags=0):
+    return WeightsT(N, K, base, base + 0x1000, base + 0x2000, base + 0x3000, base + 0x4000, flags)
+
+
+def test_workspace_bytes(lib):
+    _setup(lib)
+    assert lib.w4a4_workspace_bytes(10992, 1024) == ((10992 * 512 + 255) // 256) * 256 + 4 * 10992
+    assert lib.w4a4_workspace_bytes(3, 4096) == 6144 + 12
+    assert lib.w4a4_workspace_bytes(0, 1024) == 0
+    assert lib.w4a4_workspace_bytes(10, 1000) == 0
+    assert lib.w4a4_workspace_bytes(-1, 1024) == 0
+
+
+def test_quantize_act_argument_checks(lib):
+    _setup(lib)
+    q = lib.w4a4_quantize_act
+    assert q(A, 10, 1000, A, A, A, 0, None) == 4                 # K unsupported
+    assert q(A, 10, 1024, A, A, A, 0x80, None) == 4              # unknown flag
+    assert q(None, 10, 1024, A, A, A, 0, None) == 1              # null X
+    assert q(A, 10, 1024, None, A, A, 0, None) == 1              # null inv_smooth (DSFQ)
+    assert q(A + 8, 10, 1024, A, A, A, 0, None) == 3             # misaligned X
+    assert q(A, -1, 1024, A, A, A, 0, None) == 2                 # negative M
+    assert q(A, 1 << 31, 1024, A, A, A, 0, None) == 2            # M too large
+    assert q(A, 0, 1024, A, A, A, 0, None) == 0                  # empty input: no-op
+    assert q(A, 0, 4096, None, A, A, 2, None) == 0               # plain: inv_smooth may be null
+
+
+def test_linear_argument_checks(lib):
+    _setup(lib)
+    w = _weights()
+    L = lib.w4a4_linear
+    assert L(A, A, 10, None, A, None) == 1
+    assert L(A, A, 10, ctypes.byref(_weights(N=1000)), A, None) == 2
+    assert L(A, A, 10, ctypes.byref(_weights(K=2048)), A, None) == 4
+    assert L(A, A, 10, ctypes.byref(_weights(base=A + 4)), A, None) == 3
+    assert L(A, A, 10, ctypes.byref(_weights(flags=0x10)), A, None) == 4
+    assert L(None, A, 10, ctypes.byref(w), A, None) == 1
+    assert L(A, A, 10, ctypes.byref(w), A + 2, None) == 3
+    assert L(A, A, 0, ctypes.byref(w), A, None) == 0
+
+
+def test_linear_fused_argument_checks(lib):
+    _setup(lib)
+    w = _weights()
+    F = lib.w4a4_linear_fused
+    need = lib.w4a4_workspace_bytes(100, 1024)
+    assert F(A, 100, ctypes.byref(w), A, A, need - 1, 0, None) == 2     # workspace too small
+    assert F(A, 100, ctypes.byref(w), A, A, need, 2, None) == 1         # plain flag vs DSFQ weights
+    assert F(A, 100, ctypes.byref(w), A, None, need, 0, None) == 1
+    assert F(A, 100, ctypes.byref(w), A, A + 1, need, 0, None) == 3
+    assert F(A, 0, ctypes.byref(w), A, A, 0, 0, None) == 0
+
+
+def test_prepare_and_gemm_argument_checks(lib):
+    _setup(lib)
+    P = lib.w4a4_prepare_weights
+    w = _weights()
+    assert P(A, None, 1024, 1024, A, 10, 0.5, 0, ctypes.byref(_weights(N=512)), None) == 2
+    assert P(A, None, 1024, 1024, None, 10, 0.5, 0, ctypes.byref(w), None) == 1
+    assert P(A, None, 1024, 1024, A, 0, 0.5, 0, ctypes.byref(w), None) == 1
+    assert P(A, None, 1024, 1024, A, 10, 1.5, 0, ctypes.byref(w), None) == 1
+    assert P(A, None, 1024, 1024, A, 10, float("nan"), 0, ctypes.byref(w), None) == 1
+    assert P(A, None, 1024, 1000, A, 10, 0.5, 0, ctypes.byref(w), None) == 4
+    assert P(A, None, 100, 1024, A, 10, 0.5, 0, ctypes.byref(w), None) == 2
+    assert P(A + 2, None, 1024, 1024, A, 10, 0.5, 0, ctypes.byref(w), None) == 3
+    G = lib.w4a4_gemm_s32
+    assert G(A, A, 10, 1024, 1024, None, None) == 1
+    assert G(A, A, 10, 1000, 1024, A, None) == 2
+    assert G(A, A, 10, 1024, 64, A, None) == 4
+    assert G(A, A, 0, 1024, 1024, A, None) == 0
+
+
+def test_status_strings(lib):
+    _setup(lib)
+    assert lib.w4a4_status_string(0) == b"ok"
+    assert lib.w4a4_status_string(6) == b"device wait timed out"
+    assert b"sm_100a" in lib.w4a4_version()

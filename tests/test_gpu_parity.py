@@ -1,0 +1,231 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bars (the quantized linear's numerical contract):
+  * integer accumulators: bit-exact against the oracle's int64 GEMM on
+    identical seeded codes;
+  * activation / weight codes: bit-exact except +-1 flips at rounding ties
+    within the fp32 bound of tests/parity.py, at most 1e-4 of the elements;
+    per-token / per-channel steps within 1e-5 relative;
+  * end to end: relative Frobenius error of Y against the oracle's fp64 Y at
+    most 2e-3 (bf16 output rounding alone contributes about 1e-3); the
+    epilogue on identical codes matches the oracle's dequantization rounded
+    to bf16 to within one bf16 step everywhere.
+Inputs are seeded synthetic VGGT-shaped tensors (w4a4_post_quantized_b200.synth).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w4a4_post_quantized_b200 import synth
+from parity import compare_codes, rel_fro, tie_bound
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def w4():
+    from w4a4_post_quantized_b200 import w4a4
+    return w4a4
+
+
+def dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.view(dtype)
+    return t.cuda()
+
+
+def bf16_dev(bits):
+    return dev(bits.view(np.int16), torch.int16).view(torch.bfloat16)
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+def y_to_f64(Y):
+    return synth.bf16_bits_to_f32(host(Y.view(torch.int16)).view(np.uint16)).astype(np.float64)
+
+
+# ------------------------------------------------------------------ integer GEMM
+@pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (128, 256, 1024), (300, 512, 1024),
+                                   (1374, 1024, 1024), (257, 256, 4096), (640, 1024, 4096)])
+def test_gemm_s32_bit_exact(w4, M, N, K):
+    A = synth.random_packed_codes(M, K, seed=M + 7)
+    B = synth.random_packed_codes(N, K, seed=N + 11)
+    acc = host(w4.w4a4_gemm_s32(dev(A), dev(B)))
+    torch.cuda.synchronize()
+    want = oracle.int_gemm(oracle.unpack_int4(A, K), oracle.unpack_int4(B, K))
+    assert np.array_equal(acc.astype(np.int64), want)
+
+
+def test_gemm_s32_extreme_codes(w4):
+    K = 4096
+    A = np.full((130, K // 2), 0x88, np.uint8)    # every code -8
+    B = np.full((256, K // 2), 0x88, np.uint8)
+    acc = host(w4.w4a4_gemm_s32(dev(A), dev(B)))
+    assert np.all(acc == 64 * K)
+    B2 = np.full((256, K // 2), 0x77, np.uint8)   # every code 7
+    acc = host(w4.w4a4_gemm_s32(dev(A), dev(B2)))
+    assert np.all(acc == -56 * K)
+
+
+# -------------------------------------------------------------- activation quantizer
+def _check_quant(w4, X, K, inv_s32, flags, max_frac):
+    M = X.shape[0]
+    qx, st = w4.w4a4_quantize_act(bf16_dev(X), dev(inv_s32) if inv_s32 is not None else None, flags)
+    qx, st = host(qx), host(st)
+    plain = bool(flags & w4.W4A4_FLAG_PLAIN)
+    gelu = bool(flags & w4.W4A4_FLAG_GELU)
+    s = np.ones(K) if inv_s32 is None else 1.0 / inv_s32.astype(np.float64)
+    hat = oracle.act_hat(X, s, gelu=gelu, plain=plain)
+    want_q, want_d = oracle.quantize_rows(hat, 4, "f32")
+    np.testing.assert_allclose(st, want_d, rtol=1e-5, atol=0)
+    xin = oracle.bf16_to_f64(oracle.gelu_bf16(X) if gelu else X)
+    amax = np.max(np.abs(hat), axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = np.where(amax[:, None] > 0, hat * 7.0 / amax[:, None], 0.0)
+    bound = tie_bound(xin, 1.0 / s, ratio, amax, K)
+    if gelu:  # GELU in fp32 may land one bf16 step away from the fp64 GELU
+        bound = bound + 4.0 * 2.0 ** -8 * np.max(np.abs(xin), axis=1) * np.max(1.0 / s) / np.sqrt(K) * 7.0 / np.maximum(amax, 1e-300)
+    got = oracle.unpack_int4(qx, K)
+    return compare_codes(got, want_q, ratio, bound, max_frac)
+
+
+@pytest.mark.parametrize("K", [1024, 4096])
+@pytest.mark.parametrize("M", [1, 37, 1374])
+def test_quantize_act_parity(w4, M, K):
+    X = synth.activations(M, K, seed=100 + M)
+    inv_s = synth.random_scales(K, seed=K, lo=0.25, hi=4.0)
+    _check_quant(w4, X, K, inv_s, 0, None)
+
+
+def test_quantize_act_parity_frame_batch(w4):
+    M, K = 4 * 1374, 1024
+    X = synth.activations(M, K, seed=5)
+    inv_s = synth.random_scales(K, seed=6, lo=0.25, hi=4.0)
+    _check_quant(w4, X, K, inv_s, 0, 1e-4)
+
+
+@pytest.mark.parametrize("K", [1024, 4096])
+def test_quantize_act_plain(w4, K):
+    X = synth.activations(300, K, seed=9)
+    _check_quant(w4, X, K, None, 2, 1e-4)
+
+
+def test_quantize_act_gelu(w4):
+    K = 4096
+    X = synth.to_bf16_bits(np.random.default_rng(3).standard_normal((700, K)).astype(np.float32) * 2)
+    inv_s = synth.random_scales(K, seed=12, lo=0.5, hi=2.0)
+    _check_quant(w4, X, K, inv_s, 1, 2e-4)
+
+
+def test_quantize_act_zero_rows(w4):
+    K = 1024
+    X = synth.activations(20, K, seed=4)
+    X[[0, 7, 19]] = 0
+    qx, st = w4.w4a4_quantize_act(bf16_dev(X), dev(np.ones(K, np.float32)))
+    qx, st = host(qx), host(st)
+    assert np.all(st[[0, 7, 19]] == 0) and np.all(qx[[0, 7, 19]] == 0)
+    assert np.all(st[[1, 2, 18]] > 0)
+
+
+# ------------------------------------------------------------------ weight preparation
+@pytest.mark.parametrize("N,K", [(256, 1024), (1024, 4096)])
+def test_prepare_weights_parity(w4, N, K):
+    W = synth.weights(N, K, seed=N)
+    b = synth.bias(N, seed=N + 1)
+    Xc = synth.activations(1374, K, seed=K + 2)
+    pw = w4.w4a4_prepare_weights(bf16_dev(W), bf16_dev(b), bf16_dev(Xc))
+    ow = oracle.prepare_weights(W, b, Xc)
+    np.testing.assert_allclose(host(pw.smooth), ow.s, rtol=2e-6)
+    np.testing.assert_allclose(host(pw.inv_smooth), 1.0 / ow.s, rtol=2e-6)
+    np.testing.assert_allclose(host(pw.bias), ow.bias, rtol=0, atol=0)
+    # codes: the oracle's binary32 decision on the GPU's own (binary32) s
+    s32 = host(pw.smooth).astype(np.float64)
+    hat = ow.Wt * s32[None, :]
+    want_q, want_d = oracle.quantize_rows(hat, 4, "f32")
+    np.testing.assert_allclose(host(pw.scale_ch), want_d, rtol=1e-5)
+    amax = np.max(np.abs(hat), axis=1)
+    ratio = hat * 7.0 / amax[:, None]
+    bound = tie_bound(oracle.bf16_to_f64(W), s32, ratio, amax, K)
+    compare_codes(oracle.unpack_int4(host(pw.qw), K), want_q, ratio, bound, 2e-4)
+
+
+# -------------------------------------------------------------------- epilogue
+@pytest.mark.parametrize("M,N,K", [(300, 512, 1024), (1374, 1024, 4096)])
+def test_linear_epilogue_on_identical_codes(w4, M, N, K):
+    A = synth.random_packed_codes(M, K, seed=1)
+    B = synth.random_packed_codes(N, K, seed=2)
+    st = synth.random_scales(M, seed=3, lo=1e-3, hi=1e-1)
+    sc = synth.random_scales(N, seed=4, lo=1e-3, hi=1e-2)
+    bias = synth.random_scales(N, seed=5, lo=-0.5, hi=0.5)
+    pw = w4.PreparedWeights(N, K)
+    pw.qw.copy_(dev(B))
+    pw.scale_ch.copy_(dev(sc))
+    pw.bias.copy_(dev(bias))
+    Y = w4.w4a4_linear(dev(A), dev(st), pw)
+    got = y_to_f64(Y)
+    acc = oracle.int_gemm(oracle.unpack_int4(A, K), oracle.unpack_int4(B, K))
+    want = oracle.dequant(acc, st.astype(np.float64), sc.astype(np.float64), bias.astype(np.float64))
+    want_bf = oracle.bf16_to_f64(oracle.f64_to_bf16(want))
+    ulp = np.abs(want_bf) * 2.0 ** -7
+    assert np.all(np.abs(got - want_bf) <= ulp + 1e-30)
+    assert np.mean(got == want_bf) > 0.999
+
+
+# -------------------------------------------------------------------- end to end
+def _linear_case(w4, M, N, K, seed, gelu=False, plain=False, sample=None):
+    X = synth.activations(M, K, seed=seed)
+    W = synth.weights(N, K, seed=seed + 1)
+    b = synth.bias(N, seed=seed + 2)
+    Xc = X[:synth.calibration_rows(M)]
+    flags = (w4.W4A4_FLAG_GELU if gelu else 0) | (w4.W4A4_FLAG_PLAIN if plain else 0)
+    pw = w4.w4a4_prepare_weights(bf16_dev(W), bf16_dev(b), bf16_dev(Xc),
+                                 flags=w4.W4A4_FLAG_PLAIN if plain else 0)
+    Y = y_to_f64(w4.w4a4_linear_fused(bf16_dev(X), pw, flags=flags))
+    assert w4.w4a4_get_device_status() == 0
+    ow = oracle.prepare_weights(W, b, Xc, plain=plain)
+    rows = np.arange(M) if sample is None else sample
+    Yo = oracle.linear(X[rows], ow, gelu=gelu, plain=plain)[0]
+    err = rel_fro(Y[rows], Yo)
+    ref = oracle.reference_fp(X[rows], W, b, gelu=gelu)
+    return err, oracle.sqnr_db(ref, Y[rows]), oracle.sqnr_db(ref, Yo)
+
+
+@pytest.mark.parametrize("M,N,K", [(1374, 1024, 1024), (1, 256, 1024), (200, 256, 4096),
+                                   (1500, 3072, 1024)])
+def test_linear_fused_end_to_end(w4, M, N, K):
+    err, sq_gpu, sq_or = _linear_case(w4, M, N, K, seed=M + N)
+    assert err <= 2e-3, err
+    assert abs(sq_gpu - sq_or) < 0.1
+
+
+def test_linear_fused_gelu_and_plain(w4):
+    err, _, _ = _linear_case(w4, 640, 1024, 4096, seed=77, gelu=True)
+    assert err <= 2e-3, err
+    err, _, _ = _linear_case(w4, 640, 1024, 1024, seed=78, plain=True)
+    assert err <= 2e-3, err
+
+
+def test_linear_fused_full_size_sampled(w4):
+    """Frame-attention QKV at 8 frames (10992 x 1024 -> 3072), the benchmark's
+    launch configuration; the oracle checks sampled rows, special tokens included."""
+    M = 8 * synth.FRAME_TOKENS
+    rows = np.unique(np.concatenate([synth.special_rows(M), np.arange(17, M, 211)]))
+    err, sq_gpu, sq_or = _linear_case(w4, M, 3072, 1024, seed=2, sample=rows)
+    assert err <= 2e-3, err
+
+
+def test_empty_input_is_a_no_op(w4):
+    pw = w4.PreparedWeights(256, 1024)
+    X = torch.empty((0, 1024), dtype=torch.bfloat16, device="cuda")
+    Y = w4.w4a4_linear_fused(X, pw)
+    assert Y.shape == (0, 256)
+    torch.cuda.synchronize()
+
+
+def test_device_status_clear(w4):
+    w4.w4a4_clear_device_status()
+    assert w4.w4a4_get_device_status() == 0

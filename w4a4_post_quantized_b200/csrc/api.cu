@@ -1,0 +1,183 @@
+// api.cu -- the C ABI of libw4a4 (include/w4a4.h): argument checks on the
+// host, then kernel launches on the caller's stream.  No allocation, no
+// synchronization (except w4a4_get_device_status), no exceptions.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "kernels.h"
+#include "w4a4.h"
+
+namespace {
+
+constexpr uint32_t kKnownFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool k_ok(int32_t K) { return K == 1024 || K == 4096; }
+bool n_ok(int32_t N) { return N > 0 && N % 256 == 0; }
+bool m_ok(int64_t M) { return M >= 0 && M < (int64_t(1) << 31); }
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+w4a4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA; }
+
+w4a4_status check_weights(const w4a4_weights_t *w) {
+  if (!w) return W4A4_ERR_ARG;
+  if (!k_ok(w->K)) return W4A4_ERR_UNSUPPORTED;
+  if (!n_ok(w->N)) return W4A4_ERR_SHAPE;
+  if (!w->qw || !w->scale_ch || !w->bias || !w->smooth || !w->inv_smooth) return W4A4_ERR_ARG;
+  if (!aligned16(w->qw) || !aligned16(w->scale_ch) || !aligned16(w->bias) || !aligned16(w->smooth) ||
+      !aligned16(w->inv_smooth))
+    return W4A4_ERR_ALIGN;
+  if (w->flags & ~W4A4_FLAG_PLAIN) return W4A4_ERR_UNSUPPORTED;
+  return W4A4_OK;
+}
+
+w4a4_status check_act(const void *X, int64_t M, int32_t K, const float *inv_smooth, const void *qx,
+                      const float *scale_tok, uint32_t flags) {
+  if (flags & ~kKnownFlags) return W4A4_ERR_UNSUPPORTED;
+  if (!k_ok(K)) return W4A4_ERR_UNSUPPORTED;
+  if (!m_ok(M)) return W4A4_ERR_SHAPE;
+  if (!X || !qx || !scale_tok) return W4A4_ERR_ARG;
+  if (!(flags & W4A4_FLAG_PLAIN) && !inv_smooth) return W4A4_ERR_ARG;
+  if (!aligned16(X) || !aligned16(qx) || !aligned16(scale_tok) ||
+      (inv_smooth && !aligned16(inv_smooth)))
+    return W4A4_ERR_ALIGN;
+  return W4A4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t w4a4_workspace_bytes(int64_t M, int32_t K) {
+  if (!k_ok(K) || !m_ok(M)) return 0;
+  return round256(static_cast<size_t>(M) * (K / 2)) + sizeof(float) * static_cast<size_t>(M);
+}
+
+w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_t N, int32_t K,
+                                 const uint16_t *X_calib, int64_t M_calib, float alpha,
+                                 uint32_t flags, w4a4_weights_t *out, void *stream) {
+  if (flags & ~W4A4_FLAG_PLAIN) return W4A4_ERR_UNSUPPORTED;
+  if (!k_ok(K)) return W4A4_ERR_UNSUPPORTED;
+  if (!n_ok(N)) return W4A4_ERR_SHAPE;
+  if (!out || !W) return W4A4_ERR_ARG;
+  if (out->N != N || out->K != K) return W4A4_ERR_SHAPE;
+  const bool plain = (flags & W4A4_FLAG_PLAIN) != 0;
+  if (!plain) {
+    if (!X_calib || M_calib < 1) return W4A4_ERR_ARG;
+    if (!m_ok(M_calib)) return W4A4_ERR_SHAPE;
+    if (!(alpha >= 0.0f && alpha <= 1.0f)) return W4A4_ERR_ARG;
+    if (!aligned16(X_calib)) return W4A4_ERR_ALIGN;
+  }
+  if (!out->qw || !out->scale_ch || !out->bias || !out->smooth || !out->inv_smooth)
+    return W4A4_ERR_ARG;
+  if (!aligned16(W) || (bias && !aligned16(bias)) || !aligned16(out->qw) ||
+      !aligned16(out->scale_ch) || !aligned16(out->bias) || !aligned16(out->smooth) ||
+      !aligned16(out->inv_smooth))
+    return W4A4_ERR_ALIGN;
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e;
+  if (plain) {
+    if ((e = w4a4::launch_fill(out->smooth, K, 1.0f, st)) != cudaSuccess) return cuda_status(e);
+    if ((e = w4a4::launch_fill(out->inv_smooth, K, 1.0f, st)) != cudaSuccess) return cuda_status(e);
+    e = w4a4::launch_quantize_rows(W, N, K, nullptr, out->qw, out->scale_ch, false, false, st);
+  } else {
+    // column maxima of the rotated calibration activations -> out->smooth,
+    // of the rotated weights -> out->inv_smooth; then s and 1/s in place
+    if ((e = w4a4::launch_colmax(X_calib, M_calib, K, out->smooth, st)) != cudaSuccess)
+      return cuda_status(e);
+    if ((e = w4a4::launch_colmax(W, N, K, out->inv_smooth, st)) != cudaSuccess) return cuda_status(e);
+    if ((e = w4a4::launch_smooth_factors(out->smooth, out->inv_smooth, K, alpha, st)) != cudaSuccess)
+      return cuda_status(e);
+    e = w4a4::launch_quantize_rows(W, N, K, out->smooth, out->qw, out->scale_ch, true, false, st);
+  }
+  if (e != cudaSuccess) return cuda_status(e);
+  if ((e = w4a4::launch_bias_to_f32(bias, out->bias, N, st)) != cudaSuccess) return cuda_status(e);
+  out->flags = flags & W4A4_FLAG_PLAIN;
+  return W4A4_OK;
+}
+
+w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const float *inv_smooth,
+                              uint8_t *qx, float *scale_tok, uint32_t flags, void *stream) {
+  w4a4_status s = check_act(X, M, K, inv_smooth, qx, scale_tok, flags);
+  if (s != W4A4_OK) return s;
+  return cuda_status(w4a4::launch_quantize_rows(X, M, K, inv_smooth, qx, scale_tok,
+                                                !(flags & W4A4_FLAG_PLAIN),
+                                                (flags & W4A4_FLAG_GELU) != 0, as_stream(stream)));
+}
+
+w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
+                        const w4a4_weights_t *w, uint16_t *Y, void *stream) {
+  w4a4_status s = check_weights(w);
+  if (s != W4A4_OK) return s;
+  if (!m_ok(M)) return W4A4_ERR_SHAPE;
+  if (!qx || !scale_tok || !Y) return W4A4_ERR_ARG;
+  if (!aligned16(qx) || !aligned16(scale_tok) || !aligned16(Y)) return W4A4_ERR_ALIGN;
+  w4a4::GemmArgs a{qx, w->qw, scale_tok, w->scale_ch, w->bias, Y, nullptr, M, w->N, w->K};
+  return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
+}
+
+w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t *w, uint16_t *Y,
+                              void *workspace, size_t workspace_bytes, uint32_t flags,
+                              void *stream) {
+  w4a4_status s = check_weights(w);
+  if (s != W4A4_OK) return s;
+  if (flags & ~kKnownFlags) return W4A4_ERR_UNSUPPORTED;
+  if ((flags & W4A4_FLAG_PLAIN) != (w->flags & W4A4_FLAG_PLAIN)) return W4A4_ERR_ARG;
+  if (!m_ok(M)) return W4A4_ERR_SHAPE;
+  if (!X || !Y || !workspace) return W4A4_ERR_ARG;
+  if (workspace_bytes < w4a4_workspace_bytes(M, w->K)) return W4A4_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(workspace)) return W4A4_ERR_ALIGN;
+  if (M == 0) return W4A4_OK;
+  uint8_t *qx = static_cast<uint8_t *>(workspace);
+  float *st = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (w->K / 2)));
+  cudaStream_t cs = as_stream(stream);
+  cudaError_t e = w4a4::launch_quantize_rows(X, M, w->K, w->inv_smooth, qx, st,
+                                             !(flags & W4A4_FLAG_PLAIN),
+                                             (flags & W4A4_FLAG_GELU) != 0, cs);
+  if (e != cudaSuccess) return cuda_status(e);
+  w4a4::GemmArgs a{qx, w->qw, st, w->scale_ch, w->bias, Y, nullptr, M, w->N, w->K};
+  return cuda_status(w4a4::launch_gemm(a, cs));
+}
+
+w4a4_status w4a4_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int32_t N, int32_t K,
+                          int32_t *acc, void *stream) {
+  if (!k_ok(K)) return W4A4_ERR_UNSUPPORTED;
+  if (!n_ok(N) || !m_ok(M)) return W4A4_ERR_SHAPE;
+  if (!qx || !qw || !acc) return W4A4_ERR_ARG;
+  if (!aligned16(qx) || !aligned16(qw) || !aligned16(acc)) return W4A4_ERR_ALIGN;
+  w4a4::GemmArgs a{qx, qw, nullptr, nullptr, nullptr, nullptr, acc, M, N, K};
+  return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
+}
+
+w4a4_status w4a4_get_device_status(void *stream, uint32_t *status) {
+  if (!status) return W4A4_ERR_ARG;
+  unsigned int v = 0;
+  cudaError_t e = w4a4::read_status(&v, as_stream(stream));
+  if (e != cudaSuccess) return W4A4_ERR_CUDA;
+  *status = v;
+  return v ? W4A4_ERR_TIMEOUT : W4A4_OK;
+}
+
+w4a4_status w4a4_clear_device_status(void *stream) {
+  return cuda_status(w4a4::clear_status(as_stream(stream)));
+}
+
+const char *w4a4_status_string(w4a4_status s) {
+  switch (s) {
+    case W4A4_OK: return "ok";
+    case W4A4_ERR_ARG: return "invalid argument";
+    case W4A4_ERR_SHAPE: return "unsupported shape or workspace size";
+    case W4A4_ERR_ALIGN: return "misaligned pointer";
+    case W4A4_ERR_UNSUPPORTED: return "unsupported K or flag";
+    case W4A4_ERR_CUDA: return "CUDA error";
+    case W4A4_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char *w4a4_version(void) { return "libw4a4 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// kernels.h -- internal launchers shared by the C-ABI layer (api.cu) and the
+// kernel translation units.  Not part of the public interface.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace w4a4 {
+
+int device_sm_count();
+
+// quant.cu
+cudaError_t launch_quantize_rows(const uint16_t *X, int64_t M, int K, const float *mult,
+                                 uint8_t *q, float *scale, bool rot, bool gelu, cudaStream_t st);
+cudaError_t launch_colmax(const uint16_t *X, int64_t M, int K, float *colmax, cudaStream_t st);
+cudaError_t launch_smooth_factors(float *s_io, float *inv_io, int K, double alpha, cudaStream_t st);
+cudaError_t launch_bias_to_f32(const uint16_t *b, float *out, int n, cudaStream_t st);
+cudaError_t launch_fill(float *out, int n, float v, cudaStream_t st);
+
+// gemm.cu
+struct GemmArgs {
+  const uint8_t *qx;        // [M, K/2] packed int4
+  const uint8_t *qw;        // [N, K/2] packed int4
+  const float *scale_tok;   // [M]
+  const float *scale_ch;    // [N]
+  const float *bias;        // [N]
+  uint16_t *y;              // [M, N] bf16 (when acc == nullptr)
+  int32_t *acc;             // [M, N] int32 accumulators instead of y (test path)
+  int64_t M;
+  int N, K;
+};
+cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
+
+// status word
+cudaError_t read_status(unsigned int *out, cudaStream_t st);
+cudaError_t clear_status(cudaStream_t st);
+
+}  // namespace w4a4

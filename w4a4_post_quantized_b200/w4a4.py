@@ -1,0 +1,171 @@
+"""ctypes binding of libw4a4 (include/w4a4.h) for torch tensors.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Importing this module raises ImportError when libw4a4.so has not
+been built (``python -m w4a4_post_quantized_b200.build``); there is no
+fallback.
+
+The functions carry the C names.  Tensors must be contiguous CUDA tensors;
+bf16 data is passed as torch.bfloat16, packed int4 codes as torch.uint8.
+Calls are asynchronous on the given stream (default: torch's current stream).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw4a4.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m w4a4_post_quantized_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+W4A4_OK, W4A4_ERR_ARG, W4A4_ERR_SHAPE, W4A4_ERR_ALIGN, W4A4_ERR_UNSUPPORTED, W4A4_ERR_CUDA, \
+    W4A4_ERR_TIMEOUT = range(7)
+W4A4_DEV_TIMEOUT = 0x1
+W4A4_FLAG_GELU = 0x1
+W4A4_FLAG_PLAIN = 0x2
+
+_vp, _i32, _i64, _u32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
+                                    ctypes.c_float, ctypes.c_size_t)
+
+
+class W4A4WeightsT(ctypes.Structure):
+    _fields_ = [("N", _i32), ("K", _i32), ("qw", _vp), ("scale_ch", _vp), ("bias", _vp),
+                ("smooth", _vp), ("inv_smooth", _vp), ("flags", _u32)]
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_workspace_bytes = _sig("w4a4_workspace_bytes", _sz, [_i64, _i32])
+_prepare = _sig("w4a4_prepare_weights", ctypes.c_int,
+                [_vp, _vp, _i32, _i32, _vp, _i64, _f32, _u32, ctypes.POINTER(W4A4WeightsT), _vp])
+_quantize = _sig("w4a4_quantize_act", ctypes.c_int, [_vp, _i64, _i32, _vp, _vp, _vp, _u32, _vp])
+_linear = _sig("w4a4_linear", ctypes.c_int, [_vp, _vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp])
+_fused = _sig("w4a4_linear_fused", ctypes.c_int,
+              [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp, _sz, _u32, _vp])
+_gemm_s32 = _sig("w4a4_gemm_s32", ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _vp, _vp])
+_get_status = _sig("w4a4_get_device_status", ctypes.c_int, [_vp, ctypes.POINTER(_u32)])
+_clear_status = _sig("w4a4_clear_device_status", ctypes.c_int, [_vp])
+_status_string = _sig("w4a4_status_string", ctypes.c_char_p, [ctypes.c_int])
+_version = _sig("w4a4_version", ctypes.c_char_p, [])
+
+
+class W4A4Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_status_string(code).decode()} (status {code})")
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != W4A4_OK:
+        raise W4A4Error(rc, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libw4a4 must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def version() -> str:
+    return _version().decode()
+
+
+def w4a4_workspace_bytes(M: int, K: int) -> int:
+    return int(_workspace_bytes(M, K))
+
+
+class PreparedWeights:
+    """Device arrays of one prepared layer (owned by torch) and the C struct
+    that points at them."""
+
+    def __init__(self, N: int, K: int, device="cuda"):
+        self.N, self.K = N, K
+        self.qw = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+        self.scale_ch = torch.empty(N, dtype=torch.float32, device=device)
+        self.bias = torch.empty(N, dtype=torch.float32, device=device)
+        self.smooth = torch.empty(K, dtype=torch.float32, device=device)
+        self.inv_smooth = torch.empty(K, dtype=torch.float32, device=device)
+        self.struct = W4A4WeightsT(N, K, self.qw.data_ptr(), self.scale_ch.data_ptr(),
+                                   self.bias.data_ptr(), self.smooth.data_ptr(),
+                                   self.inv_smooth.data_ptr(), 0)
+
+    @property
+    def flags(self) -> int:
+        return int(self.struct.flags)
+
+
+def w4a4_prepare_weights(W: torch.Tensor, bias, X_calib, alpha: float = 0.5, flags: int = 0,
+                         out: PreparedWeights | None = None, stream=None) -> PreparedWeights:
+    N, K = W.shape
+    out = out or PreparedWeights(N, K, W.device)
+    mc = 0 if X_calib is None else X_calib.shape[0]
+    _check(_prepare(_ptr(W), _ptr(bias), N, K, _ptr(X_calib), mc, alpha, flags,
+                    ctypes.byref(out.struct), _stream(stream)), "w4a4_prepare_weights")
+    return out
+
+
+def w4a4_quantize_act(X: torch.Tensor, inv_smooth, flags: int = 0, qx=None, scale_tok=None,
+                      stream=None):
+    M, K = X.shape
+    qx = qx if qx is not None else torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    scale_tok = scale_tok if scale_tok is not None else torch.empty(M, dtype=torch.float32, device=X.device)
+    _check(_quantize(_ptr(X), M, K, _ptr(inv_smooth), _ptr(qx), _ptr(scale_tok), flags,
+                     _stream(stream)), "w4a4_quantize_act")
+    return qx, scale_tok
+
+
+def w4a4_linear(qx: torch.Tensor, scale_tok: torch.Tensor, w: PreparedWeights, Y=None, stream=None):
+    M = qx.shape[0]
+    Y = Y if Y is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=qx.device)
+    _check(_linear(_ptr(qx), _ptr(scale_tok), M, ctypes.byref(w.struct), _ptr(Y), _stream(stream)),
+           "w4a4_linear")
+    return Y
+
+
+def w4a4_linear_fused(X: torch.Tensor, w: PreparedWeights, Y=None, workspace=None, flags: int = 0,
+                      stream=None):
+    M = X.shape[0]
+    Y = Y if Y is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    need = w4a4_workspace_bytes(M, w.K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+    _check(_fused(_ptr(X), M, ctypes.byref(w.struct), _ptr(Y), _ptr(workspace),
+                  workspace.numel() * workspace.element_size(), flags, _stream(stream)),
+           "w4a4_linear_fused")
+    return Y
+
+
+def w4a4_gemm_s32(qx: torch.Tensor, qw: torch.Tensor, acc=None, stream=None):
+    M, KP = qx.shape
+    N = qw.shape[0]
+    acc = acc if acc is not None else torch.empty((M, N), dtype=torch.int32, device=qx.device)
+    _check(_gemm_s32(_ptr(qx), _ptr(qw), M, N, 2 * KP, _ptr(acc), _stream(stream)), "w4a4_gemm_s32")
+    return acc
+
+
+def w4a4_get_device_status(stream=None) -> int:
+    v = _u32(0)
+    rc = _get_status(_stream(stream), ctypes.byref(v))
+    if rc not in (W4A4_OK, W4A4_ERR_TIMEOUT):
+        _check(rc, "w4a4_get_device_status")
+    return int(v.value)
+
+
+def w4a4_clear_device_status(stream=None) -> None:
+    _check(_clear_status(_stream(stream)), "w4a4_clear_device_status")
