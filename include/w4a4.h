@@ -37,7 +37,8 @@
  *     return W4A4_ERR_ALIGN.
  *   - Shapes: K must be 1024 or 4096 (W4A4_ERR_UNSUPPORTED otherwise); N must
  *     be a positive multiple of 256 (W4A4_ERR_SHAPE); M >= 0, and M = 0 is a
- *     no-op that returns W4A4_OK.  M must stay below 2^31.
+ *     no-op that returns W4A4_OK once the shape, flag and weight checks pass
+ *     (the M-sized pointers may then be NULL).  M must stay below 2^31.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *     only enqueues work on it and returns without synchronizing, except
  *     w4a4_get_device_status.  Launch failures return W4A4_ERR_CUDA.
@@ -92,6 +93,12 @@ typedef struct {
     float *bias;          /* [N] fp32 bias (zeros when the layer has none) */
     float *smooth;        /* [K] s */
     float *inv_smooth;    /* [K] 1/s (what the activation quantizer multiplies by) */
+    int8_t *qw8;          /* optional [N, K] int8: the codes of qw widened to 8 bits in the
+                             order the tensor-core kernel consumes them (see
+                             w4a4_expand_weights).  NULL: the GEMM widens the packed qw on
+                             every tile instead (no extra memory, lower throughput). */
+    int32_t *colsum;      /* [N] sum over k of the int4 codes of row n; required when qw8
+                             is set (NULL otherwise) */
     uint32_t flags;       /* W4A4_FLAG_PLAIN when prepared without DSFQ */
 } w4a4_weights_t;
 
@@ -107,12 +114,20 @@ size_t w4a4_workspace_bytes(int64_t M, int32_t K);
  *   alpha   smoothing exponent in [0, 1] (the page uses 0.5);
  *   flags   0 or W4A4_FLAG_PLAIN (then s = 1 and no rotation; X_calib may be NULL);
  *   out     caller-allocated arrays to fill; out->N and out->K must equal N
- *           and K; out->flags is set to (flags & W4A4_FLAG_PLAIN).
+ *           and K; out->flags is set to (flags & W4A4_FLAG_PLAIN); when
+ *           out->qw8 is set, qw8 and colsum are filled too (w4a4_expand_weights).
  * Rounding decisions are taken in binary32.  A channel whose activation or
  * weight maximum is zero gets s_j = 1. */
 w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_t N, int32_t K,
                                  const uint16_t *X_calib, int64_t M_calib, float alpha,
                                  uint32_t flags, w4a4_weights_t *out, void *stream);
+
+/* Widens the packed codes w->qw into w->qw8 (the tensor-core operand order:
+ * within every group of 8 consecutive codes k = 8g..8g+7 the bytes hold codes
+ * 8g+0, 2, 4, 6, 1, 3, 5, 7, as signed int8) and writes w->colsum[n] =
+ * sum_k code[n, k].  Both arrays must be set.  Not on the pages: weights are
+ * static, so the per-tile widening of B is hoisted to preparation time. */
+w4a4_status w4a4_expand_weights(w4a4_weights_t *w, void *stream);
 
 /* Online activation quantizer [ROT][SMOOTH][PTQ][GRAN]: for each of the M
  * rows of X [M, K] bf16: optional GELU (W4A4_FLAG_GELU), rotation X H/sqrt(K),
@@ -138,12 +153,14 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
                               void *workspace, size_t workspace_bytes, uint32_t flags,
                               void *stream);
 
-/* Integer product only: acc [M, N] int32 = qx [M, K/2] times qw [N, K/2]
- * transposed, both packed int4.  Same tensor-core path as w4a4_linear, with
- * the raw accumulators written out; used to check that the integer product is
+/* Integer product only: acc [M, N] int32 = sum_k qx[m, k] * code_w[n, k] for
+ * packed activation codes qx [M, K/2] and the weight codes of *w (w->qw8 and
+ * w->colsum when set, else the packed w->qw; scale_ch, bias and the smoothing
+ * arrays are not used and may be NULL).  Same tensor-core kernel as
+ * w4a4_linear with the raw accumulators written out: the integer product is
  * exact. */
-w4a4_status w4a4_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int32_t N, int32_t K,
-                          int32_t *acc, void *stream);
+w4a4_status w4a4_gemm_s32(const uint8_t *qx, int64_t M, const w4a4_weights_t *w, int32_t *acc,
+                          void *stream);
 
 /* Synchronizes `stream`, then copies the device status word (bits
  * W4A4_DEV_*) of the current device into *status.  Returns W4A4_ERR_TIMEOUT

@@ -49,7 +49,7 @@ class WeightsT(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("qw", ctypes.c_void_p),
                 ("scale_ch", ctypes.c_void_p), ("bias", ctypes.c_void_p),
                 ("smooth", ctypes.c_void_p), ("inv_smooth", ctypes.c_void_p),
-                ("flags", ctypes.c_uint32)]
+                ("qw8", ctypes.c_void_p), ("colsum", ctypes.c_void_p), ("flags", ctypes.c_uint32)]
 
 
 A = 0x10000  # fake, 16-byte aligned device addresses: never dereferenced on the host
@@ -65,13 +65,15 @@ def _setup(lib):
                                       ctypes.c_uint32, vp]
     lib.w4a4_prepare_weights.argtypes = [vp, vp, i32, i32, vp, i64, ctypes.c_float, ctypes.c_uint32,
                                          ctypes.POINTER(WeightsT), vp]
-    lib.w4a4_gemm_s32.argtypes = [vp, vp, i64, i32, i32, vp, vp]
+    lib.w4a4_gemm_s32.argtypes = [vp, i64, ctypes.POINTER(WeightsT), vp, vp]
+    lib.w4a4_expand_weights.argtypes = [ctypes.POINTER(WeightsT), vp]
     lib.w4a4_status_string.restype = ctypes.c_char_p
     lib.w4a4_version.restype = ctypes.c_char_p
 
 
-def _weights(N=1024, K=1024, base=A, flags=0):
-    return WeightsT(N, K, base, base + 0x1000, base + 0x2000, base + 0x3000, base + 0x4000, flags)
+def _weights(N=1024, K=1024, base=A, flags=0, expanded=True):
+    return WeightsT(N, K, base, base + 0x1000, base + 0x2000, base + 0x3000, base + 0x4000,
+                    base + 0x5000 if expanded else None, base + 0x6000 if expanded else None, flags)
 
 
 def test_workspace_bytes(lib):
@@ -136,10 +138,21 @@ def test_prepare_and_gemm_argument_checks(lib):
     assert P(A, None, 100, 1024, A, 10, 0.5, 0, ctypes.byref(w), None) == 2
     assert P(A + 2, None, 1024, 1024, A, 10, 0.5, 0, ctypes.byref(w), None) == 3
     G = lib.w4a4_gemm_s32
-    assert G(A, A, 10, 1024, 1024, None, None) == 1
-    assert G(A, A, 10, 1000, 1024, A, None) == 2
-    assert G(A, A, 10, 1024, 64, A, None) == 4
-    assert G(A, A, 0, 1024, 1024, A, None) == 0
+    w = _weights()
+    assert G(A, 10, ctypes.byref(w), None, None) == 1
+    assert G(A, 10, None, A, None) == 1
+    assert G(A, 10, ctypes.byref(_weights(N=1000)), A, None) == 2
+    assert G(A, 10, ctypes.byref(_weights(K=64)), A, None) == 4
+    assert G(A, 10, ctypes.byref(_weights(base=A + 8)), A, None) == 3
+    assert G(A, 0, ctypes.byref(w), A, None) == 0
+    half = _weights()
+    half.colsum = None                                    # qw8 without colsum
+    assert G(A, 10, ctypes.byref(half), A, None) == 1
+    E = lib.w4a4_expand_weights
+    assert E(None, None) == 1
+    assert E(ctypes.byref(_weights(expanded=False)), None) == 1
+    assert E(ctypes.byref(_weights(K=2048)), None) == 4
+    assert E(ctypes.byref(_weights(base=A + 4)), None) == 3
 
 
 def test_status_strings(lib):

@@ -49,26 +49,50 @@ def y_to_f64(Y):
 
 
 # ------------------------------------------------------------------ integer GEMM
+def _codes_weights(w4, B, K, expanded):
+    """Weights struct holding raw packed codes B (and their widened copy)."""
+    pw = w4.PreparedWeights(B.shape[0], K, expanded=expanded)
+    pw.qw.copy_(dev(B))
+    if expanded:
+        w4.w4a4_expand_weights(pw)
+    return pw
+
+
+@pytest.mark.parametrize("expanded", [True, False])
 @pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (128, 256, 1024), (300, 512, 1024),
                                    (1374, 1024, 1024), (257, 256, 4096), (640, 1024, 4096)])
-def test_gemm_s32_bit_exact(w4, M, N, K):
+def test_gemm_s32_bit_exact(w4, M, N, K, expanded):
     A = synth.random_packed_codes(M, K, seed=M + 7)
     B = synth.random_packed_codes(N, K, seed=N + 11)
-    acc = host(w4.w4a4_gemm_s32(dev(A), dev(B)))
-    torch.cuda.synchronize()
+    acc = host(w4.w4a4_gemm_s32(dev(A), _codes_weights(w4, B, K, expanded)))
     want = oracle.int_gemm(oracle.unpack_int4(A, K), oracle.unpack_int4(B, K))
     assert np.array_equal(acc.astype(np.int64), want)
 
 
-def test_gemm_s32_extreme_codes(w4):
+def test_expand_weights_layout_and_sums(w4):
+    N, K = 256, 1024
+    B = synth.random_packed_codes(N, K, seed=3)
+    pw = _codes_weights(w4, B, K, True)
+    codes = oracle.unpack_int4(B, K).astype(np.int64)
+    assert np.array_equal(host(pw.colsum).astype(np.int64), codes.sum(axis=1))
+    perm = np.array([0, 2, 4, 6, 1, 3, 5, 7])
+    want = codes.reshape(N, K // 8, 8)[:, :, perm].reshape(N, K)
+    assert np.array_equal(host(pw.qw8).astype(np.int64), want)
+
+
+@pytest.mark.parametrize("expanded", [True, False])
+def test_gemm_s32_extreme_codes(w4, expanded):
     K = 4096
     A = np.full((130, K // 2), 0x88, np.uint8)    # every code -8
     B = np.full((256, K // 2), 0x88, np.uint8)
-    acc = host(w4.w4a4_gemm_s32(dev(A), dev(B)))
+    acc = host(w4.w4a4_gemm_s32(dev(A), _codes_weights(w4, B, K, expanded)))
     assert np.all(acc == 64 * K)
     B2 = np.full((256, K // 2), 0x77, np.uint8)   # every code 7
-    acc = host(w4.w4a4_gemm_s32(dev(A), dev(B2)))
+    acc = host(w4.w4a4_gemm_s32(dev(A), _codes_weights(w4, B2, K, expanded)))
     assert np.all(acc == -56 * K)
+    A2 = np.full((130, K // 2), 0x77, np.uint8)
+    acc = host(w4.w4a4_gemm_s32(dev(A2), _codes_weights(w4, B2, K, expanded)))
+    assert np.all(acc == 49 * K)
 
 
 # -------------------------------------------------------------- activation quantizer
@@ -81,7 +105,7 @@ def _check_quant(w4, X, K, inv_s32, flags, max_frac):
     s = np.ones(K) if inv_s32 is None else 1.0 / inv_s32.astype(np.float64)
     hat = oracle.act_hat(X, s, gelu=gelu, plain=plain)
     want_q, want_d = oracle.quantize_rows(hat, 4, "f32")
-    np.testing.assert_allclose(st, want_d, rtol=1e-5, atol=0)
+    np.testing.assert_allclose(st, want_d, rtol=2e-5, atol=0)
     xin = oracle.bf16_to_f64(oracle.gelu_bf16(X) if gelu else X)
     amax = np.max(np.abs(hat), axis=1)
     with np.errstate(divide="ignore", invalid="ignore"):
@@ -139,14 +163,14 @@ def test_prepare_weights_parity(w4, N, K):
     Xc = synth.activations(1374, K, seed=K + 2)
     pw = w4.w4a4_prepare_weights(bf16_dev(W), bf16_dev(b), bf16_dev(Xc))
     ow = oracle.prepare_weights(W, b, Xc)
-    np.testing.assert_allclose(host(pw.smooth), ow.s, rtol=2e-6)
-    np.testing.assert_allclose(host(pw.inv_smooth), 1.0 / ow.s, rtol=2e-6)
+    np.testing.assert_allclose(host(pw.smooth), ow.s, rtol=2e-5)
+    np.testing.assert_allclose(host(pw.inv_smooth), 1.0 / ow.s, rtol=2e-5)
     np.testing.assert_allclose(host(pw.bias), ow.bias, rtol=0, atol=0)
     # codes: the oracle's binary32 decision on the GPU's own (binary32) s
     s32 = host(pw.smooth).astype(np.float64)
     hat = ow.Wt * s32[None, :]
     want_q, want_d = oracle.quantize_rows(hat, 4, "f32")
-    np.testing.assert_allclose(host(pw.scale_ch), want_d, rtol=1e-5)
+    np.testing.assert_allclose(host(pw.scale_ch), want_d, rtol=2e-5)
     amax = np.max(np.abs(hat), axis=1)
     ratio = hat * 7.0 / amax[:, None]
     bound = tie_bound(oracle.bf16_to_f64(W), s32, ratio, amax, K)
@@ -154,15 +178,15 @@ def test_prepare_weights_parity(w4, N, K):
 
 
 # -------------------------------------------------------------------- epilogue
+@pytest.mark.parametrize("expanded", [True, False])
 @pytest.mark.parametrize("M,N,K", [(300, 512, 1024), (1374, 1024, 4096)])
-def test_linear_epilogue_on_identical_codes(w4, M, N, K):
+def test_linear_epilogue_on_identical_codes(w4, M, N, K, expanded):
     A = synth.random_packed_codes(M, K, seed=1)
     B = synth.random_packed_codes(N, K, seed=2)
     st = synth.random_scales(M, seed=3, lo=1e-3, hi=1e-1)
     sc = synth.random_scales(N, seed=4, lo=1e-3, hi=1e-2)
     bias = synth.random_scales(N, seed=5, lo=-0.5, hi=0.5)
-    pw = w4.PreparedWeights(N, K)
-    pw.qw.copy_(dev(B))
+    pw = _codes_weights(w4, B, K, expanded)
     pw.scale_ch.copy_(dev(sc))
     pw.bias.copy_(dev(bias))
     Y = w4.w4a4_linear(dev(A), dev(st), pw)
@@ -170,25 +194,31 @@ def test_linear_epilogue_on_identical_codes(w4, M, N, K):
     acc = oracle.int_gemm(oracle.unpack_int4(A, K), oracle.unpack_int4(B, K))
     want = oracle.dequant(acc, st.astype(np.float64), sc.astype(np.float64), bias.astype(np.float64))
     want_bf = oracle.bf16_to_f64(oracle.f64_to_bf16(want))
-    ulp = np.abs(want_bf) * 2.0 ** -7
-    assert np.all(np.abs(got - want_bf) <= ulp + 1e-30)
+    # one bf16 step of the result, plus the fp32 epilogue's own error bound
+    # (a few ulp of the largest term), which matters where y ~ -bias cancels
+    terms = np.abs(acc * st.astype(np.float64)[:, None] * sc.astype(np.float64)[None, :]) + np.abs(bias)[None, :]
+    tol = np.abs(want_bf) * 2.0 ** -7 + 4 * 2.0 ** -24 * terms
+    assert np.all(np.abs(got - want_bf) <= tol)
     assert np.mean(got == want_bf) > 0.999
 
 
 # -------------------------------------------------------------------- end to end
-def _linear_case(w4, M, N, K, seed, gelu=False, plain=False, sample=None):
+def _linear_case(w4, M, N, K, seed, gelu=False, plain=False, sample=None, expanded=True):
     X = synth.activations(M, K, seed=seed)
     W = synth.weights(N, K, seed=seed + 1)
     b = synth.bias(N, seed=seed + 2)
     Xc = X[:synth.calibration_rows(M)]
     flags = (w4.W4A4_FLAG_GELU if gelu else 0) | (w4.W4A4_FLAG_PLAIN if plain else 0)
     pw = w4.w4a4_prepare_weights(bf16_dev(W), bf16_dev(b), bf16_dev(Xc),
-                                 flags=w4.W4A4_FLAG_PLAIN if plain else 0)
+                                 flags=w4.W4A4_FLAG_PLAIN if plain else 0, expanded=expanded)
     Y = y_to_f64(w4.w4a4_linear_fused(bf16_dev(X), pw, flags=flags))
     assert w4.w4a4_get_device_status() == 0
-    ow = oracle.prepare_weights(W, b, Xc, plain=plain)
+    # rounding decisions in binary32 on both sides (the kernels' precision);
+    # bf16 inputs without rotation hit exact rounding ties, which fp64 and fp32
+    # resolve differently
+    ow = oracle.prepare_weights(W, b, Xc, plain=plain, decision="f32")
     rows = np.arange(M) if sample is None else sample
-    Yo = oracle.linear(X[rows], ow, gelu=gelu, plain=plain)[0]
+    Yo = oracle.linear(X[rows], ow, gelu=gelu, plain=plain, decision="f32")[0]
     err = rel_fro(Y[rows], Yo)
     ref = oracle.reference_fp(X[rows], W, b, gelu=gelu)
     return err, oracle.sqnr_db(ref, Y[rows]), oracle.sqnr_db(ref, Yo)
@@ -200,6 +230,11 @@ def test_linear_fused_end_to_end(w4, M, N, K):
     err, sq_gpu, sq_or = _linear_case(w4, M, N, K, seed=M + N)
     assert err <= 2e-3, err
     assert abs(sq_gpu - sq_or) < 0.1
+
+
+def test_linear_fused_packed_weights_path(w4):
+    err, _, _ = _linear_case(w4, 700, 512, 1024, seed=91, expanded=False)
+    assert err <= 2e-3, err
 
 
 def test_linear_fused_gelu_and_plain(w4):

@@ -31,6 +31,8 @@ w4a4_status check_weights(const w4a4_weights_t *w) {
       !aligned16(w->inv_smooth))
     return W4A4_ERR_ALIGN;
   if (w->flags & ~W4A4_FLAG_PLAIN) return W4A4_ERR_UNSUPPORTED;
+  if ((w->qw8 == nullptr) != (w->colsum == nullptr)) return W4A4_ERR_ARG;
+  if (!aligned16(w->qw8) || !aligned16(w->colsum)) return W4A4_ERR_ALIGN;
   return W4A4_OK;
 }
 
@@ -39,6 +41,7 @@ w4a4_status check_act(const void *X, int64_t M, int32_t K, const float *inv_smoo
   if (flags & ~kKnownFlags) return W4A4_ERR_UNSUPPORTED;
   if (!k_ok(K)) return W4A4_ERR_UNSUPPORTED;
   if (!m_ok(M)) return W4A4_ERR_SHAPE;
+  if (M == 0) return W4A4_OK;
   if (!X || !qx || !scale_tok) return W4A4_ERR_ARG;
   if (!(flags & W4A4_FLAG_PLAIN) && !inv_smooth) return W4A4_ERR_ARG;
   if (!aligned16(X) || !aligned16(qx) || !aligned16(scale_tok) ||
@@ -73,6 +76,8 @@ w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_
   }
   if (!out->qw || !out->scale_ch || !out->bias || !out->smooth || !out->inv_smooth)
     return W4A4_ERR_ARG;
+  if ((out->qw8 == nullptr) != (out->colsum == nullptr)) return W4A4_ERR_ARG;
+  if (!aligned16(out->qw8) || !aligned16(out->colsum)) return W4A4_ERR_ALIGN;
   if (!aligned16(W) || (bias && !aligned16(bias)) || !aligned16(out->qw) ||
       !aligned16(out->scale_ch) || !aligned16(out->bias) || !aligned16(out->smooth) ||
       !aligned16(out->inv_smooth))
@@ -96,7 +101,18 @@ w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_
   if (e != cudaSuccess) return cuda_status(e);
   if ((e = w4a4::launch_bias_to_f32(bias, out->bias, N, st)) != cudaSuccess) return cuda_status(e);
   out->flags = flags & W4A4_FLAG_PLAIN;
+  if (out->qw8) return w4a4_expand_weights(out, stream);
   return W4A4_OK;
+}
+
+w4a4_status w4a4_expand_weights(w4a4_weights_t *w, void *stream) {
+  if (!w) return W4A4_ERR_ARG;
+  if (!k_ok(w->K)) return W4A4_ERR_UNSUPPORTED;
+  if (!n_ok(w->N)) return W4A4_ERR_SHAPE;
+  if (!w->qw || !w->qw8 || !w->colsum) return W4A4_ERR_ARG;
+  if (!aligned16(w->qw) || !aligned16(w->qw8) || !aligned16(w->colsum)) return W4A4_ERR_ALIGN;
+  return cuda_status(w4a4::launch_expand_weights(w->qw, w->N, w->K, w->qw8, w->colsum,
+                                                 as_stream(stream)));
 }
 
 w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const float *inv_smooth,
@@ -113,9 +129,11 @@ w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
   w4a4_status s = check_weights(w);
   if (s != W4A4_OK) return s;
   if (!m_ok(M)) return W4A4_ERR_SHAPE;
+  if (M == 0) return W4A4_OK;
   if (!qx || !scale_tok || !Y) return W4A4_ERR_ARG;
   if (!aligned16(qx) || !aligned16(scale_tok) || !aligned16(Y)) return W4A4_ERR_ALIGN;
-  w4a4::GemmArgs a{qx, w->qw, scale_tok, w->scale_ch, w->bias, Y, nullptr, M, w->N, w->K};
+  w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, scale_tok, w->scale_ch, w->bias, Y, nullptr,
+                   M, w->N, w->K};
   return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
 }
 
@@ -127,10 +145,10 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
   if (flags & ~kKnownFlags) return W4A4_ERR_UNSUPPORTED;
   if ((flags & W4A4_FLAG_PLAIN) != (w->flags & W4A4_FLAG_PLAIN)) return W4A4_ERR_ARG;
   if (!m_ok(M)) return W4A4_ERR_SHAPE;
+  if (M == 0) return W4A4_OK;  // empty input: nothing to read or write
   if (!X || !Y || !workspace) return W4A4_ERR_ARG;
   if (workspace_bytes < w4a4_workspace_bytes(M, w->K)) return W4A4_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(Y) || !aligned16(workspace)) return W4A4_ERR_ALIGN;
-  if (M == 0) return W4A4_OK;
   uint8_t *qx = static_cast<uint8_t *>(workspace);
   float *st = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (w->K / 2)));
   cudaStream_t cs = as_stream(stream);
@@ -138,17 +156,24 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
                                              !(flags & W4A4_FLAG_PLAIN),
                                              (flags & W4A4_FLAG_GELU) != 0, cs);
   if (e != cudaSuccess) return cuda_status(e);
-  w4a4::GemmArgs a{qx, w->qw, st, w->scale_ch, w->bias, Y, nullptr, M, w->N, w->K};
+  w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, st, w->scale_ch, w->bias, Y, nullptr,
+                   M, w->N, w->K};
   return cuda_status(w4a4::launch_gemm(a, cs));
 }
 
-w4a4_status w4a4_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int32_t N, int32_t K,
-                          int32_t *acc, void *stream) {
-  if (!k_ok(K)) return W4A4_ERR_UNSUPPORTED;
-  if (!n_ok(N) || !m_ok(M)) return W4A4_ERR_SHAPE;
-  if (!qx || !qw || !acc) return W4A4_ERR_ARG;
-  if (!aligned16(qx) || !aligned16(qw) || !aligned16(acc)) return W4A4_ERR_ALIGN;
-  w4a4::GemmArgs a{qx, qw, nullptr, nullptr, nullptr, nullptr, acc, M, N, K};
+w4a4_status w4a4_gemm_s32(const uint8_t *qx, int64_t M, const w4a4_weights_t *w, int32_t *acc,
+                          void *stream) {
+  if (!w) return W4A4_ERR_ARG;
+  if (!k_ok(w->K)) return W4A4_ERR_UNSUPPORTED;
+  if (!n_ok(w->N) || !m_ok(M)) return W4A4_ERR_SHAPE;
+  if ((w->qw8 == nullptr) != (w->colsum == nullptr)) return W4A4_ERR_ARG;
+  if (M == 0) return W4A4_OK;
+  if (!qx || !acc || (!w->qw && !w->qw8)) return W4A4_ERR_ARG;
+  if (!aligned16(qx) || !aligned16(acc) || !aligned16(w->qw) || !aligned16(w->qw8) ||
+      !aligned16(w->colsum))
+    return W4A4_ERR_ALIGN;
+  w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, nullptr, nullptr, nullptr, nullptr, acc,
+                   M, w->N, w->K};
   return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
 }
 

@@ -5,26 +5,41 @@
 // qx [M, K/2] and qw [N, K/2] hold int4 codes packed two per byte (page
 // "十亿参数的三维重建模型，能塞进手机吗？", section 训练后量化（PTQ）: symmetric
 // 4-bit codes; section 细粒度量化粒度 read as per-token x per-channel steps).
-// tcgen05 has no 4-bit integer MMA, so the kernel
-//   1. stages packed tiles in shared memory with TMA (one warp, one thread),
-//   2. unpacks them to int8 (4 warps) straight into the 128-byte-swizzled
-//      K-major layout the tensor core reads,
-//   3. issues tcgen05.mma kind::i8 (one thread) with s32 accumulators in tensor
-//      memory, double-buffered so the epilogue of one tile overlaps the main
-//      loop of the next,
-//   4. reads the accumulators back with tcgen05.ld (4 warps), applies the
-//      per-token x per-channel steps and the bias in fp32, rounds to bf16 and
-//      writes the tile with TMA stores from a swizzled staging buffer.
-// The CTA is persistent (one per SM, tiles assigned round-robin, M-major so
-// that concurrently running CTAs share activation rows through L2).
+// tcgen05 has no 4-bit integer MMA, so the int4 codes are widened to 8 bits
+// and multiplied with tcgen05.mma kind::i8 (s32 accumulators in tensor
+// memory).  Two ways of feeding B (the weights):
 //
-// Unpacking permutes K inside every group of 8 codes (even codes first, then
-// odd ones).  A and B are unpacked identically, so every dot product sums the
-// same pairs and the integer result is exact and unchanged.
+//   * expanded B (default, when the prepared weights carry qw8): the weights
+//     are static, so their int4 codes are widened once, at preparation time,
+//     into qw8 [N, K] int8 in exactly the order the kernel widens A.  The
+//     kernel TMA-loads B tiles straight into the 128-byte swizzled operand
+//     layout.  A is TMA-staged packed and widened in shared memory as the
+//     unsigned value code + 8 (a nibble XOR), which costs 3 integer ops per 8
+//     codes; sum_k (qa + 8) qb = acc + 8 * colsum[n], so the epilogue
+//     subtracts 8 * colsum[n] (colsum = per-output-channel sum of the weight
+//     codes, prepared with qw8).  The result is exact.
+//   * packed B (qw8 == NULL): both operands are TMA-staged packed and
+//     sign-extended to int8 in shared memory on every tile (no extra weight
+//     memory, more shared-memory traffic and integer work).
 //
-// Every wait is bounded (ptx.cuh): a stuck pipeline sets the device status word
-// and the CTA drains its in-flight copies and MMAs, frees its tensor memory and
-// returns.
+// Warp roles (one persistent CTA per SM, tiles round-robin, M-major):
+//   warp 0      TMA producer (one thread)
+//   warp 1      tcgen05.mma issuer (one thread)
+//   warp 2      tensor-memory allocator
+//   warps 4..7  widen packed int4 -> int8 into the swizzled operand tiles
+//   warps 8..11 epilogue: tcgen05.ld accumulators, subtract the code-offset
+//               term, scale by scale_tok[m] * scale_ch[n], add bias in fp32,
+//               round to bf16, TMA-store through a swizzled staging buffer.
+// Accumulators are double-buffered in tensor memory (2 x 256 columns) so the
+// epilogue of one tile overlaps the main loop of the next.
+//
+// Widening permutes K inside every group of 8 codes (even codes first, then
+// odd ones).  A and B use the same order, so every dot product sums the same
+// pairs and the integer result is unchanged.
+//
+// Every wait is bounded (ptx.cuh): a stuck pipeline sets the device status
+// word and the CTA drains its in-flight copies and MMAs, frees its tensor
+// memory and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,57 +62,70 @@ constexpr int BM = 128;   // tile rows (tokens)
 constexpr int BN = 256;   // tile columns (output channels)
 constexpr int BK = 128;   // int8 elements per k-block = one 128-byte swizzle row
 constexpr int BKP = 64;   // packed bytes per row per k-block
-constexpr int PST = 4;    // packed (TMA) stages
-constexpr int UST = 2;    // unpacked (MMA operand) stages
-constexpr int A_PK = BM * BKP;
-constexpr int B_PK = BN * BKP;
-constexpr int A_UN = BM * BK;
-constexpr int B_UN = BN * BK;
+constexpr int A_PK = BM * BKP;  // 8 KB
+constexpr int B_PK = BN * BKP;  // 16 KB
+constexpr int A_UN = BM * BK;   // 16 KB
+constexpr int B_UN = BN * BK;   // 32 KB
 constexpr int EPI_BYTES = 32 * 32 * 2;  // one warp's 32 x 32 bf16 staging tile
-constexpr int NUM_THREADS = 384;        // 12 warps, roles below
+constexpr int NUM_THREADS = 384;
 constexpr uint32_t TMEM_COLS = 512;     // two 128 x 256 s32 accumulators
-constexpr int OFF_A_UN = 0;
-constexpr int OFF_B_UN = OFF_A_UN + UST * A_UN;
-constexpr int OFF_A_PK = OFF_B_UN + UST * B_UN;
-constexpr int OFF_B_PK = OFF_A_PK + PST * A_PK;
-constexpr int OFF_EPI = OFF_B_PK + PST * B_PK;
-constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BYTES;
-constexpr int NUM_BARS = 2 * PST + 2 * UST + 2 * 2 + 1;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_B_UN % 1024 == 0 && OFF_A_PK % 1024 == 0 && OFF_EPI % 1024 == 0, "alignment");
 
-constexpr uint32_t IDESC = idesc_i8<BM, BN>();
+// Shared-memory plan, per pipeline stage.
+template <bool B_PACKED>
+struct Plan {
+  static constexpr int STAGES = B_PACKED ? 2 : 3;
+  static constexpr int OFF_A_PK = 0;
+  static constexpr int OFF_B_PK = A_PK;                                  // B_PACKED only
+  static constexpr int OFF_A_UN = B_PACKED ? A_PK + B_PK : A_PK;
+  static constexpr int OFF_B_UN = OFF_A_UN + A_UN;
+  static constexpr int STAGE_BYTES = OFF_B_UN + B_UN;
+  static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+  static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BYTES;
+  static constexpr int NUM_BARS = 3 * STAGES + 2 * 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(OFF_A_UN % 1024 == 0 && OFF_B_UN % 1024 == 0 && STAGE_BYTES % 1024 == 0 &&
+                    OFF_EPI % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
+  // tcgen05.mma kind::i8 instruction descriptor: s32 D; A unsigned (code + 8)
+  // with expanded B, signed with packed B; B signed; both K-major; 128 x 256.
+  static constexpr uint32_t IDESC = (2u << 4) | ((B_PACKED ? 1u : 0u) << 7) | (1u << 10) |
+                                    (static_cast<uint32_t>(BN >> 3) << 17) |
+                                    (static_cast<uint32_t>(BM >> 4) << 24);
+};
 
-// Warp roles.
 constexpr int W_TMA = 0, W_MMA = 1, W_TMEM = 2;
 constexpr int W_UNPACK0 = 4;  // warps 4..7
 constexpr int W_EPI0 = 8;     // warps 8..11 (warp % 4 selects its 32 TMEM lanes)
 
-// 4 nibbles (one per byte, values 0..15 = two's-complement int4) -> 4 int8.
+// 4 nibbles (one per byte, 0..15 = two's-complement int4) -> 4 signed int8.
 __device__ __forceinline__ uint32_t sext4x4(uint32_t n) {
   return ((n ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
 }
 
-// Packed 16-byte chunk (32 codes) -> two 16-byte int8 chunks.  Word t holds
-// codes 8t..8t+7; its even codes go first, then its odd codes.
-__device__ __forceinline__ void unpack_chunk(uint4 v, uint4 &o0, uint4 &o1) {
-  o0.x = sext4x4(v.x & 0x0F0F0F0Fu);
-  o0.y = sext4x4((v.x >> 4) & 0x0F0F0F0Fu);
-  o0.z = sext4x4(v.y & 0x0F0F0F0Fu);
-  o0.w = sext4x4((v.y >> 4) & 0x0F0F0F0Fu);
-  o1.x = sext4x4(v.z & 0x0F0F0F0Fu);
-  o1.y = sext4x4((v.z >> 4) & 0x0F0F0F0Fu);
-  o1.z = sext4x4(v.w & 0x0F0F0F0Fu);
-  o1.w = sext4x4((v.w >> 4) & 0x0F0F0F0Fu);
+// Widen a 16-byte packed chunk (32 codes) to two 16-byte chunks.  Word t
+// holds codes 8t..8t+7; its even codes go first, then its odd codes.
+// SIGNED: two's-complement int8; otherwise the unsigned value code + 8.
+template <bool SIGNED>
+__device__ __forceinline__ void widen_chunk(uint4 v, uint4 &o0, uint4 &o1) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t lo = w[t] & 0x0F0F0F0Fu, hi = (w[t] >> 4) & 0x0F0F0F0Fu;
+    o[2 * t] = SIGNED ? sext4x4(lo) : (lo ^ 0x08080808u);
+    o[2 * t + 1] = SIGNED ? sext4x4(hi) : (hi ^ 0x08080808u);
+  }
+  o0 = make_uint4(o[0], o[1], o[2], o[3]);
+  o1 = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Unpack NCH packed chunks of a tile (rows of 64 packed bytes) into the
+// Widen NCH packed chunks of a tile (rows of 64 packed bytes) into the
 // 128-byte swizzled int8 tile.  Chunk q covers row q/4, codes 32(q%4)..+31.
-template <int NCH>
-__device__ __forceinline__ void unpack_tile(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
-                                            int t) {
+template <int NCH, bool SIGNED>
+__device__ __forceinline__ void widen_tile(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
+                                           int t) {
   uint4 v[NCH];
 #pragma unroll
   for (int i = 0; i < NCH; ++i) v[i] = *reinterpret_cast<const uint4 *>(src + (t + 128 * i) * 16);
@@ -106,7 +134,7 @@ __device__ __forceinline__ void unpack_tile(const uint8_t *__restrict__ src, uin
     const int q = t + 128 * i;
     const int r = q >> 2, c = q & 3;
     uint4 o0, o1;
-    unpack_chunk(v[i], o0, o1);
+    widen_chunk<SIGNED>(v[i], o0, o1);
     uint8_t *row = dst + r * 128;
     *reinterpret_cast<uint4 *>(row + (((2 * c) ^ (r & 7)) << 4)) = o0;
     *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ (r & 7)) << 4)) = o1;
@@ -118,38 +146,42 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-template <bool OUT_S32>
+// int32 -> float for |x| < 2^22, exact: the bit pattern 0x4B400000 + x is the
+// float 1.5 * 2^23 + x.
+__device__ __forceinline__ float small_int_to_float(int32_t biased_bits) {
+  return __int_as_float(biased_bits) - 12582912.0f;
+}
+
+template <bool B_PACKED, bool OUT_S32>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmY, const float *__restrict__ scale_tok,
                      const float *__restrict__ scale_ch, const float *__restrict__ bias,
-                     int32_t *__restrict__ acc_out, int M, int N, int num_n_tiles, int num_tiles,
-                     int num_kb) {
+                     const int32_t *__restrict__ colsum, int32_t *__restrict__ acc_out, int M, int N,
+                     int num_n_tiles, int num_tiles, int num_kb) {
+  using P = Plan<B_PACKED>;
+  constexpr int ST = P::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *pk_full = bars;
-  uint64_t *pk_empty = pk_full + PST;
-  uint64_t *un_full = pk_empty + PST;
-  uint64_t *un_empty = un_full + UST;
-  uint64_t *acc_full = un_empty + UST;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + P::OFF_BAR);
+  uint64_t *full = bars;            // TMA bytes landed
+  uint64_t *widened = full + ST;    // operand tiles ready for the tensor core
+  uint64_t *freed = widened + ST;   // MMAs reading the stage have completed
+  uint64_t *acc_full = freed + ST;
   uint64_t *acc_empty = acc_full + 2;
   uint64_t *mma_done = acc_empty + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + P::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + P::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < PST; ++s) {
-      mbar_init(&pk_full[s], 1);
-      mbar_init(&pk_empty[s], 128);
-    }
-    for (int u = 0; u < UST; ++u) {
-      mbar_init(&un_full[u], 128);
-      mbar_init(&un_empty[u], 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&widened[s], 128);
+      mbar_init(&freed[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -181,20 +213,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
         for (int kb = 0; kb < num_kb; ++kb) {
-          const uint32_t s = issued % PST, ph = (issued / PST) & 1u;
-          if (!mbar_wait(&pk_empty[s], ph ^ 1u, abort_flag, &g_status)) {
+          const uint32_t s = issued % ST, ph = (issued / ST) & 1u;
+          if (!mbar_wait(&freed[s], ph ^ 1u, abort_flag, &g_status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&pk_full[s], A_PK + B_PK);
-          tma_load_2d(smem + OFF_A_PK + s * A_PK, &tmA, kb * BKP, mb * BM, &pk_full[s]);
-          tma_load_2d(smem + OFF_B_PK + s * B_PK, &tmB, kb * BKP, nb * BN, &pk_full[s]);
+          uint8_t *stage = smem + s * P::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], A_PK + (B_PACKED ? B_PK : B_UN));
+          tma_load_2d(stage + P::OFF_A_PK, &tmA, kb * BKP, mb * BM, &full[s]);
+          if (B_PACKED)
+            tma_load_2d(stage + P::OFF_B_PK, &tmB, kb * BKP, nb * BN, &full[s]);
+          else
+            tma_load_2d(stage + P::OFF_B_UN, &tmB, kb * BK, nb * BN, &full[s]);
           ++issued;
         }
       }
       // let every issued copy land before the CTA can exit
-      for (uint32_t t = (issued > PST ? issued - PST : 0); t < issued; ++t)
-        mbar_wait_drain(&pk_full[t % PST], (t / PST) & 1u, &g_status);
+      for (uint32_t t = (issued > ST ? issued - ST : 0); t < issued; ++t)
+        mbar_wait_drain(&full[t % ST], (t / ST) & 1u, &g_status);
     }
   } else if (warp == W_MMA) {
     if (lane == 0) {
@@ -208,19 +244,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
-          const uint32_t u = consumed % UST, pu = (consumed / UST) & 1u;
-          if (!mbar_wait(&un_full[u], pu, abort_flag, &g_status)) {
+          const uint32_t s = consumed % ST, ps = (consumed / ST) & 1u;
+          if (!mbar_wait(&widened[s], ps, abort_flag, &g_status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + OFF_A_UN + u * A_UN);
-          const uint32_t b0 = smem_u32(smem + OFF_B_UN + u * B_UN);
+          const uint32_t a0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_A_UN);
+          const uint32_t b0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_B_UN);
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
-            mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), IDESC,
+            mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), P::IDESC,
                    (kb | kk) != 0 ? 1u : 0u);
-          tc_commit(&un_empty[u]);
+          tc_commit(&freed[s]);
           ++consumed;
         }
         if (ok) tc_commit(&acc_full[b]);
@@ -230,23 +266,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait_drain(mma_done, 0, &g_status);
     }
   } else if (warp >= W_UNPACK0 && warp < W_UNPACK0 + 4) {
-    // ------------------------------------------------------------------ unpack
+    // ------------------------------------------------------------------ widen
     const int t = threadIdx.x - W_UNPACK0 * 32;
     uint32_t n = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb, ++n) {
-        const uint32_t s = n % PST, ps = (n / PST) & 1u;
-        const uint32_t u = n % UST, pu = (n / UST) & 1u;
-        if (!mbar_wait(&pk_full[s], ps, abort_flag, &g_status) || !mbar_wait(&un_empty[u], pu ^ 1u, abort_flag, &g_status)) {
+        const uint32_t s = n % ST, ps = (n / ST) & 1u;
+        if (!mbar_wait(&full[s], ps, abort_flag, &g_status)) {
           ok = false;
           break;
         }
-        unpack_tile<A_PK / 16 / 128>(smem + OFF_A_PK + s * A_PK, smem + OFF_A_UN + u * A_UN, t);
-        unpack_tile<B_PK / 16 / 128>(smem + OFF_B_PK + s * B_PK, smem + OFF_B_UN + u * B_UN, t);
+        uint8_t *stage = smem + s * P::STAGE_BYTES;
+        widen_tile<A_PK / 16 / 128, B_PACKED>(stage + P::OFF_A_PK, stage + P::OFF_A_UN, t);
+        if (B_PACKED) widen_tile<B_PK / 16 / 128, true>(stage + P::OFF_B_PK, stage + P::OFF_B_UN, t);
         fence_proxy_async_smem();
-        mbar_arrive(&pk_empty[s]);
-        mbar_arrive(&un_full[u]);
+        mbar_arrive(&widened[s]);
       }
     }
   } else if (warp >= W_EPI0) {
@@ -273,13 +308,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
         const int n0 = nb * BN + ch * 32;
+        // biased[j] = bit pattern 0x4B400000 + acc[m, n0 + j] (exact integer arithmetic)
+        int32_t biased[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          int4 off = make_int4(0, 0, 0, 0);
+          if (!B_PACKED) off = __ldg(reinterpret_cast<const int4 *>(colsum + n0) + c);
+          biased[4 * c + 0] = static_cast<int32_t>(r[4 * c + 0]) - 8 * off.x + 0x4B400000;
+          biased[4 * c + 1] = static_cast<int32_t>(r[4 * c + 1]) - 8 * off.y + 0x4B400000;
+          biased[4 * c + 2] = static_cast<int32_t>(r[4 * c + 2]) - 8 * off.z + 0x4B400000;
+          biased[4 * c + 3] = static_cast<int32_t>(r[4 * c + 3]) - 8 * off.w + 0x4B400000;
+        }
         if (OUT_S32) {
           if (m < M) {
             int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(m) * N + n0);
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              dst[c] = make_int4(static_cast<int>(r[4 * c]), static_cast<int>(r[4 * c + 1]),
-                                 static_cast<int>(r[4 * c + 2]), static_cast<int>(r[4 * c + 3]));
+              dst[c] = make_int4(biased[4 * c] - 0x4B400000, biased[4 * c + 1] - 0x4B400000,
+                                 biased[4 * c + 2] - 0x4B400000, biased[4 * c + 3] - 0x4B400000);
           }
         } else {
           uint32_t pk[16];
@@ -288,14 +334,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const float4 sc = __ldg(sc4 + c), bi = __ldg(bi4 + c);
-            const float y0 = fmaf(static_cast<float>(static_cast<int>(r[4 * c + 0])), st * sc.x, bi.x);
-            const float y1 = fmaf(static_cast<float>(static_cast<int>(r[4 * c + 1])), st * sc.y, bi.y);
-            const float y2 = fmaf(static_cast<float>(static_cast<int>(r[4 * c + 2])), st * sc.z, bi.z);
-            const float y3 = fmaf(static_cast<float>(static_cast<int>(r[4 * c + 3])), st * sc.w, bi.w);
+            const float y0 = fmaf(small_int_to_float(biased[4 * c + 0]), st * sc.x, bi.x);
+            const float y1 = fmaf(small_int_to_float(biased[4 * c + 1]), st * sc.y, bi.y);
+            const float y2 = fmaf(small_int_to_float(biased[4 * c + 2]), st * sc.z, bi.z);
+            const float y3 = fmaf(small_int_to_float(biased[4 * c + 3]), st * sc.w, bi.w);
             pk[2 * c] = pack_bf16x2(y0, y1);
             pk[2 * c + 1] = pack_bf16x2(y2, y3);
           }
-          uint8_t *stg = smem + OFF_EPI + (ew * 2 + (ch & 1)) * EPI_BYTES;
+          uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (ch & 1)) * EPI_BYTES;
           if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
           __syncwarp();
 #pragma unroll
@@ -318,6 +364,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == W_TMEM) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// Expand packed weight codes to the int8 operand order the kernel above
+// widens A in (signed), and sum each row's codes: one warp per row.
+__global__ void expand_weights_kernel(const uint8_t *__restrict__ qw, int N, int K,
+                                      int8_t *__restrict__ qw8, int32_t *__restrict__ colsum) {
+  const int lane = threadIdx.x & 31;
+  const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (n >= N) return;
+  const uint4 *src = reinterpret_cast<const uint4 *>(qw + static_cast<int64_t>(n) * (K / 2));
+  uint4 *dst = reinterpret_cast<uint4 *>(qw8 + static_cast<int64_t>(n) * K);
+  int sum = 0;
+  for (int c = lane; c < K / 32; c += 32) {
+    uint4 o0, o1;
+    widen_chunk<true>(src[c], o0, o1);
+    dst[2 * c] = o0;
+    dst[2 * c + 1] = o1;
+    const uint32_t w[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sum = __dp4a(static_cast<int>(w[i]), 0x01010101, sum);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) colsum[n] = sum;
 }
 
 // --------------------------------------------------------------- host side
@@ -353,22 +423,30 @@ bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool OUT_S32>
+template <bool B_PACKED, bool OUT_S32>
 cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(w4a4_gemm_kernel<OUT_S32>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
+  using P = Plan<B_PACKED>;
+  auto kern = w4a4_gemm_kernel<B_PACKED, OUT_S32>;
+  static bool attr_set[64] = {};  // per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
   CUtensorMap tmA, tmB, tmY;
   const uint64_t kp = static_cast<uint64_t>(a.K / 2);
   if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qx, kp, a.M, kp, BKP, BM,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw, kp, a.N, kp, BKP, BN,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  const bool okB = B_PACKED ? make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw, kp, a.N, kp,
+                                          BKP, BN, CU_TENSOR_MAP_SWIZZLE_NONE)
+                            : make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw8, a.K, a.N,
+                                          a.K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!okB) return cudaErrorInvalidValue;
   if (OUT_S32) {
     tmY = tmA;  // unused
   } else if (!make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, a.N, a.M,
@@ -379,9 +457,9 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   const int num_n = a.N / BN;
   const int tiles = num_m * num_n;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  w4a4_gemm_kernel<OUT_S32><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(
-      tmA, tmB, tmY, a.scale_tok, a.scale_ch, a.bias, a.acc, static_cast<int>(a.M), a.N, num_n,
-      tiles, a.K / BK);
+  kern<<<grid, NUM_THREADS, P::SMEM_BYTES, st>>>(tmA, tmB, tmY, a.scale_tok, a.scale_ch, a.bias,
+                                                 a.colsum, a.acc, static_cast<int>(a.M), a.N, num_n,
+                                                 tiles, a.K / BK);
   return cudaGetLastError();
 }
 
@@ -389,7 +467,26 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
 
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st) {
   if (a.M <= 0) return cudaSuccess;
-  return a.acc ? launch_t<true>(a, st) : launch_t<false>(a, st);
+  const bool packed = (a.qw8 == nullptr);
+  if (a.acc) return packed ? launch_t<true, true>(a, st) : launch_t<false, true>(a, st);
+  return packed ? launch_t<true, false>(a, st) : launch_t<false, false>(a, st);
+}
+
+cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,
+                                  cudaStream_t st) {
+  expand_weights_kernel<<<(N + 7) / 8, 256, 0, st>>>(qw, N, K, qw8, colsum);
+  return cudaGetLastError();
+}
+
+unsigned int *status_word() {
+  static unsigned int *addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) == cudaSuccess) addr[dev] = static_cast<unsigned int *>(p);
+  }
+  return addr[dev];
 }
 
 cudaError_t read_status(unsigned int *out, cudaStream_t st) {

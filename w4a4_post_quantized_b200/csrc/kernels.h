@@ -21,7 +21,9 @@ cudaError_t launch_fill(float *out, int n, float v, cudaStream_t st);
 // gemm.cu
 struct GemmArgs {
   const uint8_t *qx;        // [M, K/2] packed int4
-  const uint8_t *qw;        // [N, K/2] packed int4
+  const uint8_t *qw;        // [N, K/2] packed int4 (used when qw8 == nullptr)
+  const int8_t *qw8;        // [N, K] widened weight codes, or nullptr
+  const int32_t *colsum;    // [N] per-row code sums (with qw8)
   const float *scale_tok;   // [M]
   const float *scale_ch;    // [N]
   const float *bias;        // [N]
@@ -31,8 +33,11 @@ struct GemmArgs {
   int N, K;
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
+cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,
+                                  cudaStream_t st);
 
-// status word
+// status word (device address of the current device's word, for kernel arguments)
+unsigned int *status_word();
 cudaError_t read_status(unsigned int *out, cudaStream_t st);
 cudaError_t clear_status(cudaStream_t st);
 

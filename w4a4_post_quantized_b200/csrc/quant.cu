@@ -27,6 +27,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace w4a4 {
 
@@ -45,20 +46,37 @@ __device__ __forceinline__ float gelu_bf16(float x) {
   return __bfloat162float(__float2bfloat16_rn(g));
 }
 
+// (a0, a1) <- (a0 + b0, a1 + b1), (b0, b1) <- (a0 - b0, a1 - b1) with the
+// packed fp32x2 add/sub of sm_100 (each lane rounded exactly as a scalar add).
+__device__ __forceinline__ void butterfly_x2(float &a0, float &a1, float &b0, float &b1) {
+  unsigned long long A, B, S, D;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(S) : "l"(A), "l"(B));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(B));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(S));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(D));
+}
+
 // Butterflies for index bits [B0, B0 + NB) of a register array (natural order:
-// the lower index of each pair receives the sum).
+// the lower index of each pair receives the sum).  Distances >= 2 process two
+// adjacent pairs per packed instruction.
 template <int V, int B0, int NB>
 __device__ __forceinline__ void butterflies(float (&v)[V]) {
 #pragma unroll
   for (int s = 0; s < NB; ++s) {
     const int h = 1 << (B0 + s);
+    if (h == 1) {
 #pragma unroll
-    for (int j = 0; j < V; ++j) {
-      if ((j & h) == 0) {
-        const float a = v[j], b = v[j + h];
+      for (int j = 0; j < V; j += 2) {
+        const float a = v[j], b = v[j + 1];
         v[j] = a + b;
-        v[j + h] = a - b;
+        v[j + 1] = a - b;
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < V; j += 2)
+        if ((j & h) == 0) butterfly_x2(v[j], v[j + 1], v[j + h], v[j + h + 1]);
     }
   }
 }
@@ -72,22 +90,27 @@ struct RowShape {
   static_assert(K == 1024 || K == 4096, "K must be 1024 or 4096");
 };
 
-// Loads one row in phase-1 layout, applies optional GELU, runs the full
-// transform (when ROT) and leaves the row in phase-2 layout in v.
-template <int K, bool ROT, bool GELU>
-__device__ __forceinline__ void load_transform_row(const uint16_t *__restrict__ xrow, int lane,
-                                                   float *__restrict__ tile,
-                                                   float (&v)[RowShape<K>::V]) {
+// Phase-1 load of one row: u[j] = x[lane + 32 j] (optional GELU).  `x` points
+// at the row in global or shared memory.
+template <int K, bool GELU, bool FROM_SMEM>
+__device__ __forceinline__ void load_phase1(const unsigned short *__restrict__ x, int lane,
+                                            float (&u)[RowShape<K>::V]) {
   constexpr int V = RowShape<K>::V;
-  constexpr int P = RowShape<K>::P;
-  const unsigned short *x = reinterpret_cast<const unsigned short *>(xrow);
-  float u[V];
 #pragma unroll
   for (int j = 0; j < V; ++j) {
-    float f = bf16_bits_to_float(__ldcs(x + lane + 32 * j));
+    float f = bf16_bits_to_float(FROM_SMEM ? x[lane + 32 * j] : __ldcs(x + lane + 32 * j));
     if (GELU) f = gelu_bf16(f);
     u[j] = f;
   }
+}
+
+// Runs the transform (when ROT) on a phase-1 row u and leaves it in phase-2
+// layout in v.
+template <int K, bool ROT>
+__device__ __forceinline__ void transform_row(float (&u)[RowShape<K>::V], int lane,
+                                              float *__restrict__ tile, float (&v)[RowShape<K>::V]) {
+  constexpr int V = RowShape<K>::V;
+  constexpr int P = RowShape<K>::P;
   if (ROT) butterflies<V, 0, RowShape<K>::LOGV>(u);  // index bits 5 .. log2(K)-1
   // transpose: value u[P*l2 + p] of lane l moves to lane l2, register 32p + l
 #pragma unroll
@@ -102,60 +125,132 @@ __device__ __forceinline__ void load_transform_row(const uint16_t *__restrict__ 
   if (ROT) butterflies<V, 0, 5>(v);  // index bits 0..4
 }
 
-// quantize_rows: one warp per row, grid-stride over rows.
+// Per-channel multiplier (from the block's shared table), per-row absmax,
+// codes, packed store for a phase-2 row.  The transform's 1/sqrt(K) is an
+// exact power of two, so it changes neither the absmax position nor any
+// code: it is applied to the stored step only.
+template <int K, bool ROT>
+__device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], int lane, int64_t row,
+                                                   const float4 *__restrict__ mtab,
+                                                   uint8_t *__restrict__ q, float *__restrict__ scale) {
+  constexpr int V = RowShape<K>::V;
+  if (ROT) {
+#pragma unroll
+    for (int c = 0; c < V / 4; ++c) {
+      const float4 m = mtab[c * 32 + lane];
+      v[4 * c + 0] *= m.x;
+      v[4 * c + 1] *= m.y;
+      v[4 * c + 2] *= m.z;
+      v[4 * c + 3] *= m.w;
+    }
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int r = 0; r < V; ++r) amax = fmaxf(amax, fabsf(v[r]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) scale[row] = (ROT ? amax * RowShape<K>::kInvSqrtK : amax) / 7.0f;
+  if (amax < 0x1p-100f) {  // keep 7/amax finite: exact power-of-two rescale, same codes
+#pragma unroll
+    for (int r = 0; r < V; ++r) v[r] *= 0x1p+64f;
+    amax *= 0x1p+64f;
+  }
+  const float inv = (amax > 0.0f) ? 7.0f / amax : 0.0f;
+  // code = round-half-even(v * inv); |v * inv| <= 7 (1 + 2^-24), so no clamp
+  // can ever act.  Adding 1.5 * 2^23 in the same fused operation rounds the
+  // exact product to an integer whose low 4 bits are the two's-complement code.
+  uint32_t words[V / 8];
+#pragma unroll
+  for (int w = 0; w < V / 8; ++w) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float f = fmaf(v[8 * w + k], inv, 12582912.0f);
+      acc |= (__float_as_uint(f) & 0xFu) << (4 * k);
+    }
+    words[w] = acc;
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(q + row * (K / 2) + static_cast<int64_t>(lane) * (V / 2));
+#pragma unroll
+  for (int c = 0; c < V / 32; ++c)
+    dst[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+}
+
+template <int K>
+struct QuantStaging {
+  static constexpr int ROWB = 2 * K;                 // bf16 row bytes
+  static constexpr int NS = 2;                        // rows in flight per warp
+  static constexpr int WARP_BYTES = NS * ROWB + 32 * 32 * 4;
+  static constexpr int OFF_TAB = kQuantWarps * WARP_BYTES;        // multiplier table, K floats
+  static constexpr int OFF_BAR = OFF_TAB + 4 * K;
+  static constexpr int SMEM = OFF_BAR + kQuantWarps * NS * 8;
+};
+
+// quantize_rows: one warp per row, grid-stride over rows.  Each warp keeps
+// NS rows in flight: 1-D bulk copies (TMA engine) stream its next rows into a
+// private shared-memory ring while it transforms the current one, so the HBM
+// latency is hidden without occupancy.
 template <int K, bool ROT, bool GELU>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_rows_kernel(const uint16_t *__restrict__ X, int64_t M, const float *__restrict__ mult,
-                         uint8_t *__restrict__ q, float *__restrict__ scale) {
+                         uint8_t *__restrict__ q, float *__restrict__ scale,
+                         unsigned int *__restrict__ status) {
+  using S = QuantStaging<K>;
   constexpr int V = RowShape<K>::V;
-  __shared__ float tiles[kQuantWarps][32 * 32];
+  extern __shared__ __align__(1024) uint8_t qsmem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  float *tile = tiles[warp];
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantWarps;
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kQuantWarps + warp; row < M; row += stride) {
-    float v[V];
-    load_transform_row<K, ROT, GELU>(X + row * K, lane, tile, v);
-    if (ROT) {
-      const float4 *m4 = reinterpret_cast<const float4 *>(mult + static_cast<int64_t>(V) * lane);
-#pragma unroll
-      for (int c = 0; c < V / 4; ++c) {
-        const float4 m = __ldg(m4 + c);
-        v[4 * c + 0] *= m.x * RowShape<K>::kInvSqrtK;
-        v[4 * c + 1] *= m.y * RowShape<K>::kInvSqrtK;
-        v[4 * c + 2] *= m.z * RowShape<K>::kInvSqrtK;
-        v[4 * c + 3] *= m.w * RowShape<K>::kInvSqrtK;
-      }
+  uint8_t *ring = qsmem + warp * S::WARP_BYTES;
+  float *tile = reinterpret_cast<float *>(ring + S::NS * S::ROWB);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(qsmem + S::OFF_BAR) + warp * S::NS;
+  float4 *mtab = reinterpret_cast<float4 *>(qsmem + S::OFF_TAB);
+  if (ROT) {
+    // table[(r/4)*32 + l] holds mult[V l + r .. +3]: lane l's 16-byte reads of
+    // one chunk are consecutive across the warp (conflict-free)
+    float *t = reinterpret_cast<float *>(mtab);
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      const int l = j / V, r = j % V;
+      t[((r >> 2) * 32 + l) * 4 + (r & 3)] = __ldg(mult + j);
     }
-    float amax = 0.0f;
-#pragma unroll
-    for (int r = 0; r < V; ++r) amax = fmaxf(amax, fabsf(v[r]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) scale[row] = amax / 7.0f;
-    // rows whose maximum is tiny are rescaled by an exact power of two so that
-    // 7/amax stays finite; the scaled product equals the unscaled one
-    const float pre = (amax < 0x1p-100f) ? 0x1p+100f : 1.0f;
-    const float inv = (amax > 0.0f) ? 7.0f / (amax * pre) : 0.0f;
-    // code = round-half-even(v * inv); |v * inv| <= 7 (1 + 2^-24), so no clamp
-    // can ever act.  Adding 1.5 * 2^23 in the same fused operation rounds the
-    // exact product to an integer whose low 4 bits are the two's-complement code.
-    uint32_t words[V / 8];
-#pragma unroll
-    for (int w = 0; w < V / 8; ++w) {
-      uint32_t acc = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float f = fmaf(v[8 * w + k] * pre, inv, 12582912.0f);
-        acc |= (__float_as_uint(f) & 0xFu) << (4 * k);
-      }
-      words[w] = acc;
-    }
-    uint4 *dst = reinterpret_cast<uint4 *>(q + row * (K / 2) + static_cast<int64_t>(lane) * (V / 2));
-#pragma unroll
-    for (int c = 0; c < V / 32; ++c)
-      dst[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+    __syncthreads();
   }
+  const int64_t G = static_cast<int64_t>(gridDim.x) * kQuantWarps;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kQuantWarps + warp;
+  int64_t issued = 0;  // rows whose copy lane 0 has issued (sequence numbers 0..issued-1)
+  if (lane == 0) {
+    for (int s = 0; s < S::NS; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    for (int s = 0; s < S::NS; ++s) {
+      const int64_t r = r0 + s * G;
+      if (r >= M) break;
+      mbar_arrive_expect_tx(&bars[s], S::ROWB);
+      bulk_load(ring + s * S::ROWB, X + r * K, S::ROWB, &bars[s]);
+      ++issued;
+    }
+  }
+  __syncwarp();
+  int64_t i = 0;
+  for (int64_t row = r0; row < M; row += G, ++i) {
+    const int s = static_cast<int>(i % S::NS);
+    if (!mbar_wait_drain(&bars[s], static_cast<uint32_t>((i / S::NS) & 1), status)) break;
+    float u[V], v[V];
+    load_phase1<K, GELU, true>(reinterpret_cast<const unsigned short *>(ring + s * S::ROWB), lane, u);
+    transform_row<K, ROT>(u, lane, tile, v);  // ends with __syncwarp: slot s is no longer read
+    if (lane == 0) {
+      const int64_t rn = row + S::NS * G;
+      if (rn < M) {
+        mbar_arrive_expect_tx(&bars[s], S::ROWB);
+        bulk_load(ring + s * S::ROWB, X + rn * K, S::ROWB, &bars[s]);
+        ++issued;
+      }
+    }
+    quantize_store_row<K, ROT>(v, lane, row, mtab, q, scale);
+  }
+  // after a timed-out wait, let the copies still in flight land before exiting
+  if (lane == 0)
+    for (int64_t k = i; k < issued; ++k)
+      mbar_wait_drain(&bars[k % S::NS], static_cast<uint32_t>((k / S::NS) & 1), status);
 }
 
 // colmax: colmax[j] = max over rows of |(x H / sqrt(K))[j]| (as float bits,
@@ -172,8 +267,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
   const int warp = threadIdx.x >> 5;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantWarps;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * kQuantWarps + warp; row < M; row += stride) {
-    float v[V];
-    load_transform_row<K, true, false>(X + row * K, lane, tiles[warp], v);
+    float u[V], v[V];
+    load_phase1<K, false, false>(reinterpret_cast<const unsigned short *>(X + row * K), lane, u);
+    transform_row<K, true>(u, lane, tiles[warp], v);
 #pragma unroll
     for (int r = 0; r < V; ++r)
       atomicMax(&cm[V * lane + r], __float_as_uint(fabsf(v[r] * RowShape<K>::kInvSqrtK)));
@@ -207,16 +303,16 @@ __global__ void fill_kernel(float *__restrict__ out, int n, float v) {
   if (i < n) out[i] = v;
 }
 
-int g_num_sms = 0;
-
 int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
+  static int sms[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (sms[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = n > 0 ? n : 148;
   }
-  return g_num_sms;
+  return sms[dev];
 }
 
 template <typename Kern>
@@ -233,8 +329,24 @@ template <int K, bool ROT, bool GELU>
 cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint8_t *q,
                            float *scale, cudaStream_t st) {
   auto kern = quantize_rows_kernel<K, ROT, GELU>;
-  const int grid = row_grid(kern, M);
-  kern<<<grid, kQuantWarps * 32, 0, st>>>(X, M, mult, q, scale);
+  constexpr int smem = QuantStaging<K>::SMEM;
+  static int per_sm_dev[64] = {};  // per device: attribute set and occupancy known
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  int &per_sm = per_sm_dev[dev];
+  if (per_sm == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kQuantWarps * 32, smem);
+    per_sm = n < 1 ? 1 : n;
+  }
+  const int64_t need = (M + kQuantWarps - 1) / kQuantWarps;
+  const int64_t g = static_cast<int64_t>(num_sms()) * per_sm;
+  const int grid = static_cast<int>(need < g ? need : g);
+  kern<<<grid, kQuantWarps * 32, smem, st>>>(X, M, mult, q, scale, status_word());
   return cudaGetLastError();
 }
 

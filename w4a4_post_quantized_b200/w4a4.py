@@ -34,7 +34,7 @@ _vp, _i32, _i64, _u32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_in
 
 class W4A4WeightsT(ctypes.Structure):
     _fields_ = [("N", _i32), ("K", _i32), ("qw", _vp), ("scale_ch", _vp), ("bias", _vp),
-                ("smooth", _vp), ("inv_smooth", _vp), ("flags", _u32)]
+                ("smooth", _vp), ("inv_smooth", _vp), ("qw8", _vp), ("colsum", _vp), ("flags", _u32)]
 
 
 def _sig(name, res, args):
@@ -51,7 +51,8 @@ _quantize = _sig("w4a4_quantize_act", ctypes.c_int, [_vp, _i64, _i32, _vp, _vp, 
 _linear = _sig("w4a4_linear", ctypes.c_int, [_vp, _vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp])
 _fused = _sig("w4a4_linear_fused", ctypes.c_int,
               [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp, _sz, _u32, _vp])
-_gemm_s32 = _sig("w4a4_gemm_s32", ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _vp, _vp])
+_gemm_s32 = _sig("w4a4_gemm_s32", ctypes.c_int, [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp])
+_expand = _sig("w4a4_expand_weights", ctypes.c_int, [ctypes.POINTER(W4A4WeightsT), _vp])
 _get_status = _sig("w4a4_get_device_status", ctypes.c_int, [_vp, ctypes.POINTER(_u32)])
 _clear_status = _sig("w4a4_clear_device_status", ctypes.c_int, [_vp])
 _status_string = _sig("w4a4_status_string", ctypes.c_char_p, [ctypes.c_int])
@@ -92,18 +93,24 @@ def w4a4_workspace_bytes(M: int, K: int) -> int:
 
 class PreparedWeights:
     """Device arrays of one prepared layer (owned by torch) and the C struct
-    that points at them."""
+    that points at them.  expanded=True also allocates the widened int8 copy
+    of the codes (qw8, N*K bytes) and the per-row code sums the fast GEMM
+    path uses; expanded=False keeps only the packed int4 codes."""
 
-    def __init__(self, N: int, K: int, device="cuda"):
+    def __init__(self, N: int, K: int, device="cuda", expanded: bool = True):
         self.N, self.K = N, K
         self.qw = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
         self.scale_ch = torch.empty(N, dtype=torch.float32, device=device)
         self.bias = torch.empty(N, dtype=torch.float32, device=device)
         self.smooth = torch.empty(K, dtype=torch.float32, device=device)
         self.inv_smooth = torch.empty(K, dtype=torch.float32, device=device)
+        self.qw8 = torch.empty((N, K), dtype=torch.int8, device=device) if expanded else None
+        self.colsum = torch.empty(N, dtype=torch.int32, device=device) if expanded else None
         self.struct = W4A4WeightsT(N, K, self.qw.data_ptr(), self.scale_ch.data_ptr(),
                                    self.bias.data_ptr(), self.smooth.data_ptr(),
-                                   self.inv_smooth.data_ptr(), 0)
+                                   self.inv_smooth.data_ptr(),
+                                   self.qw8.data_ptr() if expanded else None,
+                                   self.colsum.data_ptr() if expanded else None, 0)
 
     @property
     def flags(self) -> int:
@@ -111,9 +118,10 @@ class PreparedWeights:
 
 
 def w4a4_prepare_weights(W: torch.Tensor, bias, X_calib, alpha: float = 0.5, flags: int = 0,
-                         out: PreparedWeights | None = None, stream=None) -> PreparedWeights:
+                         out: PreparedWeights | None = None, expanded: bool = True,
+                         stream=None) -> PreparedWeights:
     N, K = W.shape
-    out = out or PreparedWeights(N, K, W.device)
+    out = out or PreparedWeights(N, K, W.device, expanded=expanded)
     mc = 0 if X_calib is None else X_calib.shape[0]
     _check(_prepare(_ptr(W), _ptr(bias), N, K, _ptr(X_calib), mc, alpha, flags,
                     ctypes.byref(out.struct), _stream(stream)), "w4a4_prepare_weights")
@@ -151,11 +159,15 @@ def w4a4_linear_fused(X: torch.Tensor, w: PreparedWeights, Y=None, workspace=Non
     return Y
 
 
-def w4a4_gemm_s32(qx: torch.Tensor, qw: torch.Tensor, acc=None, stream=None):
-    M, KP = qx.shape
-    N = qw.shape[0]
-    acc = acc if acc is not None else torch.empty((M, N), dtype=torch.int32, device=qx.device)
-    _check(_gemm_s32(_ptr(qx), _ptr(qw), M, N, 2 * KP, _ptr(acc), _stream(stream)), "w4a4_gemm_s32")
+def w4a4_expand_weights(w: PreparedWeights, stream=None) -> PreparedWeights:
+    _check(_expand(ctypes.byref(w.struct), _stream(stream)), "w4a4_expand_weights")
+    return w
+
+
+def w4a4_gemm_s32(qx: torch.Tensor, w: PreparedWeights, acc=None, stream=None):
+    M = qx.shape[0]
+    acc = acc if acc is not None else torch.empty((M, w.N), dtype=torch.int32, device=qx.device)
+    _check(_gemm_s32(_ptr(qx), M, ctypes.byref(w.struct), _ptr(acc), _stream(stream)), "w4a4_gemm_s32")
     return acc
 
 
