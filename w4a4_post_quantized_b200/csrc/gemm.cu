@@ -27,9 +27,10 @@
 //   warp 1      tcgen05.mma issuer (one thread)
 //   warp 2      tensor-memory allocator
 //   warps 4..7  widen packed int4 -> int8 into the swizzled operand tiles
-//   warps 8..11 epilogue: tcgen05.ld accumulators, subtract the code-offset
-//               term, scale by scale_tok[m] * scale_ch[n], add bias in fp32,
-//               round to bf16, TMA-store through a swizzled staging buffer.
+//   warps 8..11 epilogue: tcgen05.ld accumulators (64 columns at a time),
+//               subtract the code-offset term, scale by scale_tok[m] *
+//               scale_ch[n], add bias in fp32, round to bf16, TMA-store
+//               32 x 64 tiles through a 128-byte-swizzled staging buffer.
 // Accumulators are double-buffered in tensor memory (2 x 256 columns) so the
 // epilogue of one tile overlaps the main loop of the next.
 //
@@ -62,31 +63,39 @@ constexpr int BM = 128;   // tile rows (tokens)
 constexpr int BN = 256;   // tile columns (output channels)
 constexpr int BK = 128;   // int8 elements per k-block = one 128-byte swizzle row
 constexpr int BKP = 64;   // packed bytes per row per k-block
-constexpr int A_PK = BM * BKP;  // 8 KB
-constexpr int B_PK = BN * BKP;  // 16 KB
-constexpr int A_UN = BM * BK;   // 16 KB
-constexpr int B_UN = BN * BK;   // 32 KB
-constexpr int EPI_BYTES = 32 * 32 * 2;  // one warp's 32 x 32 bf16 staging tile
-constexpr int NUM_THREADS = 384;
+constexpr int A_PK = BM * BKP;   // 8 KB
+constexpr int B_PK = BN * BKP;   // 16 KB
+constexpr int A_UN = BM * BK;    // 16 KB
+constexpr int B_UN = BN * BK;    // 32 KB
+constexpr int EPI_COLS = 64;             // output columns per epilogue store
+constexpr int EPI_BYTES = 32 * EPI_COLS * 2;  // one warp's 32 x 64 bf16 staging tile (128-byte rows)
+constexpr int NUM_EPI_WARPS = 4;        // one per TMEM lane quadrant
+constexpr int NUM_THREADS = (8 + NUM_EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;     // two 128 x 256 s32 accumulators
 
-// Shared-memory plan, per pipeline stage.
+// Shared-memory plan.  TMA stages hold what comes from L2 (packed A, and B as
+// int8 or packed); a ring of widened slots holds the int8 operand tiles
+// produced in shared memory (A, and B when packed).
 template <bool B_PACKED>
 struct Plan {
-  static constexpr int STAGES = B_PACKED ? 2 : 3;
-  static constexpr int OFF_A_PK = 0;
-  static constexpr int OFF_B_PK = A_PK;                                  // B_PACKED only
-  static constexpr int OFF_A_UN = B_PACKED ? A_PK + B_PK : A_PK;
-  static constexpr int OFF_B_UN = OFF_A_UN + A_UN;
-  static constexpr int STAGE_BYTES = OFF_B_UN + B_UN;
-  static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
-  static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BYTES;
-  static constexpr int NUM_BARS = 3 * STAGES + 2 * 2 + 1;
+  static constexpr int STAGES = 3;                   // TMA stages
+  static constexpr int WSLOTS = 2;                   // widened operand slots
+  static constexpr int OFF_ST_A = 0;                 // packed A  [BM x 64 B]
+  static constexpr int OFF_ST_B = A_PK;              // B: int8 [BN x 128 B] (swizzled) or packed
+  static constexpr int STAGE_BYTES = A_PK + (B_PACKED ? B_PK : B_UN);
+  static constexpr int OFF_W = STAGES * STAGE_BYTES;
+  static constexpr int OFF_W_A = 0;                  // widened A [BM x 128 B] (swizzled)
+  static constexpr int OFF_W_B = A_UN;               // widened B (B_PACKED only)
+  static constexpr int WSLOT_BYTES = A_UN + (B_PACKED ? B_UN : 0);
+  static constexpr int OFF_EPI = OFF_W + WSLOTS * WSLOT_BYTES;
+  static constexpr int OFF_COL = OFF_EPI + NUM_EPI_WARPS * 2 * EPI_BYTES;  // per-warp constants
+  static constexpr int OFF_BAR = OFF_COL + NUM_EPI_WARPS * 3 * BN * 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * WSLOTS + 2 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(OFF_A_UN % 1024 == 0 && OFF_B_UN % 1024 == 0 && STAGE_BYTES % 1024 == 0 &&
-                    OFF_EPI % 1024 == 0,
+  static_assert(OFF_ST_B % 1024 == 0 && STAGE_BYTES % 1024 == 0 && OFF_W % 1024 == 0 &&
+                    WSLOT_BYTES % 1024 == 0 && OFF_EPI % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
   // tcgen05.mma kind::i8 instruction descriptor: s32 D; A unsigned (code + 8)
   // with expanded B, signed with packed B; B signed; both K-major; 128 x 256.
@@ -97,7 +106,7 @@ struct Plan {
 
 constexpr int W_TMA = 0, W_MMA = 1, W_TMEM = 2;
 constexpr int W_UNPACK0 = 4;  // warps 4..7
-constexpr int W_EPI0 = 8;     // warps 8..11 (warp % 4 selects its 32 TMEM lanes)
+constexpr int W_EPI0 = 8;     // warps 8..11: warp % 4 selects its 32 TMEM lanes
 
 // 4 nibbles (one per byte, 0..15 = two's-complement int4) -> 4 signed int8.
 __device__ __forceinline__ uint32_t sext4x4(uint32_t n) {
@@ -146,11 +155,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// int32 -> float for |x| < 2^22, exact: the bit pattern 0x4B400000 + x is the
-// float 1.5 * 2^23 + x.
-__device__ __forceinline__ float small_int_to_float(int32_t biased_bits) {
-  return __int_as_float(biased_bits) - 12582912.0f;
+// Packed fp32x2 arithmetic of sm_100 (each lane rounded as the scalar op).
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
 }
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// Dequantize two accumulators given as biased bit patterns (0x4B400000 + acc,
+// i.e. the floats 1.5 * 2^23 + acc, exact for |acc| < 2^22):
+//   y = (float(bits) - 1.5 * 2^23) * (st * sc) + bias, all in fp32.
+__device__ __forceinline__ uint32_t dequant2_bf16(int32_t b0, int32_t b1, float st, float sc0,
+                                                  float sc1, float bi0, float bi1) {
+  const unsigned long long x = f2_pack(__int_as_float(b0), __int_as_float(b1));
+  const unsigned long long magic = f2_pack(12582912.0f, 12582912.0f);
+  const unsigned long long s = f2_pack(st, st), c = f2_pack(sc0, sc1), b = f2_pack(bi0, bi1);
+  unsigned long long a, m, y;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(a) : "l"(x), "l"(magic));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(m) : "l"(s), "l"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(y) : "l"(a), "l"(m), "l"(b));
+  float y0, y1;
+  f2_unpack(y, y0, y1);
+  return pack_bf16x2(y0, y1);
+}
+
 
 template <bool B_PACKED, bool OUT_S32>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -161,15 +192,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      int num_n_tiles, int num_tiles, int num_kb) {
   using P = Plan<B_PACKED>;
   constexpr int ST = P::STAGES;
+  constexpr int WS = P::WSLOTS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + P::OFF_BAR);
-  uint64_t *full = bars;            // TMA bytes landed
-  uint64_t *widened = full + ST;    // operand tiles ready for the tensor core
-  uint64_t *freed = widened + ST;   // MMAs reading the stage have completed
-  uint64_t *acc_full = freed + ST;
-  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *full = bars;             // TMA bytes of a stage landed
+  uint64_t *freed = full + ST;       // MMAs reading a stage completed
+  uint64_t *wready = freed + ST;     // widened slot written (one arrival per widen warp)
+  uint64_t *wfree = wready + WS;     // MMAs reading a widened slot completed
+  uint64_t *acc_full = wfree + WS;   // accumulator buffer complete
+  uint64_t *acc_empty = acc_full + 2;  // epilogue drained an accumulator buffer
   uint64_t *mma_done = acc_empty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + P::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + P::OFF_MISC + 4);
@@ -180,12 +213,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&widened[s], 128);
       mbar_init(&freed[s], 1);
+    }
+    for (int u = 0; u < WS; ++u) {
+      mbar_init(&wready[u], 4);
+      mbar_init(&wfree[u], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], NUM_EPI_WARPS);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -219,12 +255,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           uint8_t *stage = smem + s * P::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], A_PK + (B_PACKED ? B_PK : B_UN));
-          tma_load_2d(stage + P::OFF_A_PK, &tmA, kb * BKP, mb * BM, &full[s]);
-          if (B_PACKED)
-            tma_load_2d(stage + P::OFF_B_PK, &tmB, kb * BKP, nb * BN, &full[s]);
-          else
-            tma_load_2d(stage + P::OFF_B_UN, &tmB, kb * BK, nb * BN, &full[s]);
+          mbar_arrive_expect_tx(&full[s], P::STAGE_BYTES);
+          tma_load_2d(stage + P::OFF_ST_A, &tmA, kb * BKP, mb * BM, &full[s]);
+          tma_load_2d(stage + P::OFF_ST_B, &tmB, B_PACKED ? kb * BKP : kb * BK, nb * BN, &full[s]);
           ++issued;
         }
       }
@@ -244,19 +277,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
-          const uint32_t s = consumed % ST, ps = (consumed / ST) & 1u;
-          if (!mbar_wait(&widened[s], ps, abort_flag, &g_status)) {
+          const uint32_t s = consumed % ST;
+          const uint32_t u = consumed % WS, pu = (consumed / WS) & 1u;
+          // the widen warps waited for the stage's TMA bytes before signalling wready
+          if (!mbar_wait(&wready[u], pu, abort_flag, &g_status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_A_UN);
-          const uint32_t b0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_B_UN);
+          uint8_t *slot = smem + P::OFF_W + u * P::WSLOT_BYTES;
+          const uint32_t a0 = smem_u32(slot + P::OFF_W_A);
+          const uint32_t b0 = smem_u32(B_PACKED ? slot + P::OFF_W_B
+                                                : smem + s * P::STAGE_BYTES + P::OFF_ST_B);
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
             mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), P::IDESC,
                    (kb | kk) != 0 ? 1u : 0u);
           tc_commit(&freed[s]);
+          tc_commit(&wfree[u]);
           ++consumed;
         }
         if (ok) tc_commit(&acc_full[b]);
@@ -273,81 +311,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb, ++n) {
         const uint32_t s = n % ST, ps = (n / ST) & 1u;
-        if (!mbar_wait(&full[s], ps, abort_flag, &g_status)) {
+        const uint32_t u = n % WS, pu = (n / WS) & 1u;
+        if (!mbar_wait(&full[s], ps, abort_flag, &g_status) ||
+            !mbar_wait(&wfree[u], pu ^ 1u, abort_flag, &g_status)) {
           ok = false;
           break;
         }
         uint8_t *stage = smem + s * P::STAGE_BYTES;
-        widen_tile<A_PK / 16 / 128, B_PACKED>(stage + P::OFF_A_PK, stage + P::OFF_A_UN, t);
-        if (B_PACKED) widen_tile<B_PK / 16 / 128, true>(stage + P::OFF_B_PK, stage + P::OFF_B_UN, t);
+        uint8_t *slot = smem + P::OFF_W + u * P::WSLOT_BYTES;
+        widen_tile<A_PK / 16 / 128, B_PACKED>(stage + P::OFF_ST_A, slot + P::OFF_W_A, t);
+        if (B_PACKED) widen_tile<B_PK / 16 / 128, true>(stage + P::OFF_ST_B, slot + P::OFF_W_B, t);
         fence_proxy_async_smem();
-        mbar_arrive(&widened[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wready[u]);
       }
     }
   } else if (warp >= W_EPI0) {
     // ---------------------------------------------------------------- epilogue
     const int ew = warp - W_EPI0;  // == warp % 4: owns TMEM lanes 32 ew .. 32 ew + 31
+    // this warp's copy of the tile's per-column constants:
+    //   off[n] = 0x4B400000 - 8 colsum[n] (the code-offset correction folded
+    //   into the exact int -> float bias), sc[n], bias[n]
+    int32_t *coff = reinterpret_cast<int32_t *>(smem + P::OFF_COL) + ew * 3 * BN;
+    float *csc = reinterpret_cast<float *>(coff + BN);
+    float *cbi = csc + BN;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const uint32_t b = it & 1, pb = (it >> 1) & 1;
+      const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
+      __syncwarp();  // every lane is done reading the previous tile's constants
+#pragma unroll
+      for (int j = lane; j < BN; j += 32) {
+        const int n = nb * BN + j;
+        coff[j] = 0x4B400000 - (B_PACKED ? 0 : 8 * __ldg(colsum + n));
+        if (!OUT_S32) {
+          csc[j] = __ldg(scale_ch + n);
+          cbi[j] = __ldg(bias + n);
+        }
+      }
+      __syncwarp();
       if (!mbar_wait(&acc_full[b], pb, abort_flag, &g_status)) break;
       tc_fence_after();
-      const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
       const int row0 = mb * BM + ew * 32;
       const int m = row0 + lane;
       const float st = (!OUT_S32 && m < M) ? __ldg(scale_tok + m) : 0.0f;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * BN;
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + ch * 32, r);
+      for (int sc = 0; sc < BN / EPI_COLS; ++sc) {
+        // 64 accumulator columns of this warp's 32 rows: two loads, one wait
+        uint32_t r[64];
+        tmem_ld_32x32b_x32(tbase + sc * EPI_COLS, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld_32x32b_x32(tbase + sc * EPI_COLS + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_wait_ld();
-        if (ch == BN / 32 - 1) {
+        if (sc == BN / EPI_COLS - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
-        const int n0 = nb * BN + ch * 32;
-        // biased[j] = bit pattern 0x4B400000 + acc[m, n0 + j] (exact integer arithmetic)
-        int32_t biased[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          int4 off = make_int4(0, 0, 0, 0);
-          if (!B_PACKED) off = __ldg(reinterpret_cast<const int4 *>(colsum + n0) + c);
-          biased[4 * c + 0] = static_cast<int32_t>(r[4 * c + 0]) - 8 * off.x + 0x4B400000;
-          biased[4 * c + 1] = static_cast<int32_t>(r[4 * c + 1]) - 8 * off.y + 0x4B400000;
-          biased[4 * c + 2] = static_cast<int32_t>(r[4 * c + 2]) - 8 * off.z + 0x4B400000;
-          biased[4 * c + 3] = static_cast<int32_t>(r[4 * c + 3]) - 8 * off.w + 0x4B400000;
-        }
+        const int c0 = sc * EPI_COLS;
+        const int n0 = nb * BN + c0;
+        const int4 *off4 = reinterpret_cast<const int4 *>(coff + c0);
         if (OUT_S32) {
           if (m < M) {
             int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(m) * N + n0);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              dst[c] = make_int4(biased[4 * c] - 0x4B400000, biased[4 * c + 1] - 0x4B400000,
-                                 biased[4 * c + 2] - 0x4B400000, biased[4 * c + 3] - 0x4B400000);
+            for (int c = 0; c < EPI_COLS / 4; ++c) {
+              const int4 o = off4[c];
+              dst[c] = make_int4(static_cast<int32_t>(r[4 * c + 0]) + o.x - 0x4B400000,
+                                 static_cast<int32_t>(r[4 * c + 1]) + o.y - 0x4B400000,
+                                 static_cast<int32_t>(r[4 * c + 2]) + o.z - 0x4B400000,
+                                 static_cast<int32_t>(r[4 * c + 3]) + o.w - 0x4B400000);
+            }
           }
         } else {
-          uint32_t pk[16];
-          const float4 *sc4 = reinterpret_cast<const float4 *>(scale_ch + n0);
-          const float4 *bi4 = reinterpret_cast<const float4 *>(bias + n0);
+          uint32_t pk[EPI_COLS / 2];
+          const float4 *sc4 = reinterpret_cast<const float4 *>(csc + c0);
+          const float4 *bi4 = reinterpret_cast<const float4 *>(cbi + c0);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float4 sc = __ldg(sc4 + c), bi = __ldg(bi4 + c);
-            const float y0 = fmaf(small_int_to_float(biased[4 * c + 0]), st * sc.x, bi.x);
-            const float y1 = fmaf(small_int_to_float(biased[4 * c + 1]), st * sc.y, bi.y);
-            const float y2 = fmaf(small_int_to_float(biased[4 * c + 2]), st * sc.z, bi.z);
-            const float y3 = fmaf(small_int_to_float(biased[4 * c + 3]), st * sc.w, bi.w);
-            pk[2 * c] = pack_bf16x2(y0, y1);
-            pk[2 * c + 1] = pack_bf16x2(y2, y3);
+          for (int c = 0; c < EPI_COLS / 4; ++c) {
+            const int4 o = off4[c];
+            const float4 scl = sc4[c], bi = bi4[c];
+            pk[2 * c] = dequant2_bf16(static_cast<int32_t>(r[4 * c + 0]) + o.x,
+                                      static_cast<int32_t>(r[4 * c + 1]) + o.y, st, scl.x, scl.y,
+                                      bi.x, bi.y);
+            pk[2 * c + 1] = dequant2_bf16(static_cast<int32_t>(r[4 * c + 2]) + o.z,
+                                          static_cast<int32_t>(r[4 * c + 3]) + o.w, st, scl.z, scl.w,
+                                          bi.z, bi.w);
           }
-          uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (ch & 1)) * EPI_BYTES;
+          uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (sc & 1)) * EPI_BYTES;
           if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
           __syncwarp();
+          // row = lane: 128 bytes = 8 chunks of 16 B, chunk u at (u ^ (row % 8)) (128-byte swizzle)
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4 *>(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4 *>(stg + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && row0 < M) {
@@ -450,7 +508,7 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   if (OUT_S32) {
     tmY = tmA;  // unused
   } else if (!make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, a.N, a.M,
-                          static_cast<uint64_t>(a.N) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) {
+                          static_cast<uint64_t>(a.N) * 2, EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_128B)) {
     return cudaErrorInvalidValue;
   }
   const int num_m = static_cast<int>((a.M + BM - 1) / BM);

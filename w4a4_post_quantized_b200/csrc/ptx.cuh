@@ -40,14 +40,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
+// Longest a waiting thread stays parked in one try_wait before it re-checks
+// the abort flag and its deadline (it wakes earlier when the phase completes).
+constexpr uint32_t kSuspendHintNs = 20000;
+
+// Test for completion of the phase with the given parity; a thread whose phase
+// is not complete is suspended by the hardware until it completes or the hint
+// runs out, so waiting costs no issue slots or shared-memory bandwidth.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -61,15 +68,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        atomicOr(status, 1u);
-        *abort = 1;
-        return false;
-      }
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      atomicOr(status, 1u);
+      *abort = 1;
+      return false;
     }
   }
 }
@@ -79,6 +84,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
                                                 unsigned int *status) {
   const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(a, parity)) {
     if (globaltimer() - t0 > kWaitLimitNs) {
