@@ -153,6 +153,32 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
                               void *workspace, size_t workspace_bytes, uint32_t flags,
                               void *stream);
 
+/* Size of the scratch array built into the library for
+ * w4a4_linear_fused_noalloc (8 MiB on every GPU that loads the library). */
+#define W4A4_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* w4a4_linear_fused for callers that cannot allocate device memory.  No page
+ * describes this; it serves callers that may not call cudaMalloc / cudaFree
+ * where they run (cudaFree synchronizes the whole device; a serving loop with a
+ * fixed memory budget or a plugin host's enqueue callback may forbid any
+ * allocation after start-up) or that only hold the input and output buffers
+ * another runtime handed them.  Same arguments and result as
+ * w4a4_linear_fused without the workspace: the codes and steps go to a scratch
+ * array of W4A4_NOALLOC_SCRATCH_BYTES inside the library instead, so the call
+ * allocates nothing.
+ *   - Accepts M with w4a4_workspace_bytes(M, w->K) <= W4A4_NOALLOC_SCRATCH_BYTES
+ *     (M <= 16256 tokens at K = 1024, M <= 4088 at K = 4096); larger M returns
+ *     W4A4_ERR_SHAPE.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one scratch array, which keeps the
+ *     last call's contents: calls that may overlap on the GPU (different
+ *     streams without ordering between them) race on it and must not be
+ *     issued. */
+w4a4_status w4a4_linear_fused_noalloc(const uint16_t *X, int64_t M, const w4a4_weights_t *w,
+                                      uint16_t *Y, uint32_t flags, void *stream);
+
 /* Integer product only: acc [M, N] int32 = sum_k qx[m, k] * code_w[n, k] for
  * packed activation codes qx [M, K/2] and the weight codes of *w (w->qw8 and
  * w->colsum when set, else the packed w->qw; scale_ch, bias and the smoothing

@@ -51,6 +51,8 @@ _quantize = _sig("w4a4_quantize_act", ctypes.c_int, [_vp, _i64, _i32, _vp, _vp, 
 _linear = _sig("w4a4_linear", ctypes.c_int, [_vp, _vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp])
 _fused = _sig("w4a4_linear_fused", ctypes.c_int,
               [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp, _sz, _u32, _vp])
+_fused_noalloc = _sig("w4a4_linear_fused_noalloc", ctypes.c_int,
+                      [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _u32, _vp])
 _gemm_s32 = _sig("w4a4_gemm_s32", ctypes.c_int, [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp])
 _expand = _sig("w4a4_expand_weights", ctypes.c_int, [ctypes.POINTER(W4A4WeightsT), _vp])
 _get_status = _sig("w4a4_get_device_status", ctypes.c_int, [_vp, ctypes.POINTER(_u32)])
@@ -156,6 +158,23 @@ def w4a4_linear_fused(X: torch.Tensor, w: PreparedWeights, Y=None, workspace=Non
     _check(_fused(_ptr(X), M, ctypes.byref(w.struct), _ptr(Y), _ptr(workspace),
                   workspace.numel() * workspace.element_size(), flags, _stream(stream)),
            "w4a4_linear_fused")
+    return Y
+
+
+W4A4_NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def w4a4_linear_fused_noalloc(X: torch.Tensor, w: PreparedWeights, Y=None, flags: int = 0,
+                              stream=None):
+    """w4a4_linear_fused without a workspace argument, for callers that may
+    not allocate device memory where they run: the library's built-in scratch
+    array (W4A4_NOALLOC_SCRATCH_BYTES per GPU) holds the intermediate codes.
+    Calls that overlap on the GPU share that array and must not be issued."""
+    M = X.shape[0]
+    if Y is None:  # allocating the output here is a convenience of this binding only
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    _check(_fused_noalloc(_ptr(X), M, ctypes.byref(w.struct), _ptr(Y), flags, _stream(stream)),
+           "w4a4_linear_fused_noalloc")
     return Y
 
 
