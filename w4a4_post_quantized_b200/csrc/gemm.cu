@@ -13,26 +13,32 @@
 //     are static, so their int4 codes are widened once, at preparation time,
 //     into qw8 [N, K] int8 in exactly the order the kernel widens A.  The
 //     kernel TMA-loads B tiles straight into the 128-byte swizzled operand
-//     layout.  A is TMA-staged packed and widened in shared memory as the
-//     unsigned value code + 8 (a nibble XOR), which costs 3 integer ops per 8
-//     codes; sum_k (qa + 8) qb = acc + 8 * colsum[n], so the epilogue
-//     subtracts 8 * colsum[n] (colsum = per-output-channel sum of the weight
-//     codes, prepared with qw8).  The result is exact.
+//     layout.  A is TMA-staged packed; the widen warps turn each row into the
+//     unsigned values code + 8 (a nibble XOR, 3 integer ops per 8 codes) in
+//     registers and store them into tensor memory (tcgen05.st), and the MMA
+//     reads A from there, so shared memory carries only the packed A and B.
+//     sum_k (qa + 8) qb = acc + 8 * colsum[n], so the epilogue subtracts
+//     8 * colsum[n] (colsum = per-output-channel sum of the weight codes,
+//     prepared with qw8).  The result is exact.  Tiles are 128 x 192 (the
+//     last column tile of an N that is not a multiple of 192 is partly
+//     outside the matrix: TMA fills those B rows with zeros and clips the
+//     stores).
 //   * packed B (qw8 == NULL): both operands are TMA-staged packed and
 //     sign-extended to int8 in shared memory on every tile (no extra weight
-//     memory, more shared-memory traffic and integer work).
+//     memory, more shared-memory traffic and integer work); tiles 128 x 256.
 //
 // Warp roles (one persistent CTA per SM, tiles round-robin, M-major):
 //   warp 0      TMA producer (one thread)
 //   warp 1      tcgen05.mma issuer (one thread)
 //   warp 2      tensor-memory allocator
-//   warps 4..7  widen packed int4 -> int8 into the swizzled operand tiles
+//   warps 4..7  widen packed int4 -> int8 (into tensor memory, or into the
+//               swizzled shared-memory operand tiles of the packed-B path)
 //   warps 8..11 epilogue: tcgen05.ld accumulators (64 columns at a time),
 //               subtract the code-offset term, scale by scale_tok[m] *
 //               scale_ch[n], add bias in fp32, round to bf16, TMA-store
 //               32 x 64 tiles through a 128-byte-swizzled staging buffer.
-// Accumulators are double-buffered in tensor memory (2 x 256 columns) so the
-// epilogue of one tile overlaps the main loop of the next.
+// Accumulators are double-buffered in tensor memory so the epilogue of one
+// tile overlaps the main loop of the next.
 //
 // Widening permutes K inside every group of 8 codes (even codes first, then
 // odd ones).  A and B use the same order, so every dot product sums the same
@@ -60,7 +66,7 @@ __device__ unsigned int g_status = 0;
 namespace {
 
 constexpr int BM = 128;   // tile rows (tokens)
-constexpr int BN = 256;   // tile columns (output channels)
+constexpr int BN = 256;   // tile columns (output channels) of the packed-B path
 constexpr int BK = 128;   // int8 elements per k-block = one 128-byte swizzle row
 constexpr int BKP = 64;   // packed bytes per row per k-block
 constexpr int A_PK = BM * BKP;   // 8 KB
@@ -71,25 +77,35 @@ constexpr int EPI_COLS = 64;             // output columns per epilogue store
 constexpr int EPI_BYTES = 32 * EPI_COLS * 2;  // one warp's 32 x 64 bf16 staging tile (128-byte rows)
 constexpr int NUM_EPI_WARPS = 4;        // one per TMEM lane quadrant
 constexpr int NUM_THREADS = (8 + NUM_EPI_WARPS) * 32;
-constexpr uint32_t TMEM_COLS = 512;     // two 128 x 256 s32 accumulators
+constexpr uint32_t TMEM_COLS = 512;     // the whole tensor memory of the SM
 
-// Shared-memory plan.  TMA stages hold what comes from L2 (packed A, and B as
-// int8 or packed); a ring of widened slots holds the int8 operand tiles
-// produced in shared memory (A, and B when packed).
+// Shared-memory and tensor-memory plan.  TMA stages hold what comes from L2
+// (packed A, and B as int8 or packed).
+//   expanded B: A is widened into tensor memory (the MMA reads A there), so
+//     shared memory carries only B and the packed A.  Tiles are 128 x 192:
+//     two 192-column accumulators and two widened-A slots of KG k-blocks
+//     (32 columns each) fill the 512 columns.
+//   packed B: A and B are widened into a ring of shared-memory slots; tiles
+//     are 128 x 256.
 template <bool B_PACKED>
 struct Plan {
-  static constexpr int STAGES = 3;                   // TMA stages
-  static constexpr int WSLOTS = 2;                   // widened operand slots
+  static constexpr bool A_TMEM = !B_PACKED;
+  static constexpr int TN = B_PACKED ? BN : 192;     // tile columns
+  static constexpr int STAGES = B_PACKED ? 3 : 5;    // TMA stages
+  static constexpr int KG = B_PACKED ? 1 : 2;        // k-blocks per widen -> MMA handshake
+  static constexpr int WSLOTS = B_PACKED ? 2 : 2;    // widened operand slots
   static constexpr int OFF_ST_A = 0;                 // packed A  [BM x 64 B]
-  static constexpr int OFF_ST_B = A_PK;              // B: int8 [BN x 128 B] (swizzled) or packed
-  static constexpr int STAGE_BYTES = A_PK + (B_PACKED ? B_PK : B_UN);
+  static constexpr int OFF_ST_B = A_PK;              // B: int8 [TN x 128 B] (swizzled) or packed
+  static constexpr int STAGE_BYTES = A_PK + (B_PACKED ? B_PK : TN * BK);
   static constexpr int OFF_W = STAGES * STAGE_BYTES;
   static constexpr int OFF_W_A = 0;                  // widened A [BM x 128 B] (swizzled)
   static constexpr int OFF_W_B = A_UN;               // widened B (B_PACKED only)
-  static constexpr int WSLOT_BYTES = A_UN + (B_PACKED ? B_UN : 0);
+  static constexpr int WSLOT_BYTES = A_TMEM ? 0 : A_UN + (B_PACKED ? B_UN : 0);
+  static constexpr uint32_t TMEM_A0 = 2 * TN;        // first widened-A column (A_TMEM)
+  static_assert(!A_TMEM || TMEM_A0 + WSLOTS * KG * 32 <= 512, "tensor-memory budget");
   static constexpr int OFF_EPI = OFF_W + WSLOTS * WSLOT_BYTES;
   static constexpr int OFF_COL = OFF_EPI + NUM_EPI_WARPS * 2 * EPI_BYTES;  // per-warp constants
-  static constexpr int OFF_BAR = OFF_COL + NUM_EPI_WARPS * 3 * BN * 4;
+  static constexpr int OFF_BAR = OFF_COL + NUM_EPI_WARPS * 3 * TN * 4;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * WSLOTS + 2 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024
@@ -98,9 +114,9 @@ struct Plan {
                     WSLOT_BYTES % 1024 == 0 && OFF_EPI % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
   // tcgen05.mma kind::i8 instruction descriptor: s32 D; A unsigned (code + 8)
-  // with expanded B, signed with packed B; B signed; both K-major; 128 x 256.
+  // with expanded B, signed with packed B; B signed; both K-major; 128 x TN.
   static constexpr uint32_t IDESC = (2u << 4) | ((B_PACKED ? 1u : 0u) << 7) | (1u << 10) |
-                                    (static_cast<uint32_t>(BN >> 3) << 17) |
+                                    (static_cast<uint32_t>(TN >> 3) << 17) |
                                     (static_cast<uint32_t>(BM >> 4) << 24);
 };
 
@@ -257,7 +273,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t *stage = smem + s * P::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[s], P::STAGE_BYTES);
           tma_load_2d(stage + P::OFF_ST_A, &tmA, kb * BKP, mb * BM, &full[s]);
-          tma_load_2d(stage + P::OFF_ST_B, &tmB, B_PACKED ? kb * BKP : kb * BK, nb * BN, &full[s]);
+          tma_load_2d(stage + P::OFF_ST_B, &tmB, B_PACKED ? kb * BKP : kb * BK, nb * P::TN, &full[s]);
           ++issued;
         }
       }
@@ -268,34 +284,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == W_MMA) {
     if (lane == 0) {
       // ------------------------------------------------------------- MMA issuer
-      uint32_t consumed = 0;
+      uint32_t consumed = 0, group = 0;
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
         const uint32_t b = it & 1, pb = (it >> 1) & 1;
         if (!mbar_wait(&acc_empty[b], pb ^ 1u, abort_flag, &g_status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + b * BN;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          const uint32_t s = consumed % ST;
-          const uint32_t u = consumed % WS, pu = (consumed / WS) & 1u;
-          // the widen warps waited for the stage's TMA bytes before signalling wready
-          if (!mbar_wait(&wready[u], pu, abort_flag, &g_status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uint8_t *slot = smem + P::OFF_W + u * P::WSLOT_BYTES;
-          const uint32_t a0 = smem_u32(slot + P::OFF_W_A);
-          const uint32_t b0 = smem_u32(B_PACKED ? slot + P::OFF_W_B
-                                                : smem + s * P::STAGE_BYTES + P::OFF_ST_B);
+        const uint32_t d_tmem = tmem_base + b * P::TN;
+        if constexpr (P::A_TMEM) {
+          // one handshake per group of KG k-blocks: widened A of the group in
+          // slot u, B of each k-block in its TMA stage
+          for (int kb = 0; kb < num_kb; kb += P::KG, ++group) {
+            const uint32_t u = group % WS, pu = (group / WS) & 1u;
+            if (!mbar_wait(&wready[u], pu, abort_flag, &g_status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk)
-            mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), P::IDESC,
-                   (kb | kk) != 0 ? 1u : 0u);
-          tc_commit(&freed[s]);
-          tc_commit(&wfree[u]);
-          ++consumed;
+            for (int j = 0; j < P::KG; ++j) {
+              const uint32_t s = consumed % ST;
+              const uint32_t b0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_ST_B);
+              const uint32_t ta = tmem_base + P::TMEM_A0 + (u * P::KG + j) * 32;
+#pragma unroll
+              for (int kk = 0; kk < BK / 32; ++kk)
+                mma_i8_ta(d_tmem, ta + kk * 8, umma_desc_sw128(b0 + kk * 32), P::IDESC,
+                          ((kb + j) | kk) != 0 ? 1u : 0u);
+              tc_commit(&freed[s]);
+              ++consumed;
+            }
+            tc_commit(&wfree[u]);
+          }
+        } else {
+          for (int kb = 0; kb < num_kb; ++kb) {
+            const uint32_t s = consumed % ST;
+            const uint32_t u = consumed % WS, pu = (consumed / WS) & 1u;
+            // the widen warps waited for the stage's TMA bytes before signalling wready
+            if (!mbar_wait(&wready[u], pu, abort_flag, &g_status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint8_t *slot = smem + P::OFF_W + u * P::WSLOT_BYTES;
+            const uint32_t a0 = smem_u32(slot + P::OFF_W_A);
+            const uint32_t b0 = smem_u32(slot + P::OFF_W_B);
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk)
+              mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), P::IDESC,
+                     (kb | kk) != 0 ? 1u : 0u);
+            tc_commit(&freed[s]);
+            tc_commit(&wfree[u]);
+            ++consumed;
+          }
         }
         if (ok) tc_commit(&acc_full[b]);
       }
@@ -308,22 +349,74 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int t = threadIdx.x - W_UNPACK0 * 32;
     uint32_t n = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < num_kb; ++kb, ++n) {
-        const uint32_t s = n % ST, ps = (n / ST) & 1u;
-        const uint32_t u = n % WS, pu = (n / WS) & 1u;
-        if (!mbar_wait(&full[s], ps, abort_flag, &g_status) ||
-            !mbar_wait(&wfree[u], pu ^ 1u, abort_flag, &g_status)) {
-          ok = false;
-          break;
+    if constexpr (P::A_TMEM) {
+      // this warp writes tensor-memory lanes 32 (warp % 4) .. + 31 (its lane quadrant)
+      uint32_t grp = 0;
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + P::TMEM_A0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < num_kb && ok; kb += P::KG, ++grp) {
+          const uint32_t u = grp % WS, pu = (grp / WS) & 1u;
+          if (!mbar_wait(&wfree[u], pu ^ 1u, abort_flag, &g_status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();  // the MMAs that read slot u completed
+#pragma unroll 1
+          for (int j = 0; j < P::KG; ++j, ++n) {
+            const uint32_t s = n % ST, ps = (n / ST) & 1u;
+            if (!mbar_wait(&full[s], ps, abort_flag, &g_status)) {
+              ok = false;
+              break;
+            }
+            // tile row t: its 64 packed bytes (64-byte swizzled rows: 16-byte
+            // chunk c at c ^ ((row / 2) % 4)) -> 128 values code + 8 -> 32
+            // tensor-memory columns of lane t
+            const uint8_t *src = smem + s * P::STAGE_BYTES + P::OFF_ST_A + t * 64;
+            uint32_t o[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(src + ((c ^ ((t >> 1) & 3)) << 4));
+              uint4 o0, o1;
+              widen_chunk<false>(v, o0, o1);
+              o[8 * c + 0] = o0.x;
+              o[8 * c + 1] = o0.y;
+              o[8 * c + 2] = o0.z;
+              o[8 * c + 3] = o0.w;
+              o[8 * c + 4] = o1.x;
+              o[8 * c + 5] = o1.y;
+              o[8 * c + 6] = o1.z;
+              o[8 * c + 7] = o1.w;
+            }
+            tmem_st_32x32b_x32(tq + (u * P::KG + j) * 32, o);
+          }
+          if (!ok) {
+            tmem_wait_st();
+            break;
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&wready[u]);
         }
-        uint8_t *stage = smem + s * P::STAGE_BYTES;
-        uint8_t *slot = smem + P::OFF_W + u * P::WSLOT_BYTES;
-        widen_tile<A_PK / 16 / 128, B_PACKED>(stage + P::OFF_ST_A, slot + P::OFF_W_A, t);
-        if (B_PACKED) widen_tile<B_PK / 16 / 128, true>(stage + P::OFF_ST_B, slot + P::OFF_W_B, t);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&wready[u]);
+      }
+    } else {
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < num_kb; ++kb, ++n) {
+          const uint32_t s = n % ST, ps = (n / ST) & 1u;
+          const uint32_t u = n % WS, pu = (n / WS) & 1u;
+          if (!mbar_wait(&full[s], ps, abort_flag, &g_status) ||
+              !mbar_wait(&wfree[u], pu ^ 1u, abort_flag, &g_status)) {
+            ok = false;
+            break;
+          }
+          uint8_t *stage = smem + s * P::STAGE_BYTES;
+          uint8_t *slot = smem + P::OFF_W + u * P::WSLOT_BYTES;
+          widen_tile<A_PK / 16 / 128, true>(stage + P::OFF_ST_A, slot + P::OFF_W_A, t);
+          widen_tile<B_PK / 16 / 128, true>(stage + P::OFF_ST_B, slot + P::OFF_W_B, t);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&wready[u]);
+        }
       }
     }
   } else if (warp >= W_EPI0) {
@@ -332,21 +425,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // this warp's copy of the tile's per-column constants:
     //   off[n] = 0x4B400000 - 8 colsum[n] (the code-offset correction folded
     //   into the exact int -> float bias), sc[n], bias[n]
-    int32_t *coff = reinterpret_cast<int32_t *>(smem + P::OFF_COL) + ew * 3 * BN;
-    float *csc = reinterpret_cast<float *>(coff + BN);
-    float *cbi = csc + BN;
+    constexpr int TN = P::TN;
+    int32_t *coff = reinterpret_cast<int32_t *>(smem + P::OFF_COL) + ew * 3 * TN;
+    float *csc = reinterpret_cast<float *>(coff + TN);
+    float *cbi = csc + TN;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const uint32_t b = it & 1, pb = (it >> 1) & 1;
       const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
       __syncwarp();  // every lane is done reading the previous tile's constants
 #pragma unroll
-      for (int j = lane; j < BN; j += 32) {
-        const int n = nb * BN + j;
-        coff[j] = 0x4B400000 - (B_PACKED ? 0 : 8 * __ldg(colsum + n));
+      for (int j = lane; j < TN; j += 32) {
+        const int n = nb * TN + j;
+        const bool in = n < N;  // the last tile of a ragged N
+        coff[j] = 0x4B400000 - ((B_PACKED || !in) ? 0 : 8 * __ldg(colsum + n));
         if (!OUT_S32) {
-          csc[j] = __ldg(scale_ch + n);
-          cbi[j] = __ldg(bias + n);
+          csc[j] = in ? __ldg(scale_ch + n) : 0.0f;
+          cbi[j] = in ? __ldg(bias + n) : 0.0f;
         }
       }
       __syncwarp();
@@ -355,24 +450,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row0 = mb * BM + ew * 32;
       const int m = row0 + lane;
       const float st = (!OUT_S32 && m < M) ? __ldg(scale_tok + m) : 0.0f;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * BN;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * TN;
 #pragma unroll 1
-      for (int sc = 0; sc < BN / EPI_COLS; ++sc) {
+      for (int sc = 0; sc < TN / EPI_COLS; ++sc) {
         // 64 accumulator columns of this warp's 32 rows: two loads, one wait
         uint32_t r[64];
         tmem_ld_32x32b_x32(tbase + sc * EPI_COLS, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         tmem_ld_32x32b_x32(tbase + sc * EPI_COLS + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_wait_ld();
-        if (sc == BN / EPI_COLS - 1) {
+        if (sc == TN / EPI_COLS - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
         const int c0 = sc * EPI_COLS;
-        const int n0 = nb * BN + c0;
+        const int n0 = nb * TN + c0;
         const int4 *off4 = reinterpret_cast<const int4 *>(coff + c0);
         if (OUT_S32) {
-          if (m < M) {
+          if (m < M && n0 < N) {
             int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(m) * N + n0);
 #pragma unroll
             for (int c = 0; c < EPI_COLS / 4; ++c) {
@@ -408,7 +503,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && row0 < M) {
+          if (lane == 0 && row0 < M && n0 < N) {
             tma_store_2d(&tmY, stg, n0, row0);
             bulk_commit();
           }
@@ -498,12 +593,12 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   CUtensorMap tmA, tmB, tmY;
   const uint64_t kp = static_cast<uint64_t>(a.K / 2);
   if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qx, kp, a.M, kp, BKP, BM,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+                   P::A_TMEM ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const bool okB = B_PACKED ? make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw, kp, a.N, kp,
                                           BKP, BN, CU_TENSOR_MAP_SWIZZLE_NONE)
                             : make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw8, a.K, a.N,
-                                          a.K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+                                          a.K, BK, P::TN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!okB) return cudaErrorInvalidValue;
   if (OUT_S32) {
     tmY = tmA;  // unused
@@ -512,7 +607,7 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
     return cudaErrorInvalidValue;
   }
   const int num_m = static_cast<int>((a.M + BM - 1) / BM);
-  const int num_n = a.N / BN;
+  const int num_n = (a.N + P::TN - 1) / P::TN;
   const int tiles = num_m * num_n;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
   kern<<<grid, NUM_THREADS, P::SMEM_BYTES, st>>>(tmA, tmB, tmY, a.scale_tok, a.scale_ch, a.bias,

@@ -13,12 +13,18 @@
 //   phase 1: lane l holds x[l + 32 j], j < V: 16-bit loads, every warp-wide
 //            load instruction covers 64 contiguous bytes.  The butterflies over
 //            the bits of j (index bits 5 .. log2 K - 1) run in registers.
-//   transpose through a 32 x 32 fp32 shared-memory tile per warp (XOR-swizzled
-//            columns, conflict-free both ways), P = V/32 passes.
+//   transpose through a 32 x 32 fp32 shared-memory tile per warp, P = V/32
+//            passes: each lane writes its 32 values of a pass as one tile row
+//            with 16-byte stores (16-byte chunk c of row l at chunk position
+//            c ^ (l % 8): conflict-free both ways) and reads a column back.
+//            Phase-1 values sit in register slot phase1_slot(j) so that each
+//            16-byte store takes four consecutive slots.
 //   phase 2: lane l holds x[V l + r], r < V: the butterflies over index bits
 //            0..4 run in registers; each lane then owns V consecutive outputs,
 //            i.e. V/2 consecutive bytes of packed codes, stored with 16-byte
 //            stores.
+// Packed fp32x2 instructions do two butterflies, products or fused
+// multiply-adds at once; adjacent register slots (2m, 2m + 1) form the pairs.
 // The transform is the Sylvester (natural-order) Hadamard product x H, scaled
 // by 1/sqrt(K) (an exact power of two for K = 1024 and 4096).
 #include <cuda_bf16.h>
@@ -81,6 +87,16 @@ __device__ __forceinline__ void butterflies(float (&v)[V]) {
   }
 }
 
+// Register slot of phase-1 value j (x[lane + 32 j]).  The transpose pass
+// p = j % (V/32) moves value j to lane j / (V/32); pass p writes tile column
+// j / (V/32), and the four values of each 16-byte chunk of a pass sit in
+// consecutive slots.  For K = 1024 (one pass) that is the identity; for
+// K = 4096 the two low bits of j (the pass) and the next two swap places.
+template <int K>
+__host__ __device__ constexpr int phase1_slot(int j) {
+  return K == 1024 ? j : (((j >> 2) & 3) | ((j & 3) << 2) | (j & ~15));
+}
+
 template <int K>
 struct RowShape {
   static constexpr int V = K / 32;  // values per lane
@@ -100,7 +116,7 @@ __device__ __forceinline__ void load_phase1(const unsigned short *__restrict__ x
   for (int j = 0; j < V; ++j) {
     float f = bf16_bits_to_float(FROM_SMEM ? x[lane + 32 * j] : __ldcs(x + lane + 32 * j));
     if (GELU) f = gelu_bf16(f);
-    u[j] = f;
+    u[phase1_slot<K>(j)] = f;
   }
 }
 
@@ -111,18 +127,56 @@ __device__ __forceinline__ void transform_row(float (&u)[RowShape<K>::V], int la
                                               float *__restrict__ tile, float (&v)[RowShape<K>::V]) {
   constexpr int V = RowShape<K>::V;
   constexpr int P = RowShape<K>::P;
-  if (ROT) butterflies<V, 0, RowShape<K>::LOGV>(u);  // index bits 5 .. log2(K)-1
-  // transpose: value u[P*l2 + p] of lane l moves to lane l2, register 32p + l
+  // index bits 5 .. log2(K)-1 (phase1_slot permutes them among themselves)
+  if (ROT) butterflies<V, 0, RowShape<K>::LOGV>(u);
+  float4 *trow = reinterpret_cast<float4 *>(tile + lane * 32);
 #pragma unroll
   for (int p = 0; p < P; ++p) {
+    // pass p: tile row `lane`, column c <- value j = P c + p of this lane
 #pragma unroll
-    for (int l2 = 0; l2 < 32; ++l2) tile[l2 * 32 + (lane ^ l2)] = u[P * l2 + p];
+    for (int m = 0; m < 8; ++m) {
+      const int s0 = (K == 1024) ? 4 * m : 16 * m + 4 * p;
+      trow[m ^ (lane & 7)] = make_float4(u[s0], u[s0 + 1], u[s0 + 2], u[s0 + 3]);
+    }
     __syncwarp();
+    // x[V lane + 32 p + l] is value j = P lane + p of lane l: column `lane` of row l
 #pragma unroll
-    for (int l = 0; l < 32; ++l) v[32 * p + l] = tile[lane * 32 + (l ^ lane)];
+    for (int l = 0; l < 32; ++l)
+      v[32 * p + l] = tile[l * 32 + ((((lane >> 2) ^ (l & 7)) << 2) | (lane & 3))];
     __syncwarp();
   }
   if (ROT) butterflies<V, 0, 5>(v);  // index bits 0..4
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(unsigned long long v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ void mul_x2(float &a0, float &a1, float b0, float b1) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(a0, a1)), "l"(pack2(b0, b1)));
+  unpack2(d, a0, a1);
+}
+__device__ __forceinline__ void fma_x2(float &a0, float &a1, unsigned long long b,
+                                       unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pack2(a0, a1)), "l"(b), "l"(c));
+  unpack2(d, a0, a1);
+}
+
+// Low bytes of a, b, c, d as the bytes 0..3 of one word.
+__device__ __forceinline__ uint32_t low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 // Per-channel multiplier (from the block's shared table), per-row absmax,
@@ -138,15 +192,16 @@ __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], i
 #pragma unroll
     for (int c = 0; c < V / 4; ++c) {
       const float4 m = mtab[c * 32 + lane];
-      v[4 * c + 0] *= m.x;
-      v[4 * c + 1] *= m.y;
-      v[4 * c + 2] *= m.z;
-      v[4 * c + 3] *= m.w;
+      mul_x2(v[4 * c + 0], v[4 * c + 1], m.x, m.y);
+      mul_x2(v[4 * c + 2], v[4 * c + 3], m.z, m.w);
     }
   }
-  float amax = 0.0f;
+  float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int r = 0; r < V; ++r) amax = fmaxf(amax, fabsf(v[r]));
+  for (int r = 0; r < V; r += 8)
+#pragma unroll
+    for (int a = 0; a < 4; ++a) am[a] = fmax3(am[a], fabsf(v[r + 2 * a]), fabsf(v[r + 2 * a + 1]));
+  float amax = fmax3(am[0], am[1], fmaxf(am[2], am[3]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (lane == 0) scale[row] = (ROT ? amax * RowShape<K>::kInvSqrtK : amax) / 7.0f;
@@ -159,16 +214,19 @@ __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], i
   // code = round-half-even(v * inv); |v * inv| <= 7 (1 + 2^-24), so no clamp
   // can ever act.  Adding 1.5 * 2^23 in the same fused operation rounds the
   // exact product to an integer whose low 4 bits are the two's-complement code.
+  const unsigned long long inv2 = pack2(inv, inv), magic2 = pack2(12582912.0f, 12582912.0f);
+#pragma unroll
+  for (int k = 0; k < V; k += 2) fma_x2(v[k], v[k + 1], inv2, magic2);
+  // word w: codes of elements 8w .. 8w + 7, element 2i in the low nibble of byte i
   uint32_t words[V / 8];
 #pragma unroll
   for (int w = 0; w < V / 8; ++w) {
-    uint32_t acc = 0;
+    uint32_t b[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float f = fmaf(v[8 * w + k], inv, 12582912.0f);
-      acc |= (__float_as_uint(f) & 0xFu) << (4 * k);
-    }
-    words[w] = acc;
+    for (int e = 0; e < 8; ++e) b[e] = __float_as_uint(v[8 * w + e]);
+    const uint32_t even = low_bytes(b[0], b[2], b[4], b[6]);
+    const uint32_t odd = low_bytes(b[1], b[3], b[5], b[7]);
+    words[w] = (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
   }
   uint4 *dst = reinterpret_cast<uint4 *>(q + row * (K / 2) + static_cast<int64_t>(lane) * (V / 2));
 #pragma unroll
@@ -204,18 +262,10 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
   float *tile = reinterpret_cast<float *>(ring + S::NS * S::ROWB);
   uint64_t *bars = reinterpret_cast<uint64_t *>(qsmem + S::OFF_BAR) + warp * S::NS;
   float4 *mtab = reinterpret_cast<float4 *>(qsmem + S::OFF_TAB);
-  if (ROT) {
-    // table[(r/4)*32 + l] holds mult[V l + r .. +3]: lane l's 16-byte reads of
-    // one chunk are consecutive across the warp (conflict-free)
-    float *t = reinterpret_cast<float *>(mtab);
-    for (int j = threadIdx.x; j < K; j += blockDim.x) {
-      const int l = j / V, r = j % V;
-      t[((r >> 2) * 32 + l) * 4 + (r & 3)] = __ldg(mult + j);
-    }
-    __syncthreads();
-  }
+  // rows r0, r0 + G, ...: consecutive r0 go to different blocks, so the rows
+  // of the last, partial round are spread over all SMs
   const int64_t G = static_cast<int64_t>(gridDim.x) * kQuantWarps;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kQuantWarps + warp;
+  const int64_t r0 = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x;
   int64_t issued = 0;  // rows whose copy lane 0 has issued (sequence numbers 0..issued-1)
   if (lane == 0) {
     for (int s = 0; s < S::NS; ++s) mbar_init(&bars[s], 1);
@@ -228,6 +278,17 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
       bulk_load(ring + s * S::ROWB, X + r * K, S::ROWB, &bars[s]);
       ++issued;
     }
+  }
+  if (ROT) {
+    // (after the first copies are on their way) table[(r/4)*32 + l] holds
+    // mult[V l + r .. +3]: lane l's 16-byte reads of one chunk are consecutive
+    // across the warp (conflict-free)
+    float *t = reinterpret_cast<float *>(mtab);
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      const int l = j / V, r = j % V;
+      t[((r >> 2) * 32 + l) * 4 + (r & 3)] = __ldg(mult + j);
+    }
+    __syncthreads();
   }
   __syncwarp();
   int64_t i = 0;
