@@ -256,6 +256,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above (barriers, tensor memory, descriptor prefetch) may overlap
+  // the tail of the kernel that produced qx and scale_tok; from here on this
+  // CTA reads what earlier kernels wrote.
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp == W_TMA) {
     if (lane == 0) {
@@ -610,9 +615,21 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   const int num_n = (a.N + P::TN - 1) / P::TN;
   const int tiles = num_m * num_n;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  kern<<<grid, NUM_THREADS, P::SMEM_BYTES, st>>>(tmA, tmB, tmY, a.scale_tok, a.scale_ch, a.bias,
-                                                 a.colsum, a.acc, static_cast<int>(a.M), a.N, num_n,
-                                                 tiles, a.K / BK);
+  // programmatic stream serialization: the prologue may overlap the previous
+  // kernel's tail (the kernel waits for it before reading any input)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = P::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmY, a.scale_tok, a.scale_ch, a.bias, a.colsum, a.acc,
+                         static_cast<int>(a.M), a.N, num_n, tiles, a.K / BK);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

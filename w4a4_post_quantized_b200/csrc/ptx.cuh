@@ -137,6 +137,19 @@ __device__ __forceinline__ void bulk_wait() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel of the stream is still running.  griddep_wait() blocks until
+// that kernel has completed and its memory writes are visible (it returns at
+// once for a kernel launched without the attribute); nothing that kernel (or an
+// earlier one) writes may be touched before it.  griddep_launch_dependents()
+// lets the next such kernel of the stream be scheduled before this one ends.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy accesses (tensor-core reads, TMA stores).
 __device__ __forceinline__ void fence_proxy_async_smem() {

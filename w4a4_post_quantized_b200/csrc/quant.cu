@@ -270,6 +270,12 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
   if (lane == 0) {
     for (int s = 0; s < S::NS; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
+  }
+  // The barrier setup above may overlap the tail of the previous kernel of the
+  // stream; X, mult, q and scale are touched only after it has completed.
+  griddep_launch_dependents();
+  griddep_wait();
+  if (lane == 0) {
     fence_proxy_async_smem();
     for (int s = 0; s < S::NS; ++s) {
       const int64_t r = r0 + s * G;
@@ -407,7 +413,20 @@ cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint
   const int64_t need = (M + kQuantWarps - 1) / kQuantWarps;
   const int64_t g = static_cast<int64_t>(num_sms()) * per_sm;
   const int grid = static_cast<int>(need < g ? need : g);
-  kern<<<grid, kQuantWarps * 32, smem, st>>>(X, M, mult, q, scale, status_word());
+  // programmatic stream serialization: the block setup may overlap the
+  // previous kernel's tail (the kernel waits for it before touching memory)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kQuantWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, X, M, mult, q, scale, status_word());
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
