@@ -277,16 +277,16 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
   griddep_wait();
   if (lane == 0) {
     fence_proxy_async_smem();
-    for (int s = 0; s < S::NS; ++s) {
-      const int64_t r = r0 + s * G;
-      if (r >= M) break;
-      mbar_arrive_expect_tx(&bars[s], S::ROWB);
-      bulk_load(ring + s * S::ROWB, X + r * K, S::ROWB, &bars[s]);
+    // the first row now; the ring's second slot is filled once it has landed
+    // (below), so at start-up every warp's first row arrives sooner
+    if (r0 < M) {
+      mbar_arrive_expect_tx(&bars[0], S::ROWB);
+      bulk_load(ring, X + r0 * K, S::ROWB, &bars[0]);
       ++issued;
     }
   }
   if (ROT) {
-    // (after the first copies are on their way) table[(r/4)*32 + l] holds
+    // (after the first copy is on its way) table[(r/4)*32 + l] holds
     // mult[V l + r .. +3]: lane l's 16-byte reads of one chunk are consecutive
     // across the warp (conflict-free)
     float *t = reinterpret_cast<float *>(mtab);
@@ -301,6 +301,15 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
   for (int64_t row = r0; row < M; row += G, ++i) {
     const int s = static_cast<int>(i % S::NS);
     if (!mbar_wait_drain(&bars[s], static_cast<uint32_t>((i / S::NS) & 1), status)) break;
+    static_assert(S::NS == 2, "the ring's second slot is filled here");
+    if (i == 0 && lane == 0) {
+      const int64_t r = r0 + G;
+      if (r < M) {
+        mbar_arrive_expect_tx(&bars[1], S::ROWB);
+        bulk_load(ring + S::ROWB, X + r * K, S::ROWB, &bars[1]);
+        ++issued;
+      }
+    }
     float u[V], v[V];
     load_phase1<K, GELU, true>(reinterpret_cast<const unsigned short *>(ring + s * S::ROWB), lane, u);
     transform_row<K, ROT>(u, lane, tile, v);  // ends with __syncwarp: slot s is no longer read
