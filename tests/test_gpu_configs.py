@@ -1,0 +1,116 @@
+"""Full-size parity for the benchmark configurations other than the frame-QKV
+one: the MLP pair at 8 frames, the global-attention block's four linears at
+32 frames and the full-depth stack's four layer shapes at 64 frames.
+
+Each layer runs at its full token count through w4a4_linear_fused, in the
+launch configuration the benchmark uses; the oracle recomputes sampled rows
+(every special-token row plus a regular stride of the rest) one by one, and
+the bar is the end-to-end one: relative Frobenius error of the sampled rows at
+most 2e-3, and the same SQNR against the unquantized product on both sides.
+The MLP pair is also run as a chain (fc1's bf16 output, through GELU, is fc2's
+input on the GPU; the oracle runs its own chain on the sampled rows and the
+calibration rows): quantization noise compounds along the chain, so there
+the check is on the SQNR of the final output, which must agree within 0.3 dB.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w4a4_post_quantized_b200 import synth
+from parity import rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def w4():
+    from w4a4_post_quantized_b200 import w4a4
+    return w4a4
+
+
+def bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def y_bits(Y):
+    return Y.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def sample_rows(M, stride):
+    return np.unique(np.concatenate([synth.special_rows(M), np.arange(7, M, stride)]))
+
+
+def layer_case(w4, M, N, K, seed, gelu=False, stride=211):
+    X = synth.activations(M, K, seed=seed)
+    W = synth.weights(N, K, seed=seed + 1)
+    b = synth.bias(N, seed=seed + 2)
+    Xc = X[:synth.calibration_rows(M)]
+    pw = w4.w4a4_prepare_weights(bf16_dev(W), bf16_dev(b), bf16_dev(Xc))
+    Y = w4.w4a4_linear_fused(bf16_dev(X), pw, flags=w4.W4A4_FLAG_GELU if gelu else 0)
+    assert w4.w4a4_get_device_status() == 0
+    rows = sample_rows(M, stride)
+    got = synth.bf16_bits_to_f32(y_bits(Y)[rows]).astype(np.float64)
+    ow = oracle.prepare_weights(W, b, Xc, decision="f32")
+    want = oracle.linear(X[rows], ow, gelu=gelu, decision="f32")[0]
+    ref = oracle.reference_fp(X[rows], W, b, gelu=gelu)
+    return rel_fro(got, want), oracle.sqnr_db(ref, got), oracle.sqnr_db(ref, want)
+
+
+def check(case):
+    err, sq_gpu, sq_or = case
+    assert err <= 2e-3, err
+    assert abs(sq_gpu - sq_or) < 0.1, (sq_gpu, sq_or)
+
+
+@pytest.mark.parametrize("name,N,K,gelu", [("fc1", 4096, 1024, False), ("fc2", 1024, 4096, True)])
+def test_mlp_pair_layers_8_frames(w4, name, N, K, gelu):
+    check(layer_case(w4, 8 * synth.FRAME_TOKENS, N, K, seed=300 + K, gelu=gelu))
+
+
+@pytest.mark.parametrize("name,K,N", [l for l in synth.CONFIGS["c4_global_block"]["layers"]])
+def test_global_block_layers_32_frames(w4, name, K, N):
+    M = synth.CONFIGS["c4_global_block"]["frames"] * synth.FRAME_TOKENS
+    check(layer_case(w4, M, N, K, seed=400 + N + K, gelu=(name == "fc2"), stride=997))
+
+
+@pytest.mark.parametrize("name,K,N", [l for l in synth.CONFIGS["c5_full_stack"]["layers"]])
+def test_full_stack_layer_shapes_64_frames(w4, name, K, N):
+    """One layer of each shape of the 48-block stack at its full token count
+    (the stack repeats these four kernels with fresh weights)."""
+    M = synth.CONFIGS["c5_full_stack"]["frames"] * synth.FRAME_TOKENS
+    check(layer_case(w4, M, N, K, seed=500 + N + K, gelu=(name == "fc2"), stride=1999))
+
+
+def test_mlp_pair_chain_8_frames(w4):
+    """fc1 -> GELU -> fc2 on the GPU, fc2 quantizing fc1's bf16 output with the
+    GELU folded into its load, against the oracle's own chain on sampled rows."""
+    M = 8 * synth.FRAME_TOKENS
+    X = synth.activations(M, 1024, seed=31)
+    W1, b1 = synth.weights(4096, 1024, seed=32), synth.bias(4096, seed=33)
+    W2, b2 = synth.weights(1024, 4096, seed=34), synth.bias(1024, seed=35)
+    C = synth.calibration_rows(M)
+    rows = sample_rows(M, 211)
+    need = np.union1d(np.arange(C), rows)
+    # oracle chain on the rows it needs: calibration rows and sampled rows
+    o1 = oracle.prepare_weights(W1, b1, X[:C], decision="f32")
+    Y1o = oracle.linear(X[need], o1, decision="f32")[0]
+    H1o = oracle.f64_to_bf16(Y1o)                  # fc1's bf16 output (bits)
+    pos = np.searchsorted(need, np.arange(C))
+    G1c = oracle.gelu_bf16(H1o[pos])               # fc2's calibration input (bf16 bits)
+    o2 = oracle.prepare_weights(W2, b2, G1c, decision="f32")
+    Y2o = oracle.linear(H1o[np.searchsorted(need, rows)], o2, gelu=True, decision="f32")[0]
+    # GPU chain; fc2's calibration input is GELU of the GPU's own fc1 output
+    p1 = w4.w4a4_prepare_weights(bf16_dev(W1), bf16_dev(b1), bf16_dev(X[:C]))
+    Y1 = w4.w4a4_linear_fused(bf16_dev(X), p1)
+    G1 = torch.nn.functional.gelu(Y1[:C].float()).to(torch.bfloat16)
+    p2 = w4.w4a4_prepare_weights(bf16_dev(W2), bf16_dev(b2), G1)
+    Y2 = w4.w4a4_linear_fused(Y1, p2, flags=w4.W4A4_FLAG_GELU)
+    assert w4.w4a4_get_device_status() == 0
+    got = synth.bf16_bits_to_f32(y_bits(Y2)[rows]).astype(np.float64)
+    # unquantized fp64 chain on the sampled rows
+    r1 = oracle.reference_fp(X[rows], W1, b1)
+    ref = oracle.reference_fp(oracle.f64_to_bf16(r1), W2, b2, gelu=True)
+    sq_gpu, sq_or = oracle.sqnr_db(ref, got), oracle.sqnr_db(ref, Y2o)
+    assert abs(sq_gpu - sq_or) < 0.3, (sq_gpu, sq_or)
+    assert rel_fro(got, Y2o) < 0.05
