@@ -284,29 +284,63 @@ def run_ours(args, wl, world, rank, local):
     value = world * ops * args.steps / (elapsed_ms * 1e-3) / 1e12
 
     # ------------------------------------------------------------- end to end
+    # the C-ABI host-buffer call a user with host tensors makes: every step
+    # copies its X from pinned host memory and its Y back, in row chunks whose
+    # copies in, kernels and copies out overlap on three streams
     Xh = [torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
     for x, src in zip(Xh, Xs):
         x.copy_(src.cpu())
-    Yh = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    Yh = [torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    chunk = args.e2e_chunk
+    pipe = w4a4.HostPipe()
+    hws = torch.empty(w4a4.w4a4_host_workspace_bytes(chunk, K, N), dtype=torch.uint8, device=dev)
+
+    def host_step(i):
+        w4a4.w4a4_linear_fused_host(Xh[i % 2], pw, Y_host=Yh[i % 2], chunk_rows=chunk, workspace=hws,
+                                    pipe=pipe, flags=flags)
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
-    for i in range(2):
-        Xs[0].copy_(Xh[i], non_blocking=True)
-        step(0)
-        Yh.copy_(Ys[0], non_blocking=True)
+    for i in range(3):
+        host_step(i)
     torch.cuda.synchronize()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     a0.record(stream)
     for i in range(e2e_steps):
-        Xs[0].copy_(Xh[i % 2], non_blocking=True)
-        step(0)
-        Yh.copy_(Ys[0], non_blocking=True)
+        host_step(i)
     a1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
+    pipe.close()
     e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / e2e_steps
     e2e_value = world * ops / (e2e_ms * 1e-3) / 1e12
+
+    # ------------------------------------------------- DSFQ overhead (M7) and bytes (M2)
+    # the same fused call with the rotation and smoothing skipped (plain
+    # per-token / per-channel int4, weights prepared the same way), timed over
+    # the same rotating buffers; the pages put DSFQ's extra latency at 0.2 %
+    n7 = max(3, min(args.steps, 400))
+    pw_plain = w4a4.w4a4_prepare_weights(W, b, Xs[0][:synth.calibration_rows(M)],
+                                         flags=w4a4.W4A4_FLAG_PLAIN)
+    m7 = {}
+    for mode, p, fl in (("dsfq", pw, flags), ("plain", pw_plain, flags | w4a4.W4A4_FLAG_PLAIN)):
+        for i in range(3):
+            w4a4.w4a4_linear_fused(Xs[i % NSETS], p, Y=Ys[i % NSETS], workspace=WSs[i % NSETS], flags=fl)
+        barrier(world)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for i in range(n7):
+            w4a4.w4a4_linear_fused(Xs[i % NSETS], p, Y=Ys[i % NSETS], workspace=WSs[i % NSETS], flags=fl)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        m7[mode] = max_over_ranks(world, b0.elapsed_time(b1)) / n7 * 1e3
+    dsfq_overhead = {"dsfq_us_per_step": m7["dsfq"], "plain_us_per_step": m7["plain"],
+                     "overhead_pct": 100.0 * (m7["dsfq"] - m7["plain"]) / m7["plain"],
+                     "steps": n7, "pages_figure_pct": 0.2}
+    weight_bytes = {"packed_int4": N * K // 2 + 12 * N + 4 * K, "bf16": 2 * N * K + 2 * N,
+                    "expanded_int8_copy": N * K + 4 * N,
+                    "ratio_bf16_over_packed": (2 * N * K + 2 * N) / (N * K // 2 + 12 * N + 4 * K)}
 
     # ------------------------------------------------------------- roofline
     peaks = load_peaks()
@@ -335,10 +369,13 @@ def run_ours(args, wl, world, rank, local):
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "TOPS", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
-                "api": "w4a4_linear_fused with pinned-host X/Y copies on the same stream"},
+                "api": f"w4a4_linear_fused_host (C ABI, pinned host X/Y, {chunk}-row chunks, "
+                       "copies in / kernels / copies out overlapped)"},
         "gpu_launches": 2 * args.steps,
         "roofline": roofline,
         "roofline_quantize": roofline_q,
+        "dsfq_overhead": dsfq_overhead,
+        "weight_bytes": weight_bytes,
         "device_status": status,
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -368,6 +405,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c2_frame_qkv")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-chunk", type=int, default=1408, help="row chunk of the host-buffer call")
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

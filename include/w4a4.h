@@ -179,6 +179,53 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
 w4a4_status w4a4_linear_fused_noalloc(const uint16_t *X, int64_t M, const w4a4_weights_t *w,
                                       uint16_t *Y, uint32_t flags, void *stream);
 
+/* ---------------------------------------------------------------------------
+ * Host-buffer entry point.  No page describes one: it is the layer as a caller
+ * with inputs and outputs in host memory uses it (the pages' deployment keeps
+ * activations on the accelerator).  The M rows are processed in chunks of
+ * chunk_rows; the host->device copy of a chunk, the two kernels of the
+ * previous chunk and the device->host copy of the one before run at the same
+ * time on three streams, so the call takes about as long as its larger copy
+ * direction instead of the sum of both copies and the kernels.  Every row's
+ * result is the same as w4a4_linear_fused's (rows are independent).
+ * ------------------------------------------------------------------------- */
+
+/* Chunk buffers in flight (per direction). */
+#define W4A4_PIPE_DEPTH 2
+
+/* The streams and events of the pipeline: created by w4a4_host_pipe_create on
+ * the current device, owned by the caller, reusable across calls (calls on one
+ * pipe must be issued from one host thread at a time). */
+typedef struct w4a4_host_pipe w4a4_host_pipe_t;
+
+/* Creates a pipe on the current device (two non-blocking streams and
+ * 3 * W4A4_PIPE_DEPTH events without timing).  *out receives the handle;
+ * W4A4_ERR_CUDA if a stream or event cannot be created. */
+w4a4_status w4a4_host_pipe_create(w4a4_host_pipe_t **out);
+
+/* Waits for the pipe's streams and frees it (NULL is a no-op). */
+w4a4_status w4a4_host_pipe_destroy(w4a4_host_pipe_t *pipe);
+
+/* Device workspace for w4a4_linear_fused_host: W4A4_PIPE_DEPTH slots, each
+ * holding one chunk's X (2 chunk_rows K bytes), Y (2 chunk_rows N bytes),
+ * codes and steps (w4a4_workspace_bytes(chunk_rows, K)), each part 256-byte
+ * aligned. */
+size_t w4a4_host_workspace_bytes(int64_t chunk_rows, int32_t K, int32_t N);
+
+/* Y_host [M, N] bf16 = w4a4_linear_fused(X_host [M, K] bf16) with X_host and
+ * Y_host in host memory (page-locked memory for the copies to overlap; pageable
+ * memory works but serializes).  workspace: device memory of at least
+ * w4a4_host_workspace_bytes(chunk_rows, w->K, w->N) bytes, 16-byte aligned;
+ * chunk_rows > 0 (a multiple of 128 uses whole GEMM tiles).  The call enqueues
+ * the work and returns; `stream` (the compute stream; NULL = legacy default
+ * stream) is made to wait for the last copy, so work enqueued on it afterwards,
+ * or a synchronize of it, sees Y_host complete.  Flags and errors as
+ * w4a4_linear_fused; M = 0 is a no-op. */
+w4a4_status w4a4_linear_fused_host(const uint16_t *X_host, int64_t M, const w4a4_weights_t *w,
+                                   uint16_t *Y_host, int64_t chunk_rows, void *workspace,
+                                   size_t workspace_bytes, w4a4_host_pipe_t *pipe,
+                                   uint32_t flags, void *stream);
+
 /* Integer product only: acc [M, N] int32 = sum_k qx[m, k] * code_w[n, k] for
  * packed activation codes qx [M, K/2] and the weight codes of *w (w->qw8 and
  * w->colsum when set, else the packed w->qw; scale_ch, bias and the smoothing

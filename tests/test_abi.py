@@ -160,3 +160,32 @@ def test_status_strings(lib):
     assert lib.w4a4_status_string(0) == b"ok"
     assert lib.w4a4_status_string(6) == b"device wait timed out"
     assert b"sm_100a" in lib.w4a4_version()
+
+
+def test_host_pipeline_argument_checks(lib):
+    """w4a4_linear_fused_host rejects bad arguments before touching the pipe or
+    the GPU; w4a4_host_workspace_bytes follows its documented layout."""
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    lib.w4a4_host_workspace_bytes.restype = sz
+    lib.w4a4_host_workspace_bytes.argtypes = [i64, i32, i32]
+    lib.w4a4_workspace_bytes.restype = sz
+    lib.w4a4_workspace_bytes.argtypes = [i64, i32]
+    r256 = lambda b: (b + 255) // 256 * 256
+    for rows, K, N in [(2816, 1024, 3072), (1, 4096, 1024), (300, 1024, 256)]:
+        slot = r256(2 * rows * K) + r256(2 * rows * N) + r256(lib.w4a4_workspace_bytes(rows, K))
+        assert lib.w4a4_host_workspace_bytes(rows, K, N) == 2 * slot
+    assert lib.w4a4_host_workspace_bytes(0, 1024, 256) == 0
+    f = lib.w4a4_linear_fused_host
+    f.restype = ctypes.c_int
+    f.argtypes = [vp, i64, ctypes.POINTER(WeightsT), vp, i64, vp, sz, vp, ctypes.c_uint32, vp]
+    w = WeightsT(256, 1024, A, A, A, A, A, None, None, 0)
+    need = lib.w4a4_host_workspace_bytes(128, 1024, 256)
+    fake_pipe = vp(A)  # never dereferenced on these paths
+    assert f(A, 10, ctypes.byref(w), A, 128, A, need, None, 0, None) == 1        # no pipe
+    assert f(A, 10, None, A, 128, A, need, fake_pipe, 0, None) == 1              # no weights
+    assert f(A, 0, ctypes.byref(w), A, 128, A, need, fake_pipe, 0, None) == 0    # empty: no-op
+    assert f(A, 10, ctypes.byref(w), A, 0, A, need, fake_pipe, 0, None) == 2     # chunk_rows 0
+    assert f(A, -1, ctypes.byref(w), A, 128, A, need, fake_pipe, 0, None) == 2   # negative M
+    assert f(None, 10, ctypes.byref(w), A, 128, A, need, fake_pipe, 0, None) == 1
+    assert f(A, 10, ctypes.byref(w), A, 128, A + 4, need, fake_pipe, 0, None) == 3  # misaligned
+    assert f(A, 10, ctypes.byref(w), A, 128, A, need - 1, fake_pipe, 0, None) == 2  # too small

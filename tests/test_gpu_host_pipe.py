@@ -1,0 +1,41 @@
+"""The host-buffer entry point: w4a4_linear_fused_host on pinned host memory
+must give exactly the rows w4a4_linear_fused gives on device memory (the same
+kernels on independent rows), for chunkings that split M evenly, raggedly or
+not at all, across repeated calls on one pipe."""
+import numpy as np
+import pytest
+import torch
+
+from w4a4_post_quantized_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def w4():
+    from w4a4_post_quantized_b200 import w4a4
+    return w4a4
+
+
+def bf16(bits, device):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+@pytest.mark.parametrize("M,N,K,chunk,gelu", [(10992, 3072, 1024, 2816, False), (1000, 512, 1024, 384, False),
+                                              (100, 256, 4096, 2816, True), (1374, 1024, 1024, 128, False)])
+def test_host_pipeline_matches_device_call(w4, M, N, K, chunk, gelu):
+    X = synth.activations(M, K, seed=M + K)
+    W, b = synth.weights(N, K, seed=5), synth.bias(N, seed=6)
+    pw = w4.w4a4_prepare_weights(bf16(W, "cuda"), bf16(b, "cuda"), bf16(X[:synth.calibration_rows(M)], "cuda"))
+    flags = w4.W4A4_FLAG_GELU if gelu else 0
+    want = w4.w4a4_linear_fused(bf16(X, "cuda"), pw, flags=flags).cpu()
+    Xh = bf16(X, "cpu").pin_memory()
+    pipe = w4.HostPipe()
+    ws = torch.empty(w4.w4a4_host_workspace_bytes(chunk, K, N), dtype=torch.uint8, device="cuda")
+    for rep in range(2):  # the pipe and workspace are reused across calls
+        Yh = torch.full((M, N), float("nan"), dtype=torch.bfloat16).pin_memory()
+        w4.w4a4_linear_fused_host(Xh, pw, Y_host=Yh, chunk_rows=chunk, workspace=ws, pipe=pipe, flags=flags)
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(Yh.view(torch.int16), want.view(torch.int16)), rep
+    assert w4.w4a4_get_device_status() == 0
+    pipe.close()

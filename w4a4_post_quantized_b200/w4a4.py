@@ -54,6 +54,11 @@ _fused = _sig("w4a4_linear_fused", ctypes.c_int,
 _fused_noalloc = _sig("w4a4_linear_fused_noalloc", ctypes.c_int,
                       [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _u32, _vp])
 _gemm_s32 = _sig("w4a4_gemm_s32", ctypes.c_int, [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp])
+_pipe_create = _sig("w4a4_host_pipe_create", ctypes.c_int, [ctypes.POINTER(_vp)])
+_pipe_destroy = _sig("w4a4_host_pipe_destroy", ctypes.c_int, [_vp])
+_host_ws_bytes = _sig("w4a4_host_workspace_bytes", _sz, [_i64, _i32, _i32])
+_fused_host = _sig("w4a4_linear_fused_host", ctypes.c_int,
+                   [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _i64, _vp, _sz, _vp, _u32, _vp])
 _expand = _sig("w4a4_expand_weights", ctypes.c_int, [ctypes.POINTER(W4A4WeightsT), _vp])
 _get_status = _sig("w4a4_get_device_status", ctypes.c_int, [_vp, ctypes.POINTER(_u32)])
 _clear_status = _sig("w4a4_clear_device_status", ctypes.c_int, [_vp])
@@ -101,6 +106,7 @@ class PreparedWeights:
 
     def __init__(self, N: int, K: int, device="cuda", expanded: bool = True):
         self.N, self.K = N, K
+        self.device = torch.device(device)
         self.qw = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
         self.scale_ch = torch.empty(N, dtype=torch.float32, device=device)
         self.bias = torch.empty(N, dtype=torch.float32, device=device)
@@ -176,6 +182,49 @@ def w4a4_linear_fused_noalloc(X: torch.Tensor, w: PreparedWeights, Y=None, flags
     _check(_fused_noalloc(_ptr(X), M, ctypes.byref(w.struct), _ptr(Y), flags, _stream(stream)),
            "w4a4_linear_fused_noalloc")
     return Y
+
+
+class HostPipe:
+    """The copy streams and events of w4a4_linear_fused_host (created on the
+    current device by the library; freed with the object)."""
+
+    def __init__(self):
+        h = _vp()
+        _check(_pipe_create(ctypes.byref(h)), "w4a4_host_pipe_create")
+        self.handle = h
+
+    def close(self):
+        if self.handle:
+            _check(_pipe_destroy(self.handle), "w4a4_host_pipe_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def w4a4_host_workspace_bytes(chunk_rows: int, K: int, N: int) -> int:
+    return _host_ws_bytes(chunk_rows, K, N)
+
+
+def w4a4_linear_fused_host(X_host: torch.Tensor, w: PreparedWeights, Y_host=None, chunk_rows: int = 2816,
+                           workspace=None, pipe: HostPipe | None = None, flags: int = 0, stream=None):
+    """Y_host = w4a4_linear_fused(X_host) with X_host / Y_host in (pinned) host
+    memory; row chunks of chunk_rows are copied in, computed and copied out
+    concurrently.  Returns Y_host (enqueued: synchronize `stream` before reading)."""
+    M = X_host.shape[0]
+    if Y_host is None:  # a convenience of this binding only
+        Y_host = torch.empty((M, w.N), dtype=torch.bfloat16, pin_memory=True)
+    if workspace is None:
+        workspace = torch.empty(w4a4_host_workspace_bytes(chunk_rows, w.K, w.N), dtype=torch.uint8,
+                                device=w.device)
+    if pipe is None:
+        raise ValueError("w4a4_linear_fused_host needs a HostPipe")
+    _check(_fused_host(_ptr(X_host), M, ctypes.byref(w.struct), _ptr(Y_host), chunk_rows, _ptr(workspace),
+                       workspace.numel(), pipe.handle, flags, _stream(stream)), "w4a4_linear_fused_host")
+    return Y_host
 
 
 def w4a4_expand_weights(w: PreparedWeights, stream=None) -> PreparedWeights:
