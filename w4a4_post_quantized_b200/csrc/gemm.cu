@@ -37,6 +37,12 @@
 //               subtract the code-offset term, scale by scale_tok[m] *
 //               scale_ch[n], add bias in fp32, round to bf16, TMA-store
 //               32 x 64 tiles through a 128-byte-swizzled staging buffer.
+//               The expanded-B path loads the accumulators in the 16x256b
+//               fragment layout (each thread: 4 rows, 2 of every 8 columns),
+//               so a thread reads only its own columns' constants (8-byte
+//               loads instead of 16-byte broadcasts of every column, which
+//               kept the shared-memory pipe busy), and writes the bf16 pairs
+//               with stmatrix.
 // Accumulators are double-buffered in tensor memory so the epilogue of one
 // tile overlaps the main loop of the next.
 //
@@ -453,6 +459,71 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&acc_full[b], pb, abort_flag, &g_status)) break;
       tc_fence_after();
       const int row0 = mb * BM + ew * 32;
+      if constexpr (!OUT_S32 && P::A_TMEM) {
+        // 16x256b fragments: thread t holds rows q = t/4 + 8 i (i < 4) of the
+        // warp's 32 rows and, per 8-column group j, columns 8j + 2(t%4) + {0,1};
+        // its columns' constants are 8-byte loads, and the bf16 pairs go to the
+        // staging tile with stmatrix (one 8 x 8 block per register)
+        const int tq = lane >> 2, tc = 2 * (lane & 3);
+        float st4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = row0 + tq + 8 * i;
+          st4[i] = m < M ? __ldg(scale_tok + m) : 0.0f;
+        }
+        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * TN;
+#pragma unroll 1
+        for (int sc = 0; sc < TN / EPI_COLS; ++sc) {
+          uint32_t r[2][32];  // [16-row half][4 j + k]
+          tmem_ld_16x256b_x8(tbase + sc * EPI_COLS, r[0]);
+          tmem_ld_16x256b_x8(tbase + (16u << 16) + sc * EPI_COLS, r[1]);
+          tmem_wait_ld();
+          if (sc == TN / EPI_COLS - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+          }
+          const int c0 = sc * EPI_COLS;
+          const int n0 = nb * TN + c0;
+          uint32_t pk[2][2][8];  // [half][row sub-block][j]: bf16 pair of (row, columns 8j + tc + {0,1})
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int c = c0 + 8 * j + tc;
+            const int2 o = *reinterpret_cast<const int2 *>(coff + c);
+            const float2 scl = *reinterpret_cast<const float2 *>(csc + c);
+            const float2 bi = *reinterpret_cast<const float2 *>(cbi + c);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int u = 0; u < 2; ++u)
+                pk[h][u][j] = dequant2_bf16(static_cast<int32_t>(r[h][4 * j + 2 * u]) + o.x,
+                                            static_cast<int32_t>(r[h][4 * j + 2 * u + 1]) + o.y,
+                                            st4[2 * h + u], scl.x, scl.y, bi.x, bi.y);
+          }
+          uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (sc & 1)) * EPI_BYTES;
+          if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
+          __syncwarp();
+          // staging tile: 32 rows of 128 bytes, 16-byte chunk k of row R at k ^ (R % 8);
+          // stmatrix x4 #(h, jp): matrices (u, j) = (0, 2jp), (1, 2jp), (0, 2jp+1), (1, 2jp+1)
+          const int mi = lane >> 3, mr = lane & 7;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int jp = 0; jp < 4; ++jp) {
+              const int row = 16 * h + 8 * (mi & 1) + mr;
+              const int chunk = 2 * jp + (mi >> 1);
+              stmatrix_x4(smem_u32(stg + row * 128 + ((chunk ^ (row & 7)) << 4)), pk[h][0][2 * jp],
+                          pk[h][1][2 * jp], pk[h][0][2 * jp + 1], pk[h][1][2 * jp + 1]);
+            }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < M && n0 < N) {
+            tma_store_2d(&tmY, stg, n0, row0);
+            bulk_commit();
+          }
+        }
+        continue;
+      }
       const int m = row0 + lane;
       const float st = (!OUT_S32 && m < M) ? __ldg(scale_tok + m) : 0.0f;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * TN;
