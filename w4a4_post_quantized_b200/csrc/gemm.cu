@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
       __syncwarp();  // every lane is done reading the previous tile's constants
 #pragma unroll
-      for (int j = lane; j < TN; j += 32) {
+      for (int j = lane; j < ((!OUT_S32 && P::A_TMEM) ? 0 : TN); j += 32) {
         const int n = nb * TN + j;
         const bool in = n < N;  // the last tile of a ragged N
         coff[j] = 0x4B400000 - ((B_PACKED || !in) ? 0 : 8 * __ldg(colsum + n));
@@ -488,10 +488,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t pk[2][2][8];  // [half][row sub-block][j]: bf16 pair of (row, columns 8j + tc + {0,1})
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int c = c0 + 8 * j + tc;
-            const int2 o = *reinterpret_cast<const int2 *>(coff + c);
-            const float2 scl = *reinterpret_cast<const float2 *>(csc + c);
-            const float2 bi = *reinterpret_cast<const float2 *>(cbi + c);
+            const int n = nb * TN + c0 + 8 * j + tc;  // N is even: the pair is all in or all out
+            int2 o = make_int2(0x4B400000, 0x4B400000);
+            float2 scl = make_float2(0.0f, 0.0f), bi = make_float2(0.0f, 0.0f);
+            if (n < N) {
+              const int2 cs2 = __ldg(reinterpret_cast<const int2 *>(colsum + n));
+              o = make_int2(0x4B400000 - 8 * cs2.x, 0x4B400000 - 8 * cs2.y);
+              scl = __ldg(reinterpret_cast<const float2 *>(scale_ch + n));
+              bi = __ldg(reinterpret_cast<const float2 *>(bias + n));
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
