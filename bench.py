@@ -262,6 +262,21 @@ def run_ours(args, wl, world, rank, local):
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
+        # each kernel alone, launched back to back over the same rotating
+        # buffers (consecutive launches overlap their setup as in a step):
+        # the per-launch durations the rooflines use
+        n_iso = max(3, min(args.steps, 500))
+        iso = {}
+        for name, fn in (("quant", lambda j: w4a4.w4a4_quantize_act(Xs[j], pw.inv_smooth, flags,
+                                                                     qx=QX[j], scale_tok=ST[j])),
+                         ("gemm", lambda j: w4a4.w4a4_linear(QX[j], ST[j], pw, Y=Ys[j]))):
+            k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            k0.record(stream)
+            for i in range(n_iso):
+                fn(i % NSETS)
+            k1.record(stream)
+            torch.cuda.synchronize()
+            iso[name] = max_over_ranks(world, k0.elapsed_time(k1)) / n_iso
         # attribution pass (not part of `value`): the same steps with an event
         # between the two kernels, for each kernel's duration.  An event between
         # them keeps the GEMM from overlapping the quantize kernel's tail, so
@@ -277,8 +292,9 @@ def run_ours(args, wl, world, rank, local):
         torch.cuda.synchronize()
     status = w4a4.w4a4_get_device_status()
     elapsed_ms = max_over_ranks(world, t0.elapsed_time(t1))
-    q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evq)
-    g_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evq)
+    q_step_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evq)
+    g_step_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evq)
+    q_ms, g_ms = iso["quant"], iso["gemm"]
     ms_step = elapsed_ms / args.steps
     ops = 2.0 * M * N * K
     value = world * ops * args.steps / (elapsed_ms * 1e-3) / 1e12
@@ -352,11 +368,15 @@ def run_ours(args, wl, world, rank, local):
                 "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
                 "traffic": profile_traffic("gemm.cu", f"gemm_{args.workload}"),
                 "peak_note": f"int8 = {INT8_PER_BF16:g} x {peaks['src']} bf16 burst {peaks['bf16']} TFLOP/s",
-                "ms_per_launch": g_ms, "algorithmic_ops_per_launch": ops}
+                "ms_per_launch": g_ms, "algorithmic_ops_per_launch": ops,
+                "ms_per_launch_in_step": g_step_ms,
+                "timing": f"CUDA events around {n_iso} back-to-back launches of this kernel alone; "
+                          "ms_per_launch_in_step: events between the two kernels of a step"}
     roofline_q = {"bound": "hbm", "kernel": "quantize_rows_kernel", "achieved": q_gbs,
                   "peak": peaks["hbm"], "unit": "GB/s", "frac": q_gbs / peaks["hbm"],
                   "traffic": profile_traffic("quant.cu", f"quant_{args.workload}"),
-                  "ms_per_launch": q_ms, "algorithmic_bytes_per_launch": q_bytes}
+                  "ms_per_launch": q_ms, "algorithmic_bytes_per_launch": q_bytes,
+                  "ms_per_launch_in_step": q_step_ms}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
