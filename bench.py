@@ -47,6 +47,22 @@ WORKLOADS = {
     "c3_fc2": dict(frames=8, K=4096, N=1024,
                    desc="VGGT MLP fc2 (GELU on input), 8 frames: M=10992, K=4096, N=1024", gelu=True),
 }
+# Multi-layer workloads: the four linears of a transformer block (fc2 takes
+# fc1's output through GELU, folded into its quantize kernel; the other
+# layers take synthetic activations, since attention and normalisation sit
+# between them), repeated over `blocks` blocks with fresh weights per layer.
+STACKS = {
+    "c3_mlp_pair": dict(frames=8, blocks=1, layers=[("fc1", 1024, 4096), ("fc2", 4096, 1024)],
+                        desc="VGGT MLP pair, 8 frames: fc1 1024->4096, GELU, fc2 4096->1024, M=10992"),
+    "c4_global_block": dict(frames=32, blocks=1,
+                            layers=[("qkv", 1024, 3072), ("proj", 1024, 1024), ("fc1", 1024, 4096),
+                                    ("fc2", 4096, 1024)],
+                            desc="global-attention block's four linears, 32 frames: M=43968"),
+    "c5_full_stack": dict(frames=64, blocks=48,
+                          layers=[("qkv", 1024, 3072), ("proj", 1024, 1024), ("fc1", 1024, 4096),
+                                  ("fc2", 4096, 1024)],
+                          desc="48 blocks x the four linears, 64 frames: M=87936"),
+}
 METRIC = "W4A4 linear TOPS & tokens/s on VGGT shapes, % of INT8 TC peak / HBM BW"
 NSETS = 4          # input/output buffer sets rotated so no step finds its inputs in L2
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput ratio (4.5 / 2.25 POPS)
@@ -417,13 +433,133 @@ def run_ours(args, wl, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_stack(args, st, world, rank, local):
+    """A block (or stack of blocks) of quantized linears: one step = every
+    layer once, in order, on one batch of M tokens."""
+    import torch
+    from w4a4_post_quantized_b200 import w4a4
+    M = st["frames"] * synth.FRAME_TOKENS
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    layers = [(b, name, K, N) for b in range(st["blocks"]) for (name, K, N) in st["layers"]]
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    # inputs: two synthetic activation sets (K = 1024) rotate over the blocks;
+    # weights: fresh per layer (seeded normal(0, 0.02^2) / (0, 0.01^2) drawn on
+    # the device: a stack holds up to 192 of them), prepared untimed
+    Xp = [bf16(synth.activations(M, 1024, seed=1000 * rank + 10 + i)) for i in range(2)]
+    C = synth.calibration_rows(M)
+    gen = torch.Generator(device=dev)
+    pws = []
+    for i, (b, name, K, N) in enumerate(layers):
+        gen.manual_seed(1000 * rank + 7 * i + 1)
+        W = (torch.randn((N, K), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+        bias = (torch.randn(N, generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+        Xc = Xp[b % 2][:C] if K == 1024 else torch.nn.functional.gelu(
+            (torch.randn((C, K), generator=gen, device=dev))).to(torch.bfloat16)
+        pws.append(w4a4.w4a4_prepare_weights(W, bias, Xc))
+        del W
+    Ys = {name: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (name, K, N) in st["layers"]}
+    ws = torch.empty(max(w4a4.w4a4_workspace_bytes(M, K) for (_, _, K, _) in layers), dtype=torch.uint8,
+                     device=dev)
+    torch.cuda.synchronize()
+    ops_step = sum(2.0 * M * N * K for (_, _, K, N) in layers)
+
+    def run_layer(i, b, name, K, N):
+        x = Ys["fc1"] if name == "fc2" else Xp[b % 2]
+        w4a4.w4a4_linear_fused(x, pws[i], Y=Ys[name], workspace=ws,
+                               flags=w4a4.W4A4_FLAG_GELU if name == "fc2" else 0)
+
+    def step():
+        for i, (b, name, K, N) in enumerate(layers):
+            run_layer(i, b, name, K, N)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    w4a4.w4a4_clear_device_status()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        # per-layer-shape attribution: events around each layer of one step
+        per = {name: 0.0 for (name, _, _) in st["layers"]}
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+        for i, (b, name, K, N) in enumerate(layers):
+            ev[i][0].record(stream)
+            run_layer(i, b, name, K, N)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        for (e0, e1), (b, name, K, N) in zip(ev, layers):
+            per[name] += e0.elapsed_time(e1)
+    status = w4a4.w4a4_get_device_status()
+    elapsed_ms = max_over_ranks(world, t0.elapsed_time(t1))
+    ms_step = elapsed_ms / args.steps
+    value = world * ops_step * args.steps / (elapsed_ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    int8_peak = peaks["bf16"] * INT8_PER_BF16
+    per_layer = {}
+    for (name, K, N) in st["layers"]:
+        t = per[name] / st["blocks"]
+        per_layer[name] = {"K": K, "N": N, "ms_per_layer": t,
+                           "tops": 2.0 * M * N * K / (t * 1e-3) / 1e12}
+    # end to end: the first layer's input from pinned host memory, the last
+    # layer's output back, around one whole step
+    Xh = torch.empty((M, 1024), dtype=torch.bfloat16, pin_memory=True)
+    Xh.copy_(Xp[0].cpu())
+    last = st["layers"][-1]
+    Yh = torch.empty((M, last[2]), dtype=torch.bfloat16, pin_memory=True)
+    n_e2e = max(3, min(args.steps, args.e2e_steps))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a0.record(stream)
+    for _ in range(n_e2e):
+        Xp[0].copy_(Xh, non_blocking=True)
+        step()
+        Yh.copy_(Ys[last[0]], non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / n_e2e
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s4xs4->s32 (bf16 in/out, fp32 transform)",
+        "data": "synthetic (activations: seeded heavy-tailed generator; weights: seeded normal on device)",
+        "tokens_per_s": world * M * args.steps / (elapsed_ms * 1e-3),
+        "config": {"workload": st["desc"], "M": M, "blocks": st["blocks"],
+                   "layers": [f"{n} {K}->{N}" for (n, K, N) in st["layers"]],
+                   "parallelism": f"dp{world} (independent replicas)"},
+        "clocks": clk.summary(),
+        "e2e": {"value": world * ops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 2 * M * 1024, "d2h_bytes_per_step": 2 * M * last[2],
+                "api": "w4a4_linear_fused per layer; input copied in, last output copied out, same stream"},
+        "gpu_launches": 2 * len(layers) * args.steps,
+        "per_layer": per_layer,
+        "roofline": {"bound": "tensor", "kernel": "w4a4_gemm_kernel + quantize_rows_kernel (whole stack)",
+                     "achieved": value / world, "peak": int8_peak, "unit": "TOPS",
+                     "frac": value / world / int8_peak, "traffic": None},
+        "device_status": status,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c2_frame_qkv")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(STACKS), default="c2_frame_qkv")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--e2e-chunk", type=int, default=1408, help="row chunk of the host-buffer call")
     ap.add_argument("--cpu-rows", type=int, default=512)
@@ -431,9 +567,24 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    wl = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.workload in STACKS:
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable":
+                                  "multi-layer workloads are timed on the GPU only; the oracle "
+                                  "reference arm covers the single-layer workloads"}), flush=True)
+            return
+        world, rank, local = dist_setup()
+        try:
+            run_stack(args, STACKS[args.workload], world, rank, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
+    wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl, world, rank)
         return
