@@ -369,9 +369,23 @@ def run_ours(args, wl, world, rank, local):
         b1.record(stream)
         torch.cuda.synchronize()
         m7[mode] = max_over_ranks(world, b0.elapsed_time(b1)) / n7 * 1e3
+    # quantization quality of both modes on the first frame of the batch (the
+    # heavy-tailed special-token rows included): SQNR of Y against the
+    # unquantized product of the same bf16 inputs, computed in fp64 by torch
+    rows = synth.calibration_rows(M)
+    xr = Xs[0][:rows]
+    if gelu:  # the layer's input is GELU(x) in bf16
+        xr = torch.nn.functional.gelu(xr.float()).to(torch.bfloat16)
+    ref = (xr.double() @ W.double().t() + b.double())
+    sq = {}
+    for mode, p, fl in (("dsfq", pw, flags), ("plain", pw_plain, flags | w4a4.W4A4_FLAG_PLAIN)):
+        y = w4a4.w4a4_linear_fused(Xs[0][:rows], p, flags=fl).double()
+        sq[mode] = float(10.0 * torch.log10((ref ** 2).sum() / ((y - ref) ** 2).sum()))
+    torch.cuda.synchronize()
     dsfq_overhead = {"dsfq_us_per_step": m7["dsfq"], "plain_us_per_step": m7["plain"],
                      "overhead_pct": 100.0 * (m7["dsfq"] - m7["plain"]) / m7["plain"],
-                     "steps": n7, "pages_figure_pct": 0.2}
+                     "steps": n7, "pages_figure_pct": 0.2,
+                     "sqnr_db": sq, "sqnr_rows": rows}
     weight_bytes = {"packed_int4": N * K // 2 + 12 * N + 4 * K, "bf16": 2 * N * K + 2 * N,
                     "expanded_int8_copy": N * K + 4 * N,
                     "ratio_bf16_over_packed": (2 * N * K + 2 * N) / (N * K // 2 + 12 * N + 4 * K)}

@@ -290,6 +290,28 @@ def linear(X_bf16, pw: PreparedWeights, gelu: bool = False, decision: str = "f64
     return Y, qx, dt, acc
 
 
+def linear_ablation(X_bf16, W_bf16, bias_bf16, Xcal_bf16, rotate_on: bool, smooth_on: bool,
+                    alpha: float = 0.5) -> np.ndarray:
+    """The quantized linear with either half of DSFQ switched off, for the
+    pages' ablation of "rotation + scaling" [ROT][SMOOTH]: rotation of X and W
+    along the input features (rotate_on), then smoothing factors computed on
+    the (rotated or not) calibration activations and weights (smooth_on, else
+    s = 1), then per-token / per-channel symmetric int4 [PTQ][GRAN], the
+    integer product and the dequantization.  Both on is DSFQ, both off is
+    plain quantization.  Returns Y fp64 [M, N]."""
+    W = bf16_to_f64(W_bf16)
+    N, K = W.shape
+    bias = np.zeros(N) if bias_bf16 is None else bf16_to_f64(bias_bf16)
+    X = bf16_to_f64(np.asarray(X_bf16, np.uint16))
+    Xc = bf16_to_f64(np.asarray(Xcal_bf16, np.uint16))
+    if rotate_on:
+        W, X, Xc = rotate(W), rotate(X), rotate(Xc)
+    s = smooth_factors(Xc, W, alpha) if smooth_on else np.ones(K)
+    qw, dc = quantize_rows(W * s[None, :], 4)
+    qx, dt = quantize_rows(X / s[None, :], 4)
+    return dequant(int_gemm(qx, qw), dt, dc, bias)
+
+
 def reference_fp(X_bf16, W_bf16, bias_bf16, gelu: bool = False) -> np.ndarray:
     """Unquantized layer X W^T + b in fp64 from the same bf16 inputs (for SQNR)."""
     Xb = gelu_bf16(X_bf16) if gelu else np.asarray(X_bf16, np.uint16)
