@@ -323,3 +323,12 @@ def test_dsfq_ablation_on_heavy_tailed_data():
     pw = oracle.prepare_weights(W, b, X)
     np.testing.assert_allclose(oracle.linear(X, pw)[0], oracle.linear_ablation(X, W, b, X, True, True),
                                rtol=0, atol=0)
+
+
+def test_ablation_plain_matches_plain_path():
+    """Both halves off is the plain quantized linear of prepare_weights(plain=True)."""
+    X = synth.activations(300, 1024, seed=31)
+    W, b = synth.weights(256, 1024, seed=32), synth.bias(256, seed=33)
+    pw = oracle.prepare_weights(W, b, X, plain=True)
+    np.testing.assert_allclose(oracle.linear(X, pw, plain=True)[0],
+                               oracle.linear_ablation(X, W, b, X, False, False), rtol=0, atol=0)
