@@ -233,7 +233,7 @@ def matmul_nt(X, W, bias=None) -> np.ndarray:
 @dataclasses.dataclass
 class PreparedWeights:
     """Offline result of DSFQ weight preparation for one linear layer."""
-    qw: np.ndarray        # int8 [N, K] codes of W_hat = rotate(W) * s
+    qw: np.ndarray        # int8 [N, K] codes of W_hat = rotate(W) * s (bits-bit)
     delta_ch: np.ndarray  # fp64 [N] per-output-channel step
     bias: np.ndarray      # fp64 [N]
     s: np.ndarray         # fp64 [K] smoothing factors
@@ -241,7 +241,7 @@ class PreparedWeights:
 
 
 def prepare_weights(W_bf16, bias_bf16, Xcal_bf16, alpha: float = 0.5,
-                    decision: str = "f64", plain: bool = False) -> PreparedWeights:
+                    decision: str = "f64", plain: bool = False, bits: int = 4) -> PreparedWeights:
     """Offline weight side of DSFQ, in the pages' order:
     rotate W along its input features [ROT]; smoothing factors from the
     rotated calibration activations and rotated weights [SMOOTH]; scale the
@@ -249,7 +249,12 @@ def prepare_weights(W_bf16, bias_bf16, Xcal_bf16, alpha: float = 0.5,
     channel symmetric int4 quantization [PTQ][GRAN].
 
     plain=True is the baseline without DSFQ (no rotation, s = 1), used only
-    for the ablation of the pages' "rotation + scaling" claim."""
+    for the ablation of the pages' "rotation + scaling" claim.
+
+    bits=8 is the W8A8 setting the results of the summary page of
+    "量化視覺幾何基礎變換器" (lsdiaocha.cn, camera-pose paragraph) report
+    beside W4A4: the same steps with the symmetric 8-bit quantizer of [PTQ]
+    (step = absmax / 127)."""
     W = bf16_to_f64(W_bf16)
     N, K = W.shape
     bias = np.zeros(N) if bias_bf16 is None else bf16_to_f64(bias_bf16)
@@ -260,7 +265,7 @@ def prepare_weights(W_bf16, bias_bf16, Xcal_bf16, alpha: float = 0.5,
         Wt = rotate(W)
         Xt = rotate(bf16_to_f64(Xcal_bf16))
         s = smooth_factors(Xt, Wt, alpha)
-    qw, dc = quantize_rows(Wt * s[None, :], 4, decision)
+    qw, dc = quantize_rows(Wt * s[None, :], bits, decision)
     return PreparedWeights(qw=qw, delta_ch=dc, bias=bias, s=s, Wt=Wt)
 
 
@@ -274,17 +279,19 @@ def act_hat(X_bf16, s, gelu: bool = False, plain: bool = False) -> np.ndarray:
     return rotate(X) / np.asarray(s, np.float64)[None, :]
 
 
-def quantize_act(X_bf16, s, gelu: bool = False, decision: str = "f64", plain: bool = False):
-    """Per-token symmetric int4 codes of the rotated, smoothed activations;
-    returns (codes int8 [M, K], delta_tok [M])."""
-    return quantize_rows(act_hat(X_bf16, s, gelu, plain), 4, decision)
+def quantize_act(X_bf16, s, gelu: bool = False, decision: str = "f64", plain: bool = False,
+                 bits: int = 4):
+    """Per-token symmetric bits-bit codes (int4 by default, int8 for W8A8) of
+    the rotated, smoothed activations; returns (codes int8 [M, K], delta_tok [M])."""
+    return quantize_rows(act_hat(X_bf16, s, gelu, plain), bits, decision)
 
 
 def linear(X_bf16, pw: PreparedWeights, gelu: bool = False, decision: str = "f64",
-           plain: bool = False):
+           plain: bool = False, bits: int = 4):
     """The quantized linear end to end: Y = (Qx Qw^T) * delta_tok * delta_ch + b.
+    bits must equal the bit width pw was prepared with.
     Returns (Y fp64 [M, N], qx, delta_tok, acc)."""
-    qx, dt = quantize_act(X_bf16, pw.s, gelu, decision, plain)
+    qx, dt = quantize_act(X_bf16, pw.s, gelu, decision, plain, bits)
     acc = int_gemm(qx, pw.qw)
     Y = dequant(acc, dt, pw.delta_ch, pw.bias)
     return Y, qx, dt, acc
