@@ -82,6 +82,14 @@ typedef enum {
                                  per-channel int4 quantization (the baseline that
                                  DSFQ is measured against); must match between
                                  prepare_weights and the activation calls */
+#define W4A4_FLAG_INT8  0x4u  /* the W8A8 setting (reported beside W4A4 in the
+                                 results of the summary page of "量化視覺幾何基礎變換器",
+                                 lsdiaocha.cn, camera-pose paragraph): the same
+                                 steps with the symmetric 8-bit quantizer of [PTQ],
+                                 delta = absmax/127, one signed int8 code per byte
+                                 in natural order, for activations and weights;
+                                 must match between prepare_weights and the
+                                 activation calls */
 
 /* Prepared weights of one linear layer.  The caller allocates every array
  * (device memory) with the sizes given and keeps ownership. */
@@ -96,10 +104,13 @@ typedef struct {
     int8_t *qw8;          /* optional [N, K] int8: the codes of qw widened to 8 bits in the
                              order the tensor-core kernel consumes them (see
                              w4a4_expand_weights).  NULL: the GEMM widens the packed qw on
-                             every tile instead (no extra memory, lower throughput). */
+                             every tile instead (no extra memory, lower throughput).
+                             With W4A4_FLAG_INT8: required, the [N, K] 8-bit codes of W^
+                             in natural order (qw and colsum are then unused, may be NULL) */
     int32_t *colsum;      /* [N] sum over k of the int4 codes of row n; required when qw8
                              is set (NULL otherwise) */
-    uint32_t flags;       /* W4A4_FLAG_PLAIN when prepared without DSFQ */
+    uint32_t flags;       /* W4A4_FLAG_PLAIN when prepared without DSFQ, W4A4_FLAG_INT8 for
+                             8-bit codes */
 } w4a4_weights_t;
 
 /* Bytes of workspace w4a4_linear_fused needs for M tokens of width K:
@@ -107,15 +118,22 @@ typedef struct {
  * per-token steps (4*M).  Returns 0 for an unsupported K. */
 size_t w4a4_workspace_bytes(int64_t M, int32_t K);
 
+/* The same for the given flags: with W4A4_FLAG_INT8 the codes take M*K bytes
+ * (rounded up to 256), followed by the 4*M bytes of steps.  Returns 0 for an
+ * unsupported K or an unknown flag. */
+size_t w4a4_workspace_bytes_ex(int64_t M, int32_t K, uint32_t flags);
+
 /* Offline weight preparation [ROT][SMOOTH][PTQ][GRAN].
  *   W       [N, K] bf16 weights; bias [N] bf16 or NULL;
  *   X_calib [M_calib, K] bf16 calibration activations (M_calib >= 1), used
  *           only for the per-channel activation maxima of the smoothing step;
  *   alpha   smoothing exponent in [0, 1] (the page uses 0.5);
- *   flags   0 or W4A4_FLAG_PLAIN (then s = 1 and no rotation; X_calib may be NULL);
+ *   flags   0, W4A4_FLAG_PLAIN (then s = 1 and no rotation; X_calib may be
+ *           NULL) and/or W4A4_FLAG_INT8 (8-bit codes into out->qw8);
  *   out     caller-allocated arrays to fill; out->N and out->K must equal N
- *           and K; out->flags is set to (flags & W4A4_FLAG_PLAIN); when
- *           out->qw8 is set, qw8 and colsum are filled too (w4a4_expand_weights).
+ *           and K; out->flags is set to (flags & (W4A4_FLAG_PLAIN |
+ *           W4A4_FLAG_INT8)); for 4-bit codes, when out->qw8 is set, qw8 and
+ *           colsum are filled too (w4a4_expand_weights).
  * Rounding decisions are taken in binary32.  A channel whose activation or
  * weight maximum is zero gets s_j = 1. */
 w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_t N, int32_t K,
@@ -126,7 +144,8 @@ w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_
  * within every group of 8 consecutive codes k = 8g..8g+7 the bytes hold codes
  * 8g+0, 2, 4, 6, 1, 3, 5, 7, as signed int8) and writes w->colsum[n] =
  * sum_k code[n, k].  Both arrays must be set.  Not on the pages: weights are
- * static, so the per-tile widening of B is hoisted to preparation time. */
+ * static, so the per-tile widening of B is hoisted to preparation time.
+ * W4A4_ERR_ARG for weights prepared with W4A4_FLAG_INT8 (nothing to widen). */
 w4a4_status w4a4_expand_weights(w4a4_weights_t *w, void *stream);
 
 /* Online activation quantizer [ROT][SMOOTH][PTQ][GRAN]: for each of the M
@@ -134,21 +153,25 @@ w4a4_status w4a4_expand_weights(w4a4_weights_t *w, void *stream);
  * multiplication by inv_smooth [K], per-token step delta = absmax/7 written to
  * scale_tok [M] (fp32), codes round-half-even(x / delta) packed into qx
  * [M, K/2].  With W4A4_FLAG_PLAIN the rotation and smoothing are skipped
- * (inv_smooth may then be NULL).  Inputs must be finite. */
+ * (inv_smooth may then be NULL).  With W4A4_FLAG_INT8, delta = absmax/127 and
+ * qx [M, K] holds one int8 code per element.  Inputs must be finite. */
 w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const float *inv_smooth,
                               uint8_t *qx, float *scale_tok, uint32_t flags, void *stream);
 
 /* Quantized linear from codes: Y [M, N] bf16 =
  *   round-to-nearest-even( (qx qw^T)[m,n] * scale_tok[m] * w->scale_ch[n] + w->bias[n] ).
  * The integer product is exact (int32 accumulation on the tensor cores); the
- * epilogue is fp32. */
+ * epilogue is fp32.  For weights prepared with W4A4_FLAG_INT8, qx is [M, K]
+ * int8 (w4a4_quantize_act with W4A4_FLAG_INT8). */
 w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
                         const w4a4_weights_t *w, uint16_t *Y, void *stream);
 
 /* Quantized linear from bf16 activations: w4a4_quantize_act (with
  * w->inv_smooth and the given flags) into `workspace`, then w4a4_linear.
- * workspace must hold w4a4_workspace_bytes(M, w->K) bytes (workspace_bytes
- * says how many it holds); its contents afterwards are the codes and steps. */
+ * workspace must hold w4a4_workspace_bytes_ex(M, w->K, flags) bytes
+ * (workspace_bytes says how many it holds); its contents afterwards are the
+ * codes and steps.  flags must carry the same W4A4_FLAG_PLAIN and
+ * W4A4_FLAG_INT8 bits as w->flags (W4A4_ERR_ARG otherwise). */
 w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t *w, uint16_t *Y,
                               void *workspace, size_t workspace_bytes, uint32_t flags,
                               void *stream);
@@ -166,9 +189,10 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
  * w4a4_linear_fused without the workspace: the codes and steps go to a scratch
  * array of W4A4_NOALLOC_SCRATCH_BYTES inside the library instead, so the call
  * allocates nothing.
- *   - Accepts M with w4a4_workspace_bytes(M, w->K) <= W4A4_NOALLOC_SCRATCH_BYTES
- *     (M <= 16256 tokens at K = 1024, M <= 4088 at K = 4096); larger M returns
- *     W4A4_ERR_SHAPE.
+ *   - Accepts M with w4a4_workspace_bytes_ex(M, w->K, flags) <=
+ *     W4A4_NOALLOC_SCRATCH_BYTES (4-bit codes: M <= 16256 tokens at K = 1024,
+ *     M <= 4088 at K = 4096; 8-bit codes: about half of that); larger M
+ *     returns W4A4_ERR_SHAPE.
  *   - The first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
@@ -208,8 +232,8 @@ w4a4_status w4a4_host_pipe_destroy(w4a4_host_pipe_t *pipe);
 
 /* Device workspace for w4a4_linear_fused_host: W4A4_PIPE_DEPTH slots, each
  * holding one chunk's X (2 chunk_rows K bytes), Y (2 chunk_rows N bytes),
- * codes and steps (w4a4_workspace_bytes(chunk_rows, K)), each part 256-byte
- * aligned. */
+ * codes and steps (w4a4_workspace_bytes_ex(chunk_rows, K, W4A4_FLAG_INT8),
+ * room for either code width), each part 256-byte aligned. */
 size_t w4a4_host_workspace_bytes(int64_t chunk_rows, int32_t K, int32_t N);
 
 /* Y_host [M, N] bf16 = w4a4_linear_fused(X_host [M, K] bf16) with X_host and
@@ -229,7 +253,8 @@ w4a4_status w4a4_linear_fused_host(const uint16_t *X_host, int64_t M, const w4a4
 /* Integer product only: acc [M, N] int32 = sum_k qx[m, k] * code_w[n, k] for
  * packed activation codes qx [M, K/2] and the weight codes of *w (w->qw8 and
  * w->colsum when set, else the packed w->qw; scale_ch, bias and the smoothing
- * arrays are not used and may be NULL).  Same tensor-core kernel as
+ * arrays are not used and may be NULL); for weights with W4A4_FLAG_INT8, qx
+ * [M, K] and w->qw8 hold int8 codes.  Same tensor-core kernel as
  * w4a4_linear with the raw accumulators written out: the integer product is
  * exact. */
 w4a4_status w4a4_gemm_s32(const uint8_t *qx, int64_t M, const w4a4_weights_t *w, int32_t *acc,

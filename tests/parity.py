@@ -22,14 +22,16 @@ import numpy as np
 U = 2.0 ** -24
 
 
-def tie_bound(x_in: np.ndarray, mult: np.ndarray, ratio: np.ndarray, amax: np.ndarray, K: int) -> np.ndarray:
+def tie_bound(x_in: np.ndarray, mult: np.ndarray, ratio: np.ndarray, amax: np.ndarray, K: int,
+              qmax: float = 7.0) -> np.ndarray:
     """Per-row bound on |ratio_cuda - ratio_exact| (rows of x_in are the
-    transform's inputs, mult the per-channel multipliers)."""
+    transform's inputs, mult the per-channel multipliers, qmax the largest
+    code: 7 for int4, 127 for int8)."""
     l1 = np.sum(np.abs(x_in), axis=1)
     e_val = np.log2(K) * U * l1 / np.sqrt(K) * np.max(np.abs(mult))
     with np.errstate(divide="ignore", invalid="ignore"):
-        e_ratio = np.where(amax > 0, 7.0 * e_val / amax, 0.0)
-    return 4.0 * (e_ratio + 8 * U * 7.0 * (1 + np.max(np.abs(ratio), axis=1) / 7.0))
+        e_ratio = np.where(amax > 0, qmax * e_val / amax, 0.0)
+    return 4.0 * (e_ratio + 8 * U * qmax * (1 + np.max(np.abs(ratio), axis=1) / qmax))
 
 
 def compare_codes(got: np.ndarray, want: np.ndarray, ratio: np.ndarray, bound_row: np.ndarray,

@@ -59,6 +59,8 @@ def _setup(lib):
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
     lib.w4a4_workspace_bytes.restype = ctypes.c_size_t
     lib.w4a4_workspace_bytes.argtypes = [i64, i32]
+    lib.w4a4_workspace_bytes_ex.restype = ctypes.c_size_t
+    lib.w4a4_workspace_bytes_ex.argtypes = [i64, i32, ctypes.c_uint32]
     lib.w4a4_quantize_act.argtypes = [vp, i64, i32, vp, vp, vp, ctypes.c_uint32, vp]
     lib.w4a4_linear.argtypes = [vp, vp, i64, ctypes.POINTER(WeightsT), vp, vp]
     lib.w4a4_linear_fused.argtypes = [vp, i64, ctypes.POINTER(WeightsT), vp, vp, ctypes.c_size_t,
@@ -83,6 +85,48 @@ def test_workspace_bytes(lib):
     assert lib.w4a4_workspace_bytes(0, 1024) == 0
     assert lib.w4a4_workspace_bytes(10, 1000) == 0
     assert lib.w4a4_workspace_bytes(-1, 1024) == 0
+    ex = lib.w4a4_workspace_bytes_ex
+    for M, K in [(10992, 1024), (3, 4096), (0, 1024)]:
+        assert ex(M, K, 0) == lib.w4a4_workspace_bytes(M, K) == ex(M, K, 2) == ex(M, K, 1)
+    assert ex(10992, 1024, 4) == 10992 * 1024 + 4 * 10992          # 8-bit codes: one byte each
+    assert ex(3, 4096, 4 | 2) == 12288 + 12
+    assert ex(10, 1024, 0x80) == 0 and ex(10, 1000, 4) == 0
+
+
+INT8 = 0x4
+
+
+def _weights8(N=1024, K=1024, base=A, flags=INT8):
+    # 8-bit weights: codes in qw8, no packed qw and no colsum
+    return WeightsT(N, K, None, base + 0x1000, base + 0x2000, base + 0x3000, base + 0x4000,
+                    base + 0x5000, None, flags)
+
+
+def test_int8_variant_argument_checks(lib):
+    """W4A4_FLAG_INT8 (W8A8): weights need qw8 only; the flag must match between
+    the weights and the fused call; expand_weights refuses 8-bit weights; the
+    workspace check uses the 8-bit code size."""
+    _setup(lib)
+    w8 = _weights8()
+    L, F, G, E, P = (lib.w4a4_linear, lib.w4a4_linear_fused, lib.w4a4_gemm_s32,
+                     lib.w4a4_expand_weights, lib.w4a4_prepare_weights)
+    assert L(A, A, 0, ctypes.byref(w8), A, None) == 0                    # accepted (empty: no-op)
+    no_codes = _weights8()
+    no_codes.qw8 = None
+    assert L(A, A, 10, ctypes.byref(no_codes), A, None) == 1
+    assert G(A, 0, ctypes.byref(w8), A, None) == 0
+    assert G(A, 10, ctypes.byref(no_codes), A, None) == 1
+    need4 = lib.w4a4_workspace_bytes(100, 1024)
+    need8 = lib.w4a4_workspace_bytes_ex(100, 1024, INT8)
+    assert F(A, 100, ctypes.byref(w8), A, A, need8, 0, None) == 1       # flag missing on the call
+    assert F(A, 100, ctypes.byref(_weights()), A, A, need8, INT8, None) == 1  # 4-bit weights
+    assert F(A, 100, ctypes.byref(w8), A, A, need4, INT8, None) == 2    # 4-bit-sized workspace
+    assert E(ctypes.byref(_weights(flags=INT8)), None) == 1
+    assert P(A, None, 1024, 1024, A, 10, 0.5, INT8, ctypes.byref(no_codes), None) == 1
+    assert P(A, None, 1024, 1024, A, 10, 0.5, 0x8, ctypes.byref(w8), None) == 4   # unknown flag
+    q = lib.w4a4_quantize_act
+    assert q(A, 0, 1024, A, A, A, INT8, None) == 0
+    assert q(A, 10, 1024, None, A, A, INT8, None) == 1                   # DSFQ needs inv_smooth
 
 
 def test_quantize_act_argument_checks(lib):
@@ -168,11 +212,12 @@ def test_host_pipeline_argument_checks(lib):
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     lib.w4a4_host_workspace_bytes.restype = sz
     lib.w4a4_host_workspace_bytes.argtypes = [i64, i32, i32]
-    lib.w4a4_workspace_bytes.restype = sz
-    lib.w4a4_workspace_bytes.argtypes = [i64, i32]
+    lib.w4a4_workspace_bytes_ex.restype = sz
+    lib.w4a4_workspace_bytes_ex.argtypes = [i64, i32, ctypes.c_uint32]
     r256 = lambda b: (b + 255) // 256 * 256
     for rows, K, N in [(2816, 1024, 3072), (1, 4096, 1024), (300, 1024, 256)]:
-        slot = r256(2 * rows * K) + r256(2 * rows * N) + r256(lib.w4a4_workspace_bytes(rows, K))
+        # the codes part has room for 8-bit codes (either code width fits)
+        slot = r256(2 * rows * K) + r256(2 * rows * N) + r256(lib.w4a4_workspace_bytes_ex(rows, K, 4))
         assert lib.w4a4_host_workspace_bytes(rows, K, N) == 2 * slot
     assert lib.w4a4_host_workspace_bytes(0, 1024, 256) == 0
     f = lib.w4a4_linear_fused_host

@@ -11,7 +11,8 @@
 
 namespace {
 
-constexpr uint32_t kKnownFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN;
+constexpr uint32_t kKnownFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8;
+constexpr uint32_t kWeightFlags = W4A4_FLAG_PLAIN | W4A4_FLAG_INT8;  // fixed at preparation
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool k_ok(int32_t K) { return K == 1024 || K == 4096; }
@@ -22,19 +23,31 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 w4a4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA; }
 
+bool int8_weights(const w4a4_weights_t *w) { return (w->flags & W4A4_FLAG_INT8) != 0; }
+
 w4a4_status check_weights(const w4a4_weights_t *w) {
   if (!w) return W4A4_ERR_ARG;
   if (!k_ok(w->K)) return W4A4_ERR_UNSUPPORTED;
   if (!n_ok(w->N)) return W4A4_ERR_SHAPE;
-  if (!w->qw || !w->scale_ch || !w->bias || !w->smooth || !w->inv_smooth) return W4A4_ERR_ARG;
+  if (w->flags & ~kWeightFlags) return W4A4_ERR_UNSUPPORTED;
+  if (!w->scale_ch || !w->bias || !w->smooth || !w->inv_smooth) return W4A4_ERR_ARG;
+  if (int8_weights(w)) {
+    if (!w->qw8) return W4A4_ERR_ARG;  // the 8-bit codes; qw and colsum are not used
+  } else {
+    if (!w->qw) return W4A4_ERR_ARG;
+    if ((w->qw8 == nullptr) != (w->colsum == nullptr)) return W4A4_ERR_ARG;
+  }
   if (!aligned16(w->qw) || !aligned16(w->scale_ch) || !aligned16(w->bias) || !aligned16(w->smooth) ||
-      !aligned16(w->inv_smooth))
+      !aligned16(w->inv_smooth) || !aligned16(w->qw8) || !aligned16(w->colsum))
     return W4A4_ERR_ALIGN;
-  if (w->flags & ~W4A4_FLAG_PLAIN) return W4A4_ERR_UNSUPPORTED;
-  if ((w->qw8 == nullptr) != (w->colsum == nullptr)) return W4A4_ERR_ARG;
-  if (!aligned16(w->qw8) || !aligned16(w->colsum)) return W4A4_ERR_ALIGN;
   return W4A4_OK;
 }
+
+// code bytes of M rows of width K
+size_t code_bytes(int64_t M, int32_t K, uint32_t flags) {
+  return static_cast<size_t>(M) * ((flags & W4A4_FLAG_INT8) ? K : K / 2);
+}
+int code_bits(uint32_t flags) { return (flags & W4A4_FLAG_INT8) ? 8 : 4; }
 
 w4a4_status check_act(const void *X, int64_t M, int32_t K, const float *inv_smooth, const void *qx,
                       const float *scale_tok, uint32_t flags) {
@@ -54,18 +67,21 @@ w4a4_status check_act(const void *X, int64_t M, int32_t K, const float *inv_smoo
 
 extern "C" {
 
-size_t w4a4_workspace_bytes(int64_t M, int32_t K) {
-  if (!k_ok(K) || !m_ok(M)) return 0;
-  return round256(static_cast<size_t>(M) * (K / 2)) + sizeof(float) * static_cast<size_t>(M);
+size_t w4a4_workspace_bytes_ex(int64_t M, int32_t K, uint32_t flags) {
+  if (!k_ok(K) || !m_ok(M) || (flags & ~kKnownFlags)) return 0;
+  return round256(code_bytes(M, K, flags)) + sizeof(float) * static_cast<size_t>(M);
 }
+
+size_t w4a4_workspace_bytes(int64_t M, int32_t K) { return w4a4_workspace_bytes_ex(M, K, 0); }
 
 w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_t N, int32_t K,
                                  const uint16_t *X_calib, int64_t M_calib, float alpha,
                                  uint32_t flags, w4a4_weights_t *out, void *stream) {
-  if (flags & ~W4A4_FLAG_PLAIN) return W4A4_ERR_UNSUPPORTED;
+  if (flags & ~kWeightFlags) return W4A4_ERR_UNSUPPORTED;
   if (!k_ok(K)) return W4A4_ERR_UNSUPPORTED;
   if (!n_ok(N)) return W4A4_ERR_SHAPE;
   if (!out || !W) return W4A4_ERR_ARG;
+  const bool int8 = (flags & W4A4_FLAG_INT8) != 0;
   if (out->N != N || out->K != K) return W4A4_ERR_SHAPE;
   const bool plain = (flags & W4A4_FLAG_PLAIN) != 0;
   if (!plain) {
@@ -74,9 +90,9 @@ w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_
     if (!(alpha >= 0.0f && alpha <= 1.0f)) return W4A4_ERR_ARG;
     if (!aligned16(X_calib)) return W4A4_ERR_ALIGN;
   }
-  if (!out->qw || !out->scale_ch || !out->bias || !out->smooth || !out->inv_smooth)
+  if (!out->scale_ch || !out->bias || !out->smooth || !out->inv_smooth) return W4A4_ERR_ARG;
+  if (int8 ? !out->qw8 : (!out->qw || (out->qw8 == nullptr) != (out->colsum == nullptr)))
     return W4A4_ERR_ARG;
-  if ((out->qw8 == nullptr) != (out->colsum == nullptr)) return W4A4_ERR_ARG;
   if (!aligned16(out->qw8) || !aligned16(out->colsum)) return W4A4_ERR_ALIGN;
   if (!aligned16(W) || (bias && !aligned16(bias)) || !aligned16(out->qw) ||
       !aligned16(out->scale_ch) || !aligned16(out->bias) || !aligned16(out->smooth) ||
@@ -84,10 +100,13 @@ w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_
     return W4A4_ERR_ALIGN;
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
+  // 4-bit codes packed into qw, or 8-bit codes into qw8 (natural order)
+  uint8_t *codes = int8 ? reinterpret_cast<uint8_t *>(out->qw8) : out->qw;
+  const int bits = code_bits(flags);
   if (plain) {
     if ((e = w4a4::launch_fill(out->smooth, K, 1.0f, st)) != cudaSuccess) return cuda_status(e);
     if ((e = w4a4::launch_fill(out->inv_smooth, K, 1.0f, st)) != cudaSuccess) return cuda_status(e);
-    e = w4a4::launch_quantize_rows(W, N, K, nullptr, out->qw, out->scale_ch, false, false, st);
+    e = w4a4::launch_quantize_rows(W, N, K, nullptr, codes, out->scale_ch, false, false, bits, st);
   } else {
     // column maxima of the rotated calibration activations -> out->smooth,
     // of the rotated weights -> out->inv_smooth; then s and 1/s in place
@@ -96,12 +115,12 @@ w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_
     if ((e = w4a4::launch_colmax(W, N, K, out->inv_smooth, st)) != cudaSuccess) return cuda_status(e);
     if ((e = w4a4::launch_smooth_factors(out->smooth, out->inv_smooth, K, alpha, st)) != cudaSuccess)
       return cuda_status(e);
-    e = w4a4::launch_quantize_rows(W, N, K, out->smooth, out->qw, out->scale_ch, true, false, st);
+    e = w4a4::launch_quantize_rows(W, N, K, out->smooth, codes, out->scale_ch, true, false, bits, st);
   }
   if (e != cudaSuccess) return cuda_status(e);
   if ((e = w4a4::launch_bias_to_f32(bias, out->bias, N, st)) != cudaSuccess) return cuda_status(e);
-  out->flags = flags & W4A4_FLAG_PLAIN;
-  if (out->qw8) return w4a4_expand_weights(out, stream);
+  out->flags = flags & kWeightFlags;
+  if (!int8 && out->qw8) return w4a4_expand_weights(out, stream);
   return W4A4_OK;
 }
 
@@ -110,6 +129,7 @@ w4a4_status w4a4_expand_weights(w4a4_weights_t *w, void *stream) {
   if (!k_ok(w->K)) return W4A4_ERR_UNSUPPORTED;
   if (!n_ok(w->N)) return W4A4_ERR_SHAPE;
   if (!w->qw || !w->qw8 || !w->colsum) return W4A4_ERR_ARG;
+  if (w->flags & W4A4_FLAG_INT8) return W4A4_ERR_ARG;  // 8-bit codes need no widening
   if (!aligned16(w->qw) || !aligned16(w->qw8) || !aligned16(w->colsum)) return W4A4_ERR_ALIGN;
   return cuda_status(w4a4::launch_expand_weights(w->qw, w->N, w->K, w->qw8, w->colsum,
                                                  as_stream(stream)));
@@ -121,7 +141,8 @@ w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const flo
   if (s != W4A4_OK) return s;
   return cuda_status(w4a4::launch_quantize_rows(X, M, K, inv_smooth, qx, scale_tok,
                                                 !(flags & W4A4_FLAG_PLAIN),
-                                                (flags & W4A4_FLAG_GELU) != 0, as_stream(stream)));
+                                                (flags & W4A4_FLAG_GELU) != 0, code_bits(flags),
+                                                as_stream(stream)));
 }
 
 w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
@@ -133,7 +154,7 @@ w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
   if (!qx || !scale_tok || !Y) return W4A4_ERR_ARG;
   if (!aligned16(qx) || !aligned16(scale_tok) || !aligned16(Y)) return W4A4_ERR_ALIGN;
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, scale_tok, w->scale_ch, w->bias, Y, nullptr,
-                   M, w->N, w->K};
+                   M, w->N, w->K, int8_weights(w)};
   return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
 }
 
@@ -143,21 +164,21 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
   w4a4_status s = check_weights(w);
   if (s != W4A4_OK) return s;
   if (flags & ~kKnownFlags) return W4A4_ERR_UNSUPPORTED;
-  if ((flags & W4A4_FLAG_PLAIN) != (w->flags & W4A4_FLAG_PLAIN)) return W4A4_ERR_ARG;
+  if ((flags ^ w->flags) & kWeightFlags) return W4A4_ERR_ARG;
   if (!m_ok(M)) return W4A4_ERR_SHAPE;
   if (M == 0) return W4A4_OK;  // empty input: nothing to read or write
   if (!X || !Y || !workspace) return W4A4_ERR_ARG;
-  if (workspace_bytes < w4a4_workspace_bytes(M, w->K)) return W4A4_ERR_SHAPE;
+  if (workspace_bytes < w4a4_workspace_bytes_ex(M, w->K, flags)) return W4A4_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(Y) || !aligned16(workspace)) return W4A4_ERR_ALIGN;
   uint8_t *qx = static_cast<uint8_t *>(workspace);
-  float *st = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (w->K / 2)));
+  float *st = reinterpret_cast<float *>(qx + round256(code_bytes(M, w->K, flags)));
   cudaStream_t cs = as_stream(stream);
   cudaError_t e = w4a4::launch_quantize_rows(X, M, w->K, w->inv_smooth, qx, st,
                                              !(flags & W4A4_FLAG_PLAIN),
-                                             (flags & W4A4_FLAG_GELU) != 0, cs);
+                                             (flags & W4A4_FLAG_GELU) != 0, code_bits(flags), cs);
   if (e != cudaSuccess) return cuda_status(e);
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, st, w->scale_ch, w->bias, Y, nullptr,
-                   M, w->N, w->K};
+                   M, w->N, w->K, int8_weights(w)};
   return cuda_status(w4a4::launch_gemm(a, cs));
 }
 
@@ -166,14 +187,16 @@ w4a4_status w4a4_gemm_s32(const uint8_t *qx, int64_t M, const w4a4_weights_t *w,
   if (!w) return W4A4_ERR_ARG;
   if (!k_ok(w->K)) return W4A4_ERR_UNSUPPORTED;
   if (!n_ok(w->N) || !m_ok(M)) return W4A4_ERR_SHAPE;
-  if ((w->qw8 == nullptr) != (w->colsum == nullptr)) return W4A4_ERR_ARG;
+  if (w->flags & ~kWeightFlags) return W4A4_ERR_UNSUPPORTED;
+  const bool int8 = int8_weights(w);
+  if (int8 ? !w->qw8 : ((w->qw8 == nullptr) != (w->colsum == nullptr))) return W4A4_ERR_ARG;
   if (M == 0) return W4A4_OK;
   if (!qx || !acc || (!w->qw && !w->qw8)) return W4A4_ERR_ARG;
   if (!aligned16(qx) || !aligned16(acc) || !aligned16(w->qw) || !aligned16(w->qw8) ||
       !aligned16(w->colsum))
     return W4A4_ERR_ALIGN;
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, nullptr, nullptr, nullptr, nullptr, acc,
-                   M, w->N, w->K};
+                   M, w->N, w->K, int8};
   return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
 }
 

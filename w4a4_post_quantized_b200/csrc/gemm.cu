@@ -26,6 +26,11 @@
 //   * packed B (qw8 == NULL): both operands are TMA-staged packed and
 //     sign-extended to int8 in shared memory on every tile (no extra weight
 //     memory, more shared-memory traffic and integer work); tiles 128 x 256.
+//   * int8 (the W8A8 setting): activations and weights carry one 8-bit code
+//     per byte in natural order; TMA loads both straight into the 128-byte
+//     swizzled operand layout and the MMA reads them there (signed x signed).
+//     No widening at all, so comparing it with the expanded path isolates
+//     what the 4-bit codes cost; tiles 128 x 256.
 //
 // Warp roles (one persistent CTA per SM, tiles round-robin, M-major):
 //   warp 0      TMA producer (one thread)
@@ -86,33 +91,42 @@ constexpr int NUM_THREADS = (8 + NUM_EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;     // the whole tensor memory of the SM
 
 // Shared-memory and tensor-memory plan.  TMA stages hold what comes from L2
-// (packed A, and B as int8 or packed).
+// (A packed or int8, B int8 or packed).
 //   expanded B: A is widened into tensor memory (the MMA reads A there), so
 //     shared memory carries only B and the packed A.  Tiles are 128 x 192:
 //     two 192-column accumulators and two widened-A slots of KG k-blocks
 //     (32 columns each) fill the 512 columns.
 //   packed B: A and B are widened into a ring of shared-memory slots; tiles
 //     are 128 x 256.
-template <bool B_PACKED>
+//   int8: A and B arrive as int8 operand tiles; tiles are 128 x 256, two
+//     256-column accumulators.
+enum : int { kExpanded = 0, kPacked = 1, kInt8 = 2 };
+
+template <int MODE>
 struct Plan {
-  static constexpr bool A_TMEM = !B_PACKED;
-  static constexpr int TN = B_PACKED ? BN : 192;     // tile columns
-  static constexpr int STAGES = B_PACKED ? 3 : 5;    // TMA stages
-  static constexpr int KG = B_PACKED ? 1 : 2;        // k-blocks per widen -> MMA handshake
-  static constexpr int WSLOTS = B_PACKED ? 2 : 2;    // widened operand slots
-  static constexpr int OFF_ST_A = 0;                 // packed A  [BM x 64 B]
-  static constexpr int OFF_ST_B = A_PK;              // B: int8 [TN x 128 B] (swizzled) or packed
-  static constexpr int STAGE_BYTES = A_PK + (B_PACKED ? B_PK : TN * BK);
+  static constexpr bool B_PACKED = MODE == kPacked;
+  static constexpr bool A_TMEM = MODE == kExpanded;
+  static constexpr bool A8 = MODE == kInt8;
+  static constexpr bool EPI16 = !B_PACKED;           // 16x256b epilogue fragments
+  static constexpr int TN = A_TMEM ? 192 : BN;       // tile columns
+  static constexpr int STAGES = B_PACKED ? 3 : (A8 ? 4 : 5);  // TMA stages
+  static constexpr int KG = A_TMEM ? 2 : 1;          // k-blocks per widen -> MMA handshake
+  static constexpr int WSLOTS = A8 ? 0 : 2;          // widened operand slots
+  static constexpr int A_ST = A8 ? A_UN : A_PK;      // A bytes of a stage
+  static constexpr int OFF_ST_A = 0;                 // A: packed [BM x 64 B] or int8 [BM x 128 B] (swizzled)
+  static constexpr int OFF_ST_B = A_ST;              // B: int8 [TN x 128 B] (swizzled) or packed
+  static constexpr int STAGE_BYTES = A_ST + (B_PACKED ? B_PK : TN * BK);
   static constexpr int OFF_W = STAGES * STAGE_BYTES;
   static constexpr int OFF_W_A = 0;                  // widened A [BM x 128 B] (swizzled)
   static constexpr int OFF_W_B = A_UN;               // widened B (B_PACKED only)
-  static constexpr int WSLOT_BYTES = A_TMEM ? 0 : A_UN + (B_PACKED ? B_UN : 0);
+  static constexpr int WSLOT_BYTES = B_PACKED ? A_UN + B_UN : 0;
   static constexpr uint32_t TMEM_A0 = 2 * TN;        // first widened-A column (A_TMEM)
   static_assert(!A_TMEM || TMEM_A0 + WSLOTS * KG * 32 <= 512, "tensor-memory budget");
   static constexpr int OFF_EPI = OFF_W + WSLOTS * WSLOT_BYTES;
   static constexpr int OFF_COL = OFF_EPI + NUM_EPI_WARPS * 2 * EPI_BYTES;  // per-warp constants
-  static constexpr int OFF_BAR = OFF_COL + NUM_EPI_WARPS * 3 * TN * 4;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * WSLOTS + 2 * 2 + 1;
+  static constexpr int COL_WORDS = A8 ? 0 : 3 * TN;  // (int8: no code offset, no table)
+  static constexpr int OFF_BAR = OFF_COL + NUM_EPI_WARPS * COL_WORDS * 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * (WSLOTS > 0 ? WSLOTS : 1) + 2 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -120,8 +134,8 @@ struct Plan {
                     WSLOT_BYTES % 1024 == 0 && OFF_EPI % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
   // tcgen05.mma kind::i8 instruction descriptor: s32 D; A unsigned (code + 8)
-  // with expanded B, signed with packed B; B signed; both K-major; 128 x TN.
-  static constexpr uint32_t IDESC = (2u << 4) | ((B_PACKED ? 1u : 0u) << 7) | (1u << 10) |
+  // with expanded B, signed otherwise; B signed; both K-major; 128 x TN.
+  static constexpr uint32_t IDESC = (2u << 4) | ((A_TMEM ? 0u : 1u) << 7) | (1u << 10) |
                                     (static_cast<uint32_t>(TN >> 3) << 17) |
                                     (static_cast<uint32_t>(BM >> 4) << 24);
 };
@@ -204,17 +218,32 @@ __device__ __forceinline__ uint32_t dequant2_bf16(int32_t b0, int32_t b1, float 
   return pack_bf16x2(y0, y1);
 }
 
+// The same for plain accumulators of any size (8-bit codes reach 127^2 K,
+// beyond the 2^22 the biased bit pattern above can hold): converted with
+// round-to-nearest (exact up to 2^24; the relative error stays below 2^-24).
+__device__ __forceinline__ uint32_t dequant2_bf16_cvt(int32_t a0, int32_t a1, float st, float sc0,
+                                                      float sc1, float bi0, float bi1) {
+  const unsigned long long x = f2_pack(__int2float_rn(a0), __int2float_rn(a1));
+  const unsigned long long s = f2_pack(st, st), c = f2_pack(sc0, sc1), b = f2_pack(bi0, bi1);
+  unsigned long long m, y;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(m) : "l"(s), "l"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(y) : "l"(x), "l"(m), "l"(b));
+  float y0, y1;
+  f2_unpack(y, y0, y1);
+  return pack_bf16x2(y0, y1);
+}
 
-template <bool B_PACKED, bool OUT_S32>
+template <int MODE, bool OUT_S32>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmY, const float *__restrict__ scale_tok,
                      const float *__restrict__ scale_ch, const float *__restrict__ bias,
                      const int32_t *__restrict__ colsum, int32_t *__restrict__ acc_out, int M, int N,
                      int num_n_tiles, int num_tiles, int num_kb) {
-  using P = Plan<B_PACKED>;
+  using P = Plan<MODE>;
+  constexpr bool B_PACKED = P::B_PACKED;
   constexpr int ST = P::STAGES;
-  constexpr int WS = P::WSLOTS;
+  constexpr int WS = P::WSLOTS > 0 ? P::WSLOTS : 1;  // (int8: barriers unused)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -283,7 +312,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           uint8_t *stage = smem + s * P::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[s], P::STAGE_BYTES);
-          tma_load_2d(stage + P::OFF_ST_A, &tmA, kb * BKP, mb * BM, &full[s]);
+          tma_load_2d(stage + P::OFF_ST_A, &tmA, P::A8 ? kb * BK : kb * BKP, mb * BM, &full[s]);
           tma_load_2d(stage + P::OFF_ST_B, &tmB, B_PACKED ? kb * BKP : kb * BK, nb * P::TN, &full[s]);
           ++issued;
         }
@@ -327,6 +356,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             tc_commit(&wfree[u]);
           }
+        } else if constexpr (P::A8) {
+          // both operands straight from the TMA stage
+          for (int kb = 0; kb < num_kb; ++kb) {
+            const uint32_t s = consumed % ST, ps = (consumed / ST) & 1u;
+            if (!mbar_wait(&full[s], ps, abort_flag, &g_status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_ST_A);
+            const uint32_t b0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_ST_B);
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk)
+              mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), P::IDESC,
+                     (kb | kk) != 0 ? 1u : 0u);
+            tc_commit(&freed[s]);
+            ++consumed;
+          }
         } else {
           for (int kb = 0; kb < num_kb; ++kb) {
             const uint32_t s = consumed % ST;
@@ -355,7 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit(mma_done);
       mbar_wait_drain(mma_done, 0, &g_status);
     }
-  } else if (warp >= W_UNPACK0 && warp < W_UNPACK0 + 4) {
+  } else if (!P::A8 && warp >= W_UNPACK0 && warp < W_UNPACK0 + 4) {
     // ------------------------------------------------------------------ widen
     const int t = threadIdx.x - W_UNPACK0 * 32;
     uint32_t n = 0;
@@ -410,7 +457,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) mbar_arrive(&wready[u]);
         }
       }
-    } else {
+    } else if constexpr (P::B_PACKED) {
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         for (int kb = 0; kb < num_kb; ++kb, ++n) {
           const uint32_t s = n % ST, ps = (n / ST) & 1u;
@@ -437,7 +484,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     //   off[n] = 0x4B400000 - 8 colsum[n] (the code-offset correction folded
     //   into the exact int -> float bias), sc[n], bias[n]
     constexpr int TN = P::TN;
-    int32_t *coff = reinterpret_cast<int32_t *>(smem + P::OFF_COL) + ew * 3 * TN;
+    int32_t *coff = reinterpret_cast<int32_t *>(smem + P::OFF_COL) + ew * P::COL_WORDS;
     float *csc = reinterpret_cast<float *>(coff + TN);
     float *cbi = csc + TN;
     int it = 0;
@@ -446,7 +493,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
       __syncwarp();  // every lane is done reading the previous tile's constants
 #pragma unroll
-      for (int j = lane; j < ((!OUT_S32 && P::A_TMEM) ? 0 : TN); j += 32) {
+      for (int j = lane; j < (((!OUT_S32 && P::EPI16) || P::A8) ? 0 : TN); j += 32) {
         const int n = nb * TN + j;
         const bool in = n < N;  // the last tile of a ragged N
         coff[j] = 0x4B400000 - ((B_PACKED || !in) ? 0 : 8 * __ldg(colsum + n));
@@ -459,7 +506,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&acc_full[b], pb, abort_flag, &g_status)) break;
       tc_fence_after();
       const int row0 = mb * BM + ew * 32;
-      if constexpr (!OUT_S32 && P::A_TMEM) {
+      if constexpr (!OUT_S32 && P::EPI16) {
         // 16x256b fragments: thread t holds rows q = t/4 + 8 i (i < 4) of the
         // warp's 32 rows and, per 8-column group j, columns 8j + 2(t%4) + {0,1};
         // its columns' constants are 8-byte loads, and the bf16 pairs go to the
@@ -492,8 +539,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int2 o = make_int2(0x4B400000, 0x4B400000);
             float2 scl = make_float2(0.0f, 0.0f), bi = make_float2(0.0f, 0.0f);
             if (n < N) {
-              const int2 cs2 = __ldg(reinterpret_cast<const int2 *>(colsum + n));
-              o = make_int2(0x4B400000 - 8 * cs2.x, 0x4B400000 - 8 * cs2.y);
+              if constexpr (P::A_TMEM) {
+                const int2 cs2 = __ldg(reinterpret_cast<const int2 *>(colsum + n));
+                o = make_int2(0x4B400000 - 8 * cs2.x, 0x4B400000 - 8 * cs2.y);
+              }
               scl = __ldg(reinterpret_cast<const float2 *>(scale_ch + n));
               bi = __ldg(reinterpret_cast<const float2 *>(bias + n));
             }
@@ -501,9 +550,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int h = 0; h < 2; ++h)
 #pragma unroll
               for (int u = 0; u < 2; ++u)
-                pk[h][u][j] = dequant2_bf16(static_cast<int32_t>(r[h][4 * j + 2 * u]) + o.x,
-                                            static_cast<int32_t>(r[h][4 * j + 2 * u + 1]) + o.y,
-                                            st4[2 * h + u], scl.x, scl.y, bi.x, bi.y);
+                pk[h][u][j] =
+                    P::A8 ? dequant2_bf16_cvt(static_cast<int32_t>(r[h][4 * j + 2 * u]),
+                                              static_cast<int32_t>(r[h][4 * j + 2 * u + 1]),
+                                              st4[2 * h + u], scl.x, scl.y, bi.x, bi.y)
+                          : dequant2_bf16(static_cast<int32_t>(r[h][4 * j + 2 * u]) + o.x,
+                                          static_cast<int32_t>(r[h][4 * j + 2 * u + 1]) + o.y,
+                                          st4[2 * h + u], scl.x, scl.y, bi.x, bi.y);
           }
           uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (sc & 1)) * EPI_BYTES;
           if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
@@ -552,7 +605,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(m) * N + n0);
 #pragma unroll
             for (int c = 0; c < EPI_COLS / 4; ++c) {
-              const int4 o = off4[c];
+              const int4 o = P::A8 ? make_int4(0x4B400000, 0x4B400000, 0x4B400000, 0x4B400000) : off4[c];
               dst[c] = make_int4(static_cast<int32_t>(r[4 * c + 0]) + o.x - 0x4B400000,
                                  static_cast<int32_t>(r[4 * c + 1]) + o.y - 0x4B400000,
                                  static_cast<int32_t>(r[4 * c + 2]) + o.z - 0x4B400000,
@@ -657,10 +710,10 @@ bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool B_PACKED, bool OUT_S32>
+template <int MODE, bool OUT_S32>
 cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
-  using P = Plan<B_PACKED>;
-  auto kern = w4a4_gemm_kernel<B_PACKED, OUT_S32>;
+  using P = Plan<MODE>;
+  auto kern = w4a4_gemm_kernel<MODE, OUT_S32>;
   static bool attr_set[64] = {};  // per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -673,10 +726,13 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   }
   CUtensorMap tmA, tmB, tmY;
   const uint64_t kp = static_cast<uint64_t>(a.K / 2);
-  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qx, kp, a.M, kp, BKP, BM,
-                   P::A_TMEM ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
-  const bool okB = B_PACKED ? make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw, kp, a.N, kp,
+  const bool okA = P::A8 ? make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qx, a.K, a.M, a.K, BK,
+                                       BM, CU_TENSOR_MAP_SWIZZLE_128B)
+                         : make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qx, kp, a.M, kp, BKP,
+                                       BM, P::A_TMEM ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                     : CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!okA) return cudaErrorInvalidValue;
+  const bool okB = P::B_PACKED ? make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw, kp, a.N, kp,
                                           BKP, BN, CU_TENSOR_MAP_SWIZZLE_NONE)
                             : make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw8, a.K, a.N,
                                           a.K, BK, P::TN, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -713,9 +769,10 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
 
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st) {
   if (a.M <= 0) return cudaSuccess;
+  if (a.a8) return a.acc ? launch_t<kInt8, true>(a, st) : launch_t<kInt8, false>(a, st);
   const bool packed = (a.qw8 == nullptr);
-  if (a.acc) return packed ? launch_t<true, true>(a, st) : launch_t<false, true>(a, st);
-  return packed ? launch_t<true, false>(a, st) : launch_t<false, false>(a, st);
+  if (a.acc) return packed ? launch_t<kPacked, true>(a, st) : launch_t<kExpanded, true>(a, st);
+  return packed ? launch_t<kPacked, false>(a, st) : launch_t<kExpanded, false>(a, st);
 }
 
 cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,

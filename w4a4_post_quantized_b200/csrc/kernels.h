@@ -11,8 +11,10 @@ namespace w4a4 {
 int device_sm_count();
 
 // quant.cu
+// bits = 4: q [M, K/2] packed int4; bits = 8: q [M, K] int8
 cudaError_t launch_quantize_rows(const uint16_t *X, int64_t M, int K, const float *mult,
-                                 uint8_t *q, float *scale, bool rot, bool gelu, cudaStream_t st);
+                                 uint8_t *q, float *scale, bool rot, bool gelu, int bits,
+                                 cudaStream_t st);
 cudaError_t launch_colmax(const uint16_t *X, int64_t M, int K, float *colmax, cudaStream_t st);
 cudaError_t launch_smooth_factors(float *s_io, float *inv_io, int K, double alpha, cudaStream_t st);
 cudaError_t launch_bias_to_f32(const uint16_t *b, float *out, int n, cudaStream_t st);
@@ -20,9 +22,9 @@ cudaError_t launch_fill(float *out, int n, float v, cudaStream_t st);
 
 // gemm.cu
 struct GemmArgs {
-  const uint8_t *qx;        // [M, K/2] packed int4
+  const uint8_t *qx;        // [M, K/2] packed int4, or [M, K] int8 codes when a8
   const uint8_t *qw;        // [N, K/2] packed int4 (used when qw8 == nullptr)
-  const int8_t *qw8;        // [N, K] widened weight codes, or nullptr
+  const int8_t *qw8;        // [N, K] widened weight codes (int8 codes when a8), or nullptr
   const int32_t *colsum;    // [N] per-row code sums (with qw8)
   const float *scale_tok;   // [M]
   const float *scale_ch;    // [N]
@@ -31,6 +33,7 @@ struct GemmArgs {
   int32_t *acc;             // [M, N] int32 accumulators instead of y (test path)
   int64_t M;
   int N, K;
+  bool a8;                  // W8A8: qx and qw8 hold 8-bit codes in natural order
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,

@@ -1,7 +1,8 @@
 // quant.cu -- the HBM-bound half of the DSFQ W4A4 linear on sm_100a:
 //   * quantize_rows: bf16 row -> (optional GELU) -> Hadamard rotation (fast
 //     Walsh-Hadamard transform, fp32) -> per-channel multiplier -> per-row
-//     absmax -> symmetric int4 codes packed two per byte + fp32 step.
+//     absmax -> symmetric int4 codes packed two per byte + fp32 step (or, for
+//     the W8A8 setting, one int8 code per byte with step absmax / 127).
 //     Activations use multiplier 1/s (pre-global rotation, then post-local
 //     smoothing), weights use s; both follow page "十亿参数的三维重建模型，能塞进手机吗？",
 //     sections 预全局旋转 / 后局部平滑 / 训练后量化（PTQ） / 细粒度量化粒度.
@@ -238,8 +239,9 @@ __device__ __forceinline__ uint32_t low_bytes(uint32_t a, uint32_t b, uint32_t c
 // Per-channel multiplier (from the block's shared table), per-row absmax,
 // codes, packed store for a phase-2 row.  The transform's 1/sqrt(K) is an
 // exact power of two, so it changes neither the absmax position nor any
-// code: it is applied to the stored step only.
-template <int K, bool ROT>
+// code: it is applied to the stored step only.  BITS = 4: codes in [-7, 7]
+// packed two per byte; BITS = 8: codes in [-127, 127], one per byte.
+template <int K, bool ROT, int BITS>
 __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], int lane, int64_t row,
                                                    const float4 *__restrict__ mtab,
                                                    uint8_t *__restrict__ q, float *__restrict__ scale) {
@@ -260,19 +262,35 @@ __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], i
   float amax = fmax3(am[0], am[1], fmaxf(am[2], am[3]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (lane == 0) scale[row] = (ROT ? amax * RowShape<K>::kInvSqrtK : amax) / 7.0f;
-  if (amax < 0x1p-100f) {  // keep 7/amax finite: exact power-of-two rescale, same codes
+  static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
+  constexpr float kQmax = BITS == 4 ? 7.0f : 127.0f;
+  if (lane == 0) scale[row] = (ROT ? amax * RowShape<K>::kInvSqrtK : amax) / kQmax;
+  if (amax < 0x1p-100f) {  // keep kQmax/amax finite: exact power-of-two rescale, same codes
 #pragma unroll
     for (int r = 0; r < V; ++r) v[r] *= 0x1p+64f;
     amax *= 0x1p+64f;
   }
-  const float inv = (amax > 0.0f) ? 7.0f / amax : 0.0f;
-  // code = round-half-even(v * inv); |v * inv| <= 7 (1 + 2^-24), so no clamp
-  // can ever act.  Adding 1.5 * 2^23 in the same fused operation rounds the
-  // exact product to an integer whose low 4 bits are the two's-complement code.
+  const float inv = (amax > 0.0f) ? kQmax / amax : 0.0f;
+  // code = round-half-even(v * inv); |v * inv| <= kQmax (1 + 2^-24), so no
+  // clamp can ever act.  Adding 1.5 * 2^23 in the same fused operation rounds
+  // the exact product to an integer whose low 8 bits are the two's-complement
+  // code.
   const unsigned long long inv2 = pack2(inv, inv), magic2 = pack2(12582912.0f, 12582912.0f);
 #pragma unroll
   for (int k = 0; k < V; k += 2) fma_x2(v[k], v[k + 1], inv2, magic2);
+  if constexpr (BITS == 8) {
+    // word w: the codes of elements 4w .. 4w + 3, one byte each
+    uint32_t words[V / 4];
+#pragma unroll
+    for (int w = 0; w < V / 4; ++w)
+      words[w] = low_bytes(__float_as_uint(v[4 * w]), __float_as_uint(v[4 * w + 1]),
+                           __float_as_uint(v[4 * w + 2]), __float_as_uint(v[4 * w + 3]));
+    uint4 *dst = reinterpret_cast<uint4 *>(q + row * K + static_cast<int64_t>(lane) * V);
+#pragma unroll
+    for (int c = 0; c < V / 16; ++c)
+      dst[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+    return;
+  }
   // word w: codes of elements 8w .. 8w + 7, element 2i in the low nibble of byte i
   uint32_t words[V / 8];
 #pragma unroll
@@ -304,7 +322,7 @@ struct QuantStaging {
 // NS rows in flight: 1-D bulk copies (TMA engine) stream its next rows into a
 // private shared-memory ring while it transforms the current one, so the HBM
 // latency is hidden without occupancy.
-template <int K, bool ROT, bool GELU>
+template <int K, bool ROT, bool GELU, int BITS>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_rows_kernel(const uint16_t *__restrict__ X, int64_t M, const float *__restrict__ mult,
                          uint8_t *__restrict__ q, float *__restrict__ scale,
@@ -377,7 +395,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         ++issued;
       }
     }
-    quantize_store_row<K, ROT>(v, lane, row, mtab, q, scale);
+    quantize_store_row<K, ROT, BITS>(v, lane, row, mtab, q, scale);
   }
   // after a timed-out wait, let the copies still in flight land before exiting
   if (lane == 0)
@@ -457,10 +475,10 @@ int row_grid(Kern kern, int64_t rows) {
   return static_cast<int>(need < g ? need : g);
 }
 
-template <int K, bool ROT, bool GELU>
+template <int K, bool ROT, bool GELU, int BITS>
 cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint8_t *q,
                            float *scale, cudaStream_t st) {
-  auto kern = quantize_rows_kernel<K, ROT, GELU>;
+  auto kern = quantize_rows_kernel<K, ROT, GELU, BITS>;
   constexpr int smem = QuantStaging<K>::SMEM;
   static int per_sm_dev[64] = {};  // per device: attribute set and occupancy known
   int dev = 0;
@@ -499,19 +517,26 @@ cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint
 
 int device_sm_count() { return num_sms(); }
 
+namespace {
+template <int K, int BITS>
+cudaError_t launch_quant_kb(const uint16_t *X, int64_t M, const float *mult, uint8_t *q,
+                            float *scale, bool rot, bool gelu, cudaStream_t st) {
+  if (rot) return gelu ? launch_quant_k<K, true, true, BITS>(X, M, mult, q, scale, st)
+                       : launch_quant_k<K, true, false, BITS>(X, M, mult, q, scale, st);
+  return gelu ? launch_quant_k<K, false, true, BITS>(X, M, mult, q, scale, st)
+              : launch_quant_k<K, false, false, BITS>(X, M, mult, q, scale, st);
+}
+}  // namespace
+
 cudaError_t launch_quantize_rows(const uint16_t *X, int64_t M, int K, const float *mult,
-                                 uint8_t *q, float *scale, bool rot, bool gelu, cudaStream_t st) {
+                                 uint8_t *q, float *scale, bool rot, bool gelu, int bits,
+                                 cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  if (K == 1024) {
-    if (rot) return gelu ? launch_quant_k<1024, true, true>(X, M, mult, q, scale, st)
-                         : launch_quant_k<1024, true, false>(X, M, mult, q, scale, st);
-    return gelu ? launch_quant_k<1024, false, true>(X, M, mult, q, scale, st)
-                : launch_quant_k<1024, false, false>(X, M, mult, q, scale, st);
-  }
-  if (rot) return gelu ? launch_quant_k<4096, true, true>(X, M, mult, q, scale, st)
-                       : launch_quant_k<4096, true, false>(X, M, mult, q, scale, st);
-  return gelu ? launch_quant_k<4096, false, true>(X, M, mult, q, scale, st)
-              : launch_quant_k<4096, false, false>(X, M, mult, q, scale, st);
+  if (bits == 8)
+    return K == 1024 ? launch_quant_kb<1024, 8>(X, M, mult, q, scale, rot, gelu, st)
+                     : launch_quant_kb<4096, 8>(X, M, mult, q, scale, rot, gelu, st);
+  return K == 1024 ? launch_quant_kb<1024, 4>(X, M, mult, q, scale, rot, gelu, st)
+                   : launch_quant_kb<4096, 4>(X, M, mult, q, scale, rot, gelu, st);
 }
 
 cudaError_t launch_colmax(const uint16_t *X, int64_t M, int K, float *colmax, cudaStream_t st) {

@@ -27,6 +27,7 @@ W4A4_OK, W4A4_ERR_ARG, W4A4_ERR_SHAPE, W4A4_ERR_ALIGN, W4A4_ERR_UNSUPPORTED, W4A
 W4A4_DEV_TIMEOUT = 0x1
 W4A4_FLAG_GELU = 0x1
 W4A4_FLAG_PLAIN = 0x2
+W4A4_FLAG_INT8 = 0x4
 
 _vp, _i32, _i64, _u32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
                                     ctypes.c_float, ctypes.c_size_t)
@@ -45,6 +46,7 @@ def _sig(name, res, args):
 
 
 _workspace_bytes = _sig("w4a4_workspace_bytes", _sz, [_i64, _i32])
+_workspace_bytes_ex = _sig("w4a4_workspace_bytes_ex", _sz, [_i64, _i32, _u32])
 _prepare = _sig("w4a4_prepare_weights", ctypes.c_int,
                 [_vp, _vp, _i32, _i32, _vp, _i64, _f32, _u32, ctypes.POINTER(W4A4WeightsT), _vp])
 _quantize = _sig("w4a4_quantize_act", ctypes.c_int, [_vp, _i64, _i32, _vp, _vp, _vp, _u32, _vp])
@@ -98,27 +100,30 @@ def w4a4_workspace_bytes(M: int, K: int) -> int:
     return int(_workspace_bytes(M, K))
 
 
+def w4a4_workspace_bytes_ex(M: int, K: int, flags: int) -> int:
+    return int(_workspace_bytes_ex(M, K, flags))
+
+
 class PreparedWeights:
     """Device arrays of one prepared layer (owned by torch) and the C struct
     that points at them.  expanded=True also allocates the widened int8 copy
     of the codes (qw8, N*K bytes) and the per-row code sums the fast GEMM
-    path uses; expanded=False keeps only the packed int4 codes."""
+    path uses; expanded=False keeps only the packed int4 codes.  int8=True
+    (the W8A8 setting) allocates only qw8, which then holds the 8-bit codes."""
 
-    def __init__(self, N: int, K: int, device="cuda", expanded: bool = True):
+    def __init__(self, N: int, K: int, device="cuda", expanded: bool = True, int8: bool = False):
         self.N, self.K = N, K
         self.device = torch.device(device)
-        self.qw = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+        self.qw = None if int8 else torch.empty((N, K // 2), dtype=torch.uint8, device=device)
         self.scale_ch = torch.empty(N, dtype=torch.float32, device=device)
         self.bias = torch.empty(N, dtype=torch.float32, device=device)
         self.smooth = torch.empty(K, dtype=torch.float32, device=device)
         self.inv_smooth = torch.empty(K, dtype=torch.float32, device=device)
-        self.qw8 = torch.empty((N, K), dtype=torch.int8, device=device) if expanded else None
-        self.colsum = torch.empty(N, dtype=torch.int32, device=device) if expanded else None
-        self.struct = W4A4WeightsT(N, K, self.qw.data_ptr(), self.scale_ch.data_ptr(),
+        self.qw8 = torch.empty((N, K), dtype=torch.int8, device=device) if (expanded or int8) else None
+        self.colsum = torch.empty(N, dtype=torch.int32, device=device) if (expanded and not int8) else None
+        self.struct = W4A4WeightsT(N, K, _ptr(self.qw), self.scale_ch.data_ptr(),
                                    self.bias.data_ptr(), self.smooth.data_ptr(),
-                                   self.inv_smooth.data_ptr(),
-                                   self.qw8.data_ptr() if expanded else None,
-                                   self.colsum.data_ptr() if expanded else None, 0)
+                                   self.inv_smooth.data_ptr(), _ptr(self.qw8), _ptr(self.colsum), 0)
 
     @property
     def flags(self) -> int:
@@ -129,7 +134,7 @@ def w4a4_prepare_weights(W: torch.Tensor, bias, X_calib, alpha: float = 0.5, fla
                          out: PreparedWeights | None = None, expanded: bool = True,
                          stream=None) -> PreparedWeights:
     N, K = W.shape
-    out = out or PreparedWeights(N, K, W.device, expanded=expanded)
+    out = out or PreparedWeights(N, K, W.device, expanded=expanded, int8=bool(flags & W4A4_FLAG_INT8))
     mc = 0 if X_calib is None else X_calib.shape[0]
     _check(_prepare(_ptr(W), _ptr(bias), N, K, _ptr(X_calib), mc, alpha, flags,
                     ctypes.byref(out.struct), _stream(stream)), "w4a4_prepare_weights")
@@ -139,7 +144,8 @@ def w4a4_prepare_weights(W: torch.Tensor, bias, X_calib, alpha: float = 0.5, fla
 def w4a4_quantize_act(X: torch.Tensor, inv_smooth, flags: int = 0, qx=None, scale_tok=None,
                       stream=None):
     M, K = X.shape
-    qx = qx if qx is not None else torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    width = K if flags & W4A4_FLAG_INT8 else K // 2
+    qx = qx if qx is not None else torch.empty((M, width), dtype=torch.uint8, device=X.device)
     scale_tok = scale_tok if scale_tok is not None else torch.empty(M, dtype=torch.float32, device=X.device)
     _check(_quantize(_ptr(X), M, K, _ptr(inv_smooth), _ptr(qx), _ptr(scale_tok), flags,
                      _stream(stream)), "w4a4_quantize_act")
@@ -158,7 +164,7 @@ def w4a4_linear_fused(X: torch.Tensor, w: PreparedWeights, Y=None, workspace=Non
                       stream=None):
     M = X.shape[0]
     Y = Y if Y is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
-    need = w4a4_workspace_bytes(M, w.K)
+    need = w4a4_workspace_bytes_ex(M, w.K, flags)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
     _check(_fused(_ptr(X), M, ctypes.byref(w.struct), _ptr(Y), _ptr(workspace),
