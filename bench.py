@@ -249,11 +249,14 @@ def run_ours(args, wl, world, rank, local):
     Xs = [bf16(synth.activations(M, K, seed=seed + 10 + i)) for i in range(NSETS)]
     pw = w4a4.w4a4_prepare_weights(W, b, Xs[0][:synth.calibration_rows(M)])
     Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(NSETS)]
+    # the workspace of the fused call's fastest route: int4 codes one per byte
+    # (operand order of the expanded weights), then the steps
     wsb = w4a4.w4a4_workspace_bytes(M, K)
     WSs = [torch.empty(wsb, dtype=torch.uint8, device=dev) for _ in range(NSETS)]
-    st_off = ((M * K // 2 + 255) // 256) * 256
-    QX = [ws[:M * K // 2].view(M, K // 2) for ws in WSs]
+    st_off = ((M * K + 255) // 256) * 256
+    QX = [ws[:M * K].view(M, K) for ws in WSs]
     ST = [ws[st_off:st_off + 4 * M].view(torch.float32) for ws in WSs]
+    unp = w4a4.W4A4_FLAG_UNPACKED
     torch.cuda.synchronize()
 
     def step(i):
@@ -285,9 +288,11 @@ def run_ours(args, wl, world, rank, local):
         # the per-launch durations the rooflines use
         n_iso = max(3, min(args.steps, 500))
         iso = {}
-        for name, fn in (("quant", lambda j: w4a4.w4a4_quantize_act(Xs[j], pw.inv_smooth, flags,
+        for name, fn in (("quant", lambda j: w4a4.w4a4_quantize_act(Xs[j], pw.inv_smooth, flags | unp,
                                                                      qx=QX[j], scale_tok=ST[j])),
-                         ("gemm", lambda j: w4a4.w4a4_linear(QX[j], ST[j], pw, Y=Ys[j]))):
+                         ("gemm", lambda j: w4a4.w4a4_linear_ex(QX[j], ST[j], pw, flags=unp, Y=Ys[j]))):
+            for i in range(3):  # warm-up launches of this kernel alone
+                fn(i % NSETS)
             k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             k0.record(stream)
             for i in range(n_iso):
@@ -303,9 +308,9 @@ def run_ours(args, wl, world, rank, local):
             j = i % NSETS
             e0, e1, e2 = evq[i]
             e0.record(stream)
-            w4a4.w4a4_quantize_act(Xs[j], pw.inv_smooth, flags, qx=QX[j], scale_tok=ST[j])
+            w4a4.w4a4_quantize_act(Xs[j], pw.inv_smooth, flags | unp, qx=QX[j], scale_tok=ST[j])
             e1.record(stream)
-            w4a4.w4a4_linear(QX[j], ST[j], pw, Y=Ys[j])
+            w4a4.w4a4_linear_ex(QX[j], ST[j], pw, flags=unp, Y=Ys[j])
             e2.record(stream)
         torch.cuda.synchronize()
     status = w4a4.w4a4_get_device_status()
@@ -386,6 +391,70 @@ def run_ours(args, wl, world, rank, local):
                      "overhead_pct": 100.0 * (m7["dsfq"] - m7["plain"]) / m7["plain"],
                      "steps": n7, "pages_figure_pct": 0.2,
                      "sqnr_db": sq, "sqnr_rows": rows}
+    # ------------------------------------------------------- W8A8 (8-bit codes)
+    # the setting the pages report beside W4A4, on the same inputs: 8-bit
+    # codes need no widening in the GEMM, so the isolated GEMM times of the
+    # two settings bracket what the 4-bit codes cost there (the 8-bit GEMM
+    # also reads twice the activation bytes and uses 128 x 256 tiles)
+    i8 = w4a4.W4A4_FLAG_INT8
+    pw8 = w4a4.w4a4_prepare_weights(W, b, Xs[0][:synth.calibration_rows(M)], flags=i8)
+    fl8 = flags | i8
+    t8 = {}
+    for name, fn in (("step", lambda j: w4a4.w4a4_linear_fused(Xs[j], pw8, Y=Ys[j], workspace=WSs[j], flags=fl8)),
+                     ("quant", lambda j: w4a4.w4a4_quantize_act(Xs[j], pw8.inv_smooth, fl8, qx=QX[j],
+                                                                 scale_tok=ST[j])),
+                     ("gemm", lambda j: w4a4.w4a4_linear(QX[j], ST[j], pw8, Y=Ys[j]))):
+        for i in range(3):
+            fn(i % NSETS)
+        barrier(world)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for i in range(n7):
+            fn(i % NSETS)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        t8[name] = max_over_ranks(world, b0.elapsed_time(b1)) / n7 * 1e3
+    y8 = w4a4.w4a4_linear_fused(Xs[0][:rows], pw8, flags=fl8).double()
+    sq8 = float(10.0 * torch.log10((ref ** 2).sum() / ((y8 - ref) ** 2).sum()))
+    torch.cuda.synchronize()
+    w8a8 = {"us_per_step": t8["step"], "tops": ops / (t8["step"] * 1e-6) / 1e12,
+            "quantize_us": t8["quant"], "gemm_us": t8["gemm"],
+            "gemm_tops": ops / (t8["gemm"] * 1e-6) / 1e12,
+            "quantize_gbs": (2.0 * M * K + M * K + 4.0 * M) / (t8["quant"] * 1e-6) / 1e9,
+            "w4a4_gemm_us": g_ms * 1e3, "w4a4_quantize_us": q_ms * 1e3,
+            "sqnr_db": sq8, "sqnr_db_w4a4": sq["dsfq"], "sqnr_rows": rows,
+            "timing": f"CUDA events around {n7} back-to-back launches each (step = w4a4_linear_fused)"}
+    # ------------------------------------- the packed route (codes two per byte)
+    # the fused call with the smallest workspace it accepts: packed int4 codes,
+    # which the GEMM widens on every tile (once per output tile); the one-per-
+    # byte route above is what the fused call takes with the full workspace
+    wsp = w4a4.w4a4_workspace_bytes_min(M, K, flags)
+    QP = [ws[:M * K // 2].view(M, K // 2) for ws in WSs]
+    STP = [ws[((M * K // 2 + 255) // 256) * 256:][:4 * M].view(torch.float32) for ws in WSs]
+    tp = {}
+    for name, fn in (("step", lambda j: w4a4.w4a4_linear_fused(Xs[j], pw, Y=Ys[j], workspace=WSs[j][:wsp],
+                                                                 flags=flags)),
+                     ("quant", lambda j: w4a4.w4a4_quantize_act(Xs[j], pw.inv_smooth, flags, qx=QP[j],
+                                                                 scale_tok=STP[j])),
+                     ("gemm", lambda j: w4a4.w4a4_linear(QP[j], STP[j], pw, Y=Ys[j]))):
+        for i in range(3):
+            fn(i % NSETS)
+        barrier(world)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for i in range(n7):
+            fn(i % NSETS)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        tp[name] = max_over_ranks(world, b0.elapsed_time(b1)) / n7 * 1e3
+    packed_route = {"us_per_step": tp["step"], "tops": ops / (tp["step"] * 1e-6) / 1e12,
+                    "quantize_us": tp["quant"], "gemm_us": tp["gemm"],
+                    "gemm_tops": ops / (tp["gemm"] * 1e-6) / 1e12,
+                    "workspace_bytes": wsp, "workspace_bytes_fast_route": wsb,
+                    "what": "w4a4_linear_fused with its minimum workspace: int4 codes two per byte, "
+                            "widened by the GEMM on every tile"}
     weight_bytes = {"packed_int4": N * K // 2 + 12 * N + 4 * K, "bf16": 2 * N * K + 2 * N,
                     "expanded_int8_copy": N * K + 4 * N,
                     "ratio_bf16_over_packed": (2 * N * K + 2 * N) / (N * K // 2 + 12 * N + 4 * K)}
@@ -427,6 +496,8 @@ def run_ours(args, wl, world, rank, local):
         "roofline": roofline,
         "roofline_quantize": roofline_q,
         "dsfq_overhead": dsfq_overhead,
+        "w8a8": w8a8,
+        "packed_route": packed_route,
         "weight_bytes": weight_bytes,
         "device_status": status,
     }

@@ -90,6 +90,15 @@ typedef enum {
                                  in natural order, for activations and weights;
                                  must match between prepare_weights and the
                                  activation calls */
+#define W4A4_FLAG_UNPACKED 0x8u  /* quantize_act / linear_ex: the int4 codes one per
+                                 byte (int8 values in [-7, 7]) instead of two per
+                                 byte, in the operand order of w4a4_expand_weights
+                                 (within every 8 elements: 0, 2, 4, 6, 1, 3, 5, 7).
+                                 Not on the pages: the tensor cores multiply 8-bit
+                                 operands, and codes that arrive one per byte need
+                                 no widening in the GEMM (which otherwise widens
+                                 every activation tile once per output tile).
+                                 Not with W4A4_FLAG_INT8. */
 
 /* Prepared weights of one linear layer.  The caller allocates every array
  * (device memory) with the sizes given and keeps ownership. */
@@ -113,15 +122,17 @@ typedef struct {
                              8-bit codes */
 } w4a4_weights_t;
 
-/* Bytes of workspace w4a4_linear_fused needs for M tokens of width K:
- * the packed activation codes (M*K/2, rounded up to 256) followed by the
- * per-token steps (4*M).  Returns 0 for an unsupported K. */
+/* Bytes of workspace that let w4a4_linear_fused take its fastest route for M
+ * tokens of width K, whatever the weights and flags: activation codes one per
+ * byte (M*K, rounded up to 256) followed by the per-token steps (4*M).
+ * Returns 0 for an unsupported K. */
 size_t w4a4_workspace_bytes(int64_t M, int32_t K);
 
-/* The same for the given flags: with W4A4_FLAG_INT8 the codes take M*K bytes
- * (rounded up to 256), followed by the 4*M bytes of steps.  Returns 0 for an
+/* The least workspace w4a4_linear_fused accepts for these flags: codes two per
+ * byte (M*K/2 rounded up to 256, + 4*M) for 4-bit weights, one per byte
+ * (M*K ...) with W4A4_FLAG_INT8 or W4A4_FLAG_UNPACKED.  Returns 0 for an
  * unsupported K or an unknown flag. */
-size_t w4a4_workspace_bytes_ex(int64_t M, int32_t K, uint32_t flags);
+size_t w4a4_workspace_bytes_min(int64_t M, int32_t K, uint32_t flags);
 
 /* Offline weight preparation [ROT][SMOOTH][PTQ][GRAN].
  *   W       [N, K] bf16 weights; bias [N] bf16 or NULL;
@@ -154,7 +165,8 @@ w4a4_status w4a4_expand_weights(w4a4_weights_t *w, void *stream);
  * scale_tok [M] (fp32), codes round-half-even(x / delta) packed into qx
  * [M, K/2].  With W4A4_FLAG_PLAIN the rotation and smoothing are skipped
  * (inv_smooth may then be NULL).  With W4A4_FLAG_INT8, delta = absmax/127 and
- * qx [M, K] holds one int8 code per element.  Inputs must be finite. */
+ * qx [M, K] holds one int8 code per element; with W4A4_FLAG_UNPACKED, qx [M, K]
+ * holds the int4 codes one per byte in operand order.  Inputs must be finite. */
 w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const float *inv_smooth,
                               uint8_t *qx, float *scale_tok, uint32_t flags, void *stream);
 
@@ -166,12 +178,25 @@ w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const flo
 w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
                         const w4a4_weights_t *w, uint16_t *Y, void *stream);
 
+/* w4a4_linear with the code layout of qx given by flags: 0 (as w4a4_linear)
+ * or W4A4_FLAG_UNPACKED for 4-bit weights that carry qw8 (then qx [M, K] holds
+ * the int4 codes one per byte in operand order, as w4a4_quantize_act writes
+ * them with that flag; W4A4_ERR_ARG without qw8).  Other flags:
+ * W4A4_ERR_UNSUPPORTED. */
+w4a4_status w4a4_linear_ex(const uint8_t *qx, const float *scale_tok, int64_t M,
+                           const w4a4_weights_t *w, uint16_t *Y, uint32_t flags, void *stream);
+
 /* Quantized linear from bf16 activations: w4a4_quantize_act (with
- * w->inv_smooth and the given flags) into `workspace`, then w4a4_linear.
- * workspace must hold w4a4_workspace_bytes_ex(M, w->K, flags) bytes
- * (workspace_bytes says how many it holds); its contents afterwards are the
- * codes and steps.  flags must carry the same W4A4_FLAG_PLAIN and
- * W4A4_FLAG_INT8 bits as w->flags (W4A4_ERR_ARG otherwise). */
+ * w->inv_smooth and the given flags) into `workspace`, then w4a4_linear_ex.
+ * workspace_bytes says how many bytes workspace holds: at least
+ * w4a4_workspace_bytes_min(M, w->K, flags) (W4A4_ERR_SHAPE otherwise).  For
+ * 4-bit weights with qw8 and a workspace of w4a4_workspace_bytes(M, w->K)
+ * bytes the codes go one per byte (W4A4_FLAG_UNPACKED layout) and the GEMM
+ * reads them without widening; otherwise they are packed two per byte.  The
+ * workspace afterwards holds those codes, then (at the next 256-byte boundary)
+ * the steps.  flags must carry the same W4A4_FLAG_PLAIN and W4A4_FLAG_INT8
+ * bits as w->flags (W4A4_ERR_ARG otherwise); W4A4_FLAG_UNPACKED is not a flag
+ * of this call (W4A4_ERR_UNSUPPORTED). */
 w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t *w, uint16_t *Y,
                               void *workspace, size_t workspace_bytes, uint32_t flags,
                               void *stream);
@@ -189,10 +214,11 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
  * w4a4_linear_fused without the workspace: the codes and steps go to a scratch
  * array of W4A4_NOALLOC_SCRATCH_BYTES inside the library instead, so the call
  * allocates nothing.
- *   - Accepts M with w4a4_workspace_bytes_ex(M, w->K, flags) <=
+ *   - Accepts M with w4a4_workspace_bytes_min(M, w->K, flags) <=
  *     W4A4_NOALLOC_SCRATCH_BYTES (4-bit codes: M <= 16256 tokens at K = 1024,
  *     M <= 4088 at K = 4096; 8-bit codes: about half of that); larger M
- *     returns W4A4_ERR_SHAPE.
+ *     returns W4A4_ERR_SHAPE.  Up to about half those sizes the codes go one
+ *     per byte (the faster route of w4a4_linear_fused).
  *   - The first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
@@ -232,8 +258,8 @@ w4a4_status w4a4_host_pipe_destroy(w4a4_host_pipe_t *pipe);
 
 /* Device workspace for w4a4_linear_fused_host: W4A4_PIPE_DEPTH slots, each
  * holding one chunk's X (2 chunk_rows K bytes), Y (2 chunk_rows N bytes),
- * codes and steps (w4a4_workspace_bytes_ex(chunk_rows, K, W4A4_FLAG_INT8),
- * room for either code width), each part 256-byte aligned. */
+ * codes and steps (w4a4_workspace_bytes(chunk_rows, K)), each part 256-byte
+ * aligned. */
 size_t w4a4_host_workspace_bytes(int64_t chunk_rows, int32_t K, int32_t N);
 
 /* Y_host [M, N] bf16 = w4a4_linear_fused(X_host [M, K] bf16) with X_host and

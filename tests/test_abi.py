@@ -59,8 +59,9 @@ def _setup(lib):
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
     lib.w4a4_workspace_bytes.restype = ctypes.c_size_t
     lib.w4a4_workspace_bytes.argtypes = [i64, i32]
-    lib.w4a4_workspace_bytes_ex.restype = ctypes.c_size_t
-    lib.w4a4_workspace_bytes_ex.argtypes = [i64, i32, ctypes.c_uint32]
+    lib.w4a4_workspace_bytes_min.restype = ctypes.c_size_t
+    lib.w4a4_workspace_bytes_min.argtypes = [i64, i32, ctypes.c_uint32]
+    lib.w4a4_linear_ex.argtypes = [vp, vp, i64, ctypes.POINTER(WeightsT), vp, ctypes.c_uint32, vp]
     lib.w4a4_quantize_act.argtypes = [vp, i64, i32, vp, vp, vp, ctypes.c_uint32, vp]
     lib.w4a4_linear.argtypes = [vp, vp, i64, ctypes.POINTER(WeightsT), vp, vp]
     lib.w4a4_linear_fused.argtypes = [vp, i64, ctypes.POINTER(WeightsT), vp, vp, ctypes.c_size_t,
@@ -80,17 +81,19 @@ def _weights(N=1024, K=1024, base=A, flags=0, expanded=True):
 
 def test_workspace_bytes(lib):
     _setup(lib)
-    assert lib.w4a4_workspace_bytes(10992, 1024) == ((10992 * 512 + 255) // 256) * 256 + 4 * 10992
-    assert lib.w4a4_workspace_bytes(3, 4096) == 6144 + 12
+    # the fast route's size: one code byte per element, then the steps
+    assert lib.w4a4_workspace_bytes(10992, 1024) == 10992 * 1024 + 4 * 10992
+    assert lib.w4a4_workspace_bytes(3, 4096) == 12288 + 12
     assert lib.w4a4_workspace_bytes(0, 1024) == 0
     assert lib.w4a4_workspace_bytes(10, 1000) == 0
     assert lib.w4a4_workspace_bytes(-1, 1024) == 0
-    ex = lib.w4a4_workspace_bytes_ex
+    mn = lib.w4a4_workspace_bytes_min
+    # packed int4 codes: two per byte, rounded up to 256, then the steps
+    assert mn(10992, 1024, 0) == ((10992 * 512 + 255) // 256) * 256 + 4 * 10992
+    assert mn(3, 4096, 0) == mn(3, 4096, 1) == mn(3, 4096, 2) == 6144 + 12
     for M, K in [(10992, 1024), (3, 4096), (0, 1024)]:
-        assert ex(M, K, 0) == lib.w4a4_workspace_bytes(M, K) == ex(M, K, 2) == ex(M, K, 1)
-    assert ex(10992, 1024, 4) == 10992 * 1024 + 4 * 10992          # 8-bit codes: one byte each
-    assert ex(3, 4096, 4 | 2) == 12288 + 12
-    assert ex(10, 1024, 0x80) == 0 and ex(10, 1000, 4) == 0
+        assert mn(M, K, 4) == mn(M, K, 8) == mn(M, K, 4 | 2) == lib.w4a4_workspace_bytes(M, K)
+    assert mn(10, 1024, 0x80) == 0 and mn(10, 1000, 4) == 0
 
 
 INT8 = 0x4
@@ -116,8 +119,8 @@ def test_int8_variant_argument_checks(lib):
     assert L(A, A, 10, ctypes.byref(no_codes), A, None) == 1
     assert G(A, 0, ctypes.byref(w8), A, None) == 0
     assert G(A, 10, ctypes.byref(no_codes), A, None) == 1
-    need4 = lib.w4a4_workspace_bytes(100, 1024)
-    need8 = lib.w4a4_workspace_bytes_ex(100, 1024, INT8)
+    need4 = lib.w4a4_workspace_bytes_min(100, 1024, 0)
+    need8 = lib.w4a4_workspace_bytes_min(100, 1024, INT8)
     assert F(A, 100, ctypes.byref(w8), A, A, need8, 0, None) == 1       # flag missing on the call
     assert F(A, 100, ctypes.byref(_weights()), A, A, need8, INT8, None) == 1  # 4-bit weights
     assert F(A, 100, ctypes.byref(w8), A, A, need4, INT8, None) == 2    # 4-bit-sized workspace
@@ -127,6 +130,28 @@ def test_int8_variant_argument_checks(lib):
     q = lib.w4a4_quantize_act
     assert q(A, 0, 1024, A, A, A, INT8, None) == 0
     assert q(A, 10, 1024, None, A, A, INT8, None) == 1                   # DSFQ needs inv_smooth
+
+
+UNPACKED = 0x8
+
+
+def test_unpacked_codes_argument_checks(lib):
+    """W4A4_FLAG_UNPACKED: int4 codes one per byte for quantize_act and
+    linear_ex; needs 4-bit weights with their expanded copy; not a flag of
+    the fused call (which picks its route from the workspace size)."""
+    _setup(lib)
+    q, LX, F = lib.w4a4_quantize_act, lib.w4a4_linear_ex, lib.w4a4_linear_fused
+    assert q(A, 0, 1024, A, A, A, UNPACKED, None) == 0
+    assert q(A, 10, 1024, A, A, A, UNPACKED | INT8, None) == 4
+    w = _weights()
+    assert LX(A, A, 0, ctypes.byref(w), A, UNPACKED, None) == 0
+    assert LX(A, A, 0, ctypes.byref(w), A, 0, None) == 0
+    assert LX(A, A, 10, ctypes.byref(w), A, 0x1, None) == 4                      # GELU: not a GEMM flag
+    assert LX(A, A, 10, ctypes.byref(_weights(expanded=False)), A, UNPACKED, None) == 1  # no qw8
+    assert LX(A, A, 10, ctypes.byref(_weights8()), A, UNPACKED, None) == 1       # 8-bit weights
+    full = lib.w4a4_workspace_bytes(100, 1024)
+    assert F(A, 100, ctypes.byref(w), A, A, full, UNPACKED, None) == 4
+    assert F(A, 100, ctypes.byref(w), A, A, lib.w4a4_workspace_bytes_min(100, 1024, 0) - 1, 0, None) == 2
 
 
 def test_quantize_act_argument_checks(lib):
@@ -161,7 +186,7 @@ def test_linear_fused_argument_checks(lib):
     _setup(lib)
     w = _weights()
     F = lib.w4a4_linear_fused
-    need = lib.w4a4_workspace_bytes(100, 1024)
+    need = lib.w4a4_workspace_bytes_min(100, 1024, 0)
     assert F(A, 100, ctypes.byref(w), A, A, need - 1, 0, None) == 2     # workspace too small
     assert F(A, 100, ctypes.byref(w), A, A, need, 2, None) == 1         # plain flag vs DSFQ weights
     assert F(A, 100, ctypes.byref(w), A, None, need, 0, None) == 1
@@ -212,12 +237,12 @@ def test_host_pipeline_argument_checks(lib):
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     lib.w4a4_host_workspace_bytes.restype = sz
     lib.w4a4_host_workspace_bytes.argtypes = [i64, i32, i32]
-    lib.w4a4_workspace_bytes_ex.restype = sz
-    lib.w4a4_workspace_bytes_ex.argtypes = [i64, i32, ctypes.c_uint32]
+    lib.w4a4_workspace_bytes.restype = sz
+    lib.w4a4_workspace_bytes.argtypes = [i64, i32]
     r256 = lambda b: (b + 255) // 256 * 256
     for rows, K, N in [(2816, 1024, 3072), (1, 4096, 1024), (300, 1024, 256)]:
-        # the codes part has room for 8-bit codes (either code width fits)
-        slot = r256(2 * rows * K) + r256(2 * rows * N) + r256(lib.w4a4_workspace_bytes_ex(rows, K, 4))
+        # the codes part has room for one code byte per element (every route fits)
+        slot = r256(2 * rows * K) + r256(2 * rows * N) + r256(lib.w4a4_workspace_bytes(rows, K))
         assert lib.w4a4_host_workspace_bytes(rows, K, N) == 2 * slot
     assert lib.w4a4_host_workspace_bytes(0, 1024, 256) == 0
     f = lib.w4a4_linear_fused_host

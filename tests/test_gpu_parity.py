@@ -264,3 +264,46 @@ def test_empty_input_is_a_no_op(w4):
 def test_device_status_clear(w4):
     w4.w4a4_clear_device_status()
     assert w4.w4a4_get_device_status() == 0
+
+
+# ------------------------------------------------- int4 codes one per byte (fused route)
+UNPACKED = 0x8
+OPERAND_ORDER = np.array([0, 2, 4, 6, 1, 3, 5, 7])
+
+
+@pytest.mark.parametrize("M,K,gelu", [(1, 1024, False), (1374, 1024, False), (257, 4096, True)])
+def test_unpacked_codes_equal_packed_codes(w4, M, K, gelu):
+    """The quantize kernel's one-per-byte output holds exactly the packed
+    codes, in the operand order of the expanded weights, with the same steps."""
+    X = synth.activations(M, K, seed=600 + M)
+    inv_s = synth.random_scales(K, seed=K + 3, lo=0.25, hi=4.0)
+    fl = w4.W4A4_FLAG_GELU if gelu else 0
+    qp, sp = w4.w4a4_quantize_act(bf16_dev(X), dev(inv_s), fl)
+    qu, su = w4.w4a4_quantize_act(bf16_dev(X), dev(inv_s), fl | UNPACKED)
+    assert tuple(qu.shape) == (M, K)
+    codes = oracle.unpack_int4(host(qp), K)
+    want = codes.reshape(M, K // 8, 8)[:, :, OPERAND_ORDER].reshape(M, K)
+    assert np.array_equal(host(qu).view(np.int8), want)
+    assert np.array_equal(host(sp), host(su))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (1374, 3072, 1024), (300, 1024, 4096)])
+def test_unpacked_route_matches_packed_route(w4, M, N, K):
+    """Same codes through both GEMM routes (widened per tile vs read one per
+    byte): identical accumulators, so identical bf16 outputs; and the fused
+    call gives the same output with the full and the minimum workspace."""
+    X = synth.activations(M, K, seed=700 + M)
+    W, b = synth.weights(N, K, seed=701), synth.bias(N, seed=702)
+    pw = w4.w4a4_prepare_weights(bf16_dev(W), bf16_dev(b), bf16_dev(X[:synth.calibration_rows(M)]))
+    qp, sp = w4.w4a4_quantize_act(bf16_dev(X), pw.inv_smooth, 0)
+    qu, su = w4.w4a4_quantize_act(bf16_dev(X), pw.inv_smooth, UNPACKED)
+    Yp = w4.w4a4_linear(qp, sp, pw)
+    Yu = w4.w4a4_linear_ex(qu, su, pw, flags=UNPACKED)
+    assert torch.equal(Yp.view(torch.int16), Yu.view(torch.int16))
+    Xd = bf16_dev(X)
+    small = torch.empty(w4.w4a4_workspace_bytes_min(M, K, 0), dtype=torch.uint8, device="cuda")
+    Yf_small = w4.w4a4_linear_fused(Xd, pw, workspace=small)
+    Yf_full = w4.w4a4_linear_fused(Xd, pw)
+    assert torch.equal(Yf_small.view(torch.int16), Yp.view(torch.int16))
+    assert torch.equal(Yf_full.view(torch.int16), Yp.view(torch.int16))
+    assert w4.w4a4_get_device_status() == 0

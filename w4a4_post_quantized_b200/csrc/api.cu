@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr uint32_t kKnownFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8;
+constexpr uint32_t kKnownFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED;
 constexpr uint32_t kWeightFlags = W4A4_FLAG_PLAIN | W4A4_FLAG_INT8;  // fixed at preparation
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -43,11 +43,17 @@ w4a4_status check_weights(const w4a4_weights_t *w) {
   return W4A4_OK;
 }
 
+// one code per byte (int8 codes, or int4 codes in operand order) or two
+bool one_per_byte(uint32_t flags) { return (flags & (W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED)) != 0; }
+
 // code bytes of M rows of width K
 size_t code_bytes(int64_t M, int32_t K, uint32_t flags) {
-  return static_cast<size_t>(M) * ((flags & W4A4_FLAG_INT8) ? K : K / 2);
+  return static_cast<size_t>(M) * (one_per_byte(flags) ? K : K / 2);
 }
-int code_bits(uint32_t flags) { return (flags & W4A4_FLAG_INT8) ? 8 : 4; }
+w4a4::CodeFormat code_format(uint32_t flags) {
+  if (flags & W4A4_FLAG_INT8) return w4a4::kCodeBytes8;
+  return (flags & W4A4_FLAG_UNPACKED) ? w4a4::kCodeBytes4 : w4a4::kCodePacked4;
+}
 
 w4a4_status check_act(const void *X, int64_t M, int32_t K, const float *inv_smooth, const void *qx,
                       const float *scale_tok, uint32_t flags) {
@@ -67,12 +73,14 @@ w4a4_status check_act(const void *X, int64_t M, int32_t K, const float *inv_smoo
 
 extern "C" {
 
-size_t w4a4_workspace_bytes_ex(int64_t M, int32_t K, uint32_t flags) {
+size_t w4a4_workspace_bytes_min(int64_t M, int32_t K, uint32_t flags) {
   if (!k_ok(K) || !m_ok(M) || (flags & ~kKnownFlags)) return 0;
   return round256(code_bytes(M, K, flags)) + sizeof(float) * static_cast<size_t>(M);
 }
 
-size_t w4a4_workspace_bytes(int64_t M, int32_t K) { return w4a4_workspace_bytes_ex(M, K, 0); }
+size_t w4a4_workspace_bytes(int64_t M, int32_t K) {
+  return w4a4_workspace_bytes_min(M, K, W4A4_FLAG_UNPACKED);
+}
 
 w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_t N, int32_t K,
                                  const uint16_t *X_calib, int64_t M_calib, float alpha,
@@ -102,11 +110,11 @@ w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_
   cudaError_t e;
   // 4-bit codes packed into qw, or 8-bit codes into qw8 (natural order)
   uint8_t *codes = int8 ? reinterpret_cast<uint8_t *>(out->qw8) : out->qw;
-  const int bits = code_bits(flags);
+  const w4a4::CodeFormat fmt = int8 ? w4a4::kCodeBytes8 : w4a4::kCodePacked4;
   if (plain) {
     if ((e = w4a4::launch_fill(out->smooth, K, 1.0f, st)) != cudaSuccess) return cuda_status(e);
     if ((e = w4a4::launch_fill(out->inv_smooth, K, 1.0f, st)) != cudaSuccess) return cuda_status(e);
-    e = w4a4::launch_quantize_rows(W, N, K, nullptr, codes, out->scale_ch, false, false, bits, st);
+    e = w4a4::launch_quantize_rows(W, N, K, nullptr, codes, out->scale_ch, false, false, fmt, st);
   } else {
     // column maxima of the rotated calibration activations -> out->smooth,
     // of the rotated weights -> out->inv_smooth; then s and 1/s in place
@@ -115,7 +123,7 @@ w4a4_status w4a4_prepare_weights(const uint16_t *W, const uint16_t *bias, int32_
     if ((e = w4a4::launch_colmax(W, N, K, out->inv_smooth, st)) != cudaSuccess) return cuda_status(e);
     if ((e = w4a4::launch_smooth_factors(out->smooth, out->inv_smooth, K, alpha, st)) != cudaSuccess)
       return cuda_status(e);
-    e = w4a4::launch_quantize_rows(W, N, K, out->smooth, codes, out->scale_ch, true, false, bits, st);
+    e = w4a4::launch_quantize_rows(W, N, K, out->smooth, codes, out->scale_ch, true, false, fmt, st);
   }
   if (e != cudaSuccess) return cuda_status(e);
   if ((e = w4a4::launch_bias_to_f32(bias, out->bias, N, st)) != cudaSuccess) return cuda_status(e);
@@ -137,25 +145,34 @@ w4a4_status w4a4_expand_weights(w4a4_weights_t *w, void *stream) {
 
 w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const float *inv_smooth,
                               uint8_t *qx, float *scale_tok, uint32_t flags, void *stream) {
+  if ((flags & W4A4_FLAG_INT8) && (flags & W4A4_FLAG_UNPACKED)) return W4A4_ERR_UNSUPPORTED;
   w4a4_status s = check_act(X, M, K, inv_smooth, qx, scale_tok, flags);
   if (s != W4A4_OK) return s;
   return cuda_status(w4a4::launch_quantize_rows(X, M, K, inv_smooth, qx, scale_tok,
                                                 !(flags & W4A4_FLAG_PLAIN),
-                                                (flags & W4A4_FLAG_GELU) != 0, code_bits(flags),
+                                                (flags & W4A4_FLAG_GELU) != 0, code_format(flags),
                                                 as_stream(stream)));
 }
 
-w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
-                        const w4a4_weights_t *w, uint16_t *Y, void *stream) {
+w4a4_status w4a4_linear_ex(const uint8_t *qx, const float *scale_tok, int64_t M,
+                           const w4a4_weights_t *w, uint16_t *Y, uint32_t flags, void *stream) {
   w4a4_status s = check_weights(w);
   if (s != W4A4_OK) return s;
+  if (flags & ~W4A4_FLAG_UNPACKED) return W4A4_ERR_UNSUPPORTED;
+  // one-per-byte 4-bit codes pair with the expanded weight codes
+  if ((flags & W4A4_FLAG_UNPACKED) && (int8_weights(w) || !w->qw8)) return W4A4_ERR_ARG;
   if (!m_ok(M)) return W4A4_ERR_SHAPE;
   if (M == 0) return W4A4_OK;
   if (!qx || !scale_tok || !Y) return W4A4_ERR_ARG;
   if (!aligned16(qx) || !aligned16(scale_tok) || !aligned16(Y)) return W4A4_ERR_ALIGN;
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, scale_tok, w->scale_ch, w->bias, Y, nullptr,
-                   M, w->N, w->K, int8_weights(w)};
+                   M, w->N, w->K, int8_weights(w) || (flags & W4A4_FLAG_UNPACKED) != 0};
   return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
+}
+
+w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
+                        const w4a4_weights_t *w, uint16_t *Y, void *stream) {
+  return w4a4_linear_ex(qx, scale_tok, M, w, Y, 0, stream);
 }
 
 w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t *w, uint16_t *Y,
@@ -164,21 +181,29 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
   w4a4_status s = check_weights(w);
   if (s != W4A4_OK) return s;
   if (flags & ~kKnownFlags) return W4A4_ERR_UNSUPPORTED;
+  if (flags & W4A4_FLAG_UNPACKED) return W4A4_ERR_UNSUPPORTED;  // the call picks the route
   if ((flags ^ w->flags) & kWeightFlags) return W4A4_ERR_ARG;
   if (!m_ok(M)) return W4A4_ERR_SHAPE;
   if (M == 0) return W4A4_OK;  // empty input: nothing to read or write
   if (!X || !Y || !workspace) return W4A4_ERR_ARG;
-  if (workspace_bytes < w4a4_workspace_bytes_ex(M, w->K, flags)) return W4A4_ERR_SHAPE;
+  if (workspace_bytes < w4a4_workspace_bytes_min(M, w->K, flags)) return W4A4_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(Y) || !aligned16(workspace)) return W4A4_ERR_ALIGN;
+  // 4-bit codes go one per byte (in the operand order of the expanded weights)
+  // when the weights carry that expansion and the workspace has the room: the
+  // GEMM then reads them without widening each tile again; else packed.
+  uint32_t cf = flags;
+  if (!int8_weights(w) && w->qw8 &&
+      workspace_bytes >= w4a4_workspace_bytes_min(M, w->K, flags | W4A4_FLAG_UNPACKED))
+    cf |= W4A4_FLAG_UNPACKED;
   uint8_t *qx = static_cast<uint8_t *>(workspace);
-  float *st = reinterpret_cast<float *>(qx + round256(code_bytes(M, w->K, flags)));
+  float *st = reinterpret_cast<float *>(qx + round256(code_bytes(M, w->K, cf)));
   cudaStream_t cs = as_stream(stream);
   cudaError_t e = w4a4::launch_quantize_rows(X, M, w->K, w->inv_smooth, qx, st,
                                              !(flags & W4A4_FLAG_PLAIN),
-                                             (flags & W4A4_FLAG_GELU) != 0, code_bits(flags), cs);
+                                             (flags & W4A4_FLAG_GELU) != 0, code_format(cf), cs);
   if (e != cudaSuccess) return cuda_status(e);
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, st, w->scale_ch, w->bias, Y, nullptr,
-                   M, w->N, w->K, int8_weights(w)};
+                   M, w->N, w->K, one_per_byte(cf)};
   return cuda_status(w4a4::launch_gemm(a, cs));
 }
 

@@ -34,7 +34,7 @@ struct Slot {
 Slot slot_of(void *workspace, int64_t chunk_rows, int32_t K, int32_t N, int i) {
   const size_t xb = round256(static_cast<size_t>(chunk_rows) * K * 2);
   const size_t yb = round256(static_cast<size_t>(chunk_rows) * N * 2);
-  const size_t wb = round256(w4a4_workspace_bytes_ex(chunk_rows, K, W4A4_FLAG_INT8));
+  const size_t wb = round256(w4a4_workspace_bytes(chunk_rows, K));
   uint8_t *base = static_cast<uint8_t *>(workspace) + static_cast<size_t>(i) * (xb + yb + wb);
   return Slot{reinterpret_cast<uint16_t *>(base), reinterpret_cast<uint16_t *>(base + xb),
               base + xb + yb, wb};
@@ -81,7 +81,7 @@ extern "C" size_t w4a4_host_workspace_bytes(int64_t chunk_rows, int32_t K, int32
   if (chunk_rows <= 0 || K <= 0 || N <= 0) return 0;
   const size_t xb = round256(static_cast<size_t>(chunk_rows) * K * 2);
   const size_t yb = round256(static_cast<size_t>(chunk_rows) * N * 2);
-  const size_t wb = round256(w4a4_workspace_bytes_ex(chunk_rows, K, W4A4_FLAG_INT8));
+  const size_t wb = round256(w4a4_workspace_bytes(chunk_rows, K));
   return W4A4_PIPE_DEPTH * (xb + yb + wb);
 }
 

@@ -11,9 +11,14 @@ namespace w4a4 {
 int device_sm_count();
 
 // quant.cu
-// bits = 4: q [M, K/2] packed int4; bits = 8: q [M, K] int8
+// Code formats of the quantize kernel:
+//   kCodePacked4  int4 codes, two per byte (q [M, K/2])
+//   kCodeBytes4   int4 codes, one per byte in the tensor-core operand order
+//                 (within every 8 elements: 0, 2, 4, 6, 1, 3, 5, 7) (q [M, K])
+//   kCodeBytes8   int8 codes (step absmax / 127), natural order (q [M, K])
+enum CodeFormat : int { kCodePacked4 = 0, kCodeBytes4 = 1, kCodeBytes8 = 2 };
 cudaError_t launch_quantize_rows(const uint16_t *X, int64_t M, int K, const float *mult,
-                                 uint8_t *q, float *scale, bool rot, bool gelu, int bits,
+                                 uint8_t *q, float *scale, bool rot, bool gelu, CodeFormat code,
                                  cudaStream_t st);
 cudaError_t launch_colmax(const uint16_t *X, int64_t M, int K, float *colmax, cudaStream_t st);
 cudaError_t launch_smooth_factors(float *s_io, float *inv_io, int K, double alpha, cudaStream_t st);
@@ -22,9 +27,9 @@ cudaError_t launch_fill(float *out, int n, float v, cudaStream_t st);
 
 // gemm.cu
 struct GemmArgs {
-  const uint8_t *qx;        // [M, K/2] packed int4, or [M, K] int8 codes when a8
+  const uint8_t *qx;        // [M, K/2] packed int4, or [M, K] one code per byte when a8
   const uint8_t *qw;        // [N, K/2] packed int4 (used when qw8 == nullptr)
-  const int8_t *qw8;        // [N, K] widened weight codes (int8 codes when a8), or nullptr
+  const int8_t *qw8;        // [N, K] one weight code per byte (same order as qx when a8), or nullptr
   const int32_t *colsum;    // [N] per-row code sums (with qw8)
   const float *scale_tok;   // [M]
   const float *scale_ch;    // [N]
@@ -33,7 +38,8 @@ struct GemmArgs {
   int32_t *acc;             // [M, N] int32 accumulators instead of y (test path)
   int64_t M;
   int N, K;
-  bool a8;                  // W8A8: qx and qw8 hold 8-bit codes in natural order
+  bool a8;                  // qx and qw8 hold one code per byte in the same order (int8 codes,
+                            // or int4 codes in operand order): no widening
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,

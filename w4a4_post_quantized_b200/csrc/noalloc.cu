@@ -62,7 +62,7 @@ extern "C" w4a4_status w4a4_linear_fused_noalloc(const uint16_t *X, int64_t M,
   if (M < 0) return W4A4_ERR_SHAPE;
   // the workspace this call needs must fit the built-in scratch; unsupported K
   // is reported by w4a4_linear_fused below
-  const size_t need = w4a4_workspace_bytes_ex(M, w->K, flags);
+  const size_t need = w4a4_workspace_bytes_min(M, w->K, flags);
   if (need > W4A4_NOALLOC_SCRATCH_BYTES) return W4A4_ERR_SHAPE;
   cudaError_t err = cudaSuccess;
   void *scratch = scratch_on_current_device(&err);

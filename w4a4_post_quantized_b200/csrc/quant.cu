@@ -1,8 +1,12 @@
 // quant.cu -- the HBM-bound half of the DSFQ W4A4 linear on sm_100a:
 //   * quantize_rows: bf16 row -> (optional GELU) -> Hadamard rotation (fast
 //     Walsh-Hadamard transform, fp32) -> per-channel multiplier -> per-row
-//     absmax -> symmetric int4 codes packed two per byte + fp32 step (or, for
-//     the W8A8 setting, one int8 code per byte with step absmax / 127).
+//     absmax -> symmetric int4 codes + fp32 step.  Three code formats:
+//     int4 packed two per byte (the storage format); int4 one per byte in the
+//     tensor-core operand order (within every 8 elements: 0, 2, 4, 6, 1, 3,
+//     5, 7 -- the order of the expanded weights), which the GEMM then reads
+//     without widening; int8 one per byte in natural order with step
+//     absmax / 127 (the W8A8 setting).
 //     Activations use multiplier 1/s (pre-global rotation, then post-local
 //     smoothing), weights use s; both follow page "十亿参数的三维重建模型，能塞进手机吗？",
 //     sections 预全局旋转 / 后局部平滑 / 训练后量化（PTQ） / 细粒度量化粒度.
@@ -237,11 +241,12 @@ __device__ __forceinline__ uint32_t low_bytes(uint32_t a, uint32_t b, uint32_t c
 }
 
 // Per-channel multiplier (from the block's shared table), per-row absmax,
-// codes, packed store for a phase-2 row.  The transform's 1/sqrt(K) is an
-// exact power of two, so it changes neither the absmax position nor any
-// code: it is applied to the stored step only.  BITS = 4: codes in [-7, 7]
-// packed two per byte; BITS = 8: codes in [-127, 127], one per byte.
-template <int K, bool ROT, int BITS>
+// codes, store for a phase-2 row.  The transform's 1/sqrt(K) is an exact
+// power of two, so it changes neither the absmax position nor any code: it is
+// applied to the stored step only.  CODE (CodeFormat): kCodePacked4 codes in
+// [-7, 7] two per byte; kCodeBytes4 the same codes one per byte in operand
+// order; kCodeBytes8 codes in [-127, 127] one per byte.
+template <int K, bool ROT, int CODE>
 __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], int lane, int64_t row,
                                                    const float4 *__restrict__ mtab,
                                                    uint8_t *__restrict__ q, float *__restrict__ scale) {
@@ -262,8 +267,7 @@ __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], i
   float amax = fmax3(am[0], am[1], fmaxf(am[2], am[3]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
-  constexpr float kQmax = BITS == 4 ? 7.0f : 127.0f;
+  constexpr float kQmax = CODE == kCodeBytes8 ? 127.0f : 7.0f;
   if (lane == 0) scale[row] = (ROT ? amax * RowShape<K>::kInvSqrtK : amax) / kQmax;
   if (amax < 0x1p-100f) {  // keep kQmax/amax finite: exact power-of-two rescale, same codes
 #pragma unroll
@@ -278,13 +282,18 @@ __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], i
   const unsigned long long inv2 = pack2(inv, inv), magic2 = pack2(12582912.0f, 12582912.0f);
 #pragma unroll
   for (int k = 0; k < V; k += 2) fma_x2(v[k], v[k + 1], inv2, magic2);
-  if constexpr (BITS == 8) {
-    // word w: the codes of elements 4w .. 4w + 3, one byte each
+  if constexpr (CODE != kCodePacked4) {
+    // one byte per code.  Natural order: word w holds elements 4w .. 4w + 3.
+    // Operand order: the word pair (2g, 2g + 1) holds elements 8g + 0, 2, 4, 6
+    // and 8g + 1, 3, 5, 7.
     uint32_t words[V / 4];
 #pragma unroll
-    for (int w = 0; w < V / 4; ++w)
-      words[w] = low_bytes(__float_as_uint(v[4 * w]), __float_as_uint(v[4 * w + 1]),
-                           __float_as_uint(v[4 * w + 2]), __float_as_uint(v[4 * w + 3]));
+    for (int w = 0; w < V / 4; ++w) {
+      const int e0 = CODE == kCodeBytes8 ? 4 * w : 8 * (w >> 1) + (w & 1);
+      const int d = CODE == kCodeBytes8 ? 1 : 2;
+      words[w] = low_bytes(__float_as_uint(v[e0]), __float_as_uint(v[e0 + d]),
+                           __float_as_uint(v[e0 + 2 * d]), __float_as_uint(v[e0 + 3 * d]));
+    }
     uint4 *dst = reinterpret_cast<uint4 *>(q + row * K + static_cast<int64_t>(lane) * V);
 #pragma unroll
     for (int c = 0; c < V / 16; ++c)
@@ -322,7 +331,7 @@ struct QuantStaging {
 // NS rows in flight: 1-D bulk copies (TMA engine) stream its next rows into a
 // private shared-memory ring while it transforms the current one, so the HBM
 // latency is hidden without occupancy.
-template <int K, bool ROT, bool GELU, int BITS>
+template <int K, bool ROT, bool GELU, int CODE>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_rows_kernel(const uint16_t *__restrict__ X, int64_t M, const float *__restrict__ mult,
                          uint8_t *__restrict__ q, float *__restrict__ scale,
@@ -395,7 +404,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         ++issued;
       }
     }
-    quantize_store_row<K, ROT, BITS>(v, lane, row, mtab, q, scale);
+    quantize_store_row<K, ROT, CODE>(v, lane, row, mtab, q, scale);
   }
   // after a timed-out wait, let the copies still in flight land before exiting
   if (lane == 0)
@@ -475,10 +484,10 @@ int row_grid(Kern kern, int64_t rows) {
   return static_cast<int>(need < g ? need : g);
 }
 
-template <int K, bool ROT, bool GELU, int BITS>
+template <int K, bool ROT, bool GELU, int CODE>
 cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint8_t *q,
                            float *scale, cudaStream_t st) {
-  auto kern = quantize_rows_kernel<K, ROT, GELU, BITS>;
+  auto kern = quantize_rows_kernel<K, ROT, GELU, CODE>;
   constexpr int smem = QuantStaging<K>::SMEM;
   static int per_sm_dev[64] = {};  // per device: attribute set and occupancy known
   int dev = 0;
@@ -518,25 +527,31 @@ cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint
 int device_sm_count() { return num_sms(); }
 
 namespace {
-template <int K, int BITS>
-cudaError_t launch_quant_kb(const uint16_t *X, int64_t M, const float *mult, uint8_t *q,
+template <int K, int CODE>
+cudaError_t launch_quant_kc(const uint16_t *X, int64_t M, const float *mult, uint8_t *q,
                             float *scale, bool rot, bool gelu, cudaStream_t st) {
-  if (rot) return gelu ? launch_quant_k<K, true, true, BITS>(X, M, mult, q, scale, st)
-                       : launch_quant_k<K, true, false, BITS>(X, M, mult, q, scale, st);
-  return gelu ? launch_quant_k<K, false, true, BITS>(X, M, mult, q, scale, st)
-              : launch_quant_k<K, false, false, BITS>(X, M, mult, q, scale, st);
+  if (rot) return gelu ? launch_quant_k<K, true, true, CODE>(X, M, mult, q, scale, st)
+                       : launch_quant_k<K, true, false, CODE>(X, M, mult, q, scale, st);
+  return gelu ? launch_quant_k<K, false, true, CODE>(X, M, mult, q, scale, st)
+              : launch_quant_k<K, false, false, CODE>(X, M, mult, q, scale, st);
+}
+template <int CODE>
+cudaError_t launch_quant_c(const uint16_t *X, int64_t M, int K, const float *mult, uint8_t *q,
+                           float *scale, bool rot, bool gelu, cudaStream_t st) {
+  return K == 1024 ? launch_quant_kc<1024, CODE>(X, M, mult, q, scale, rot, gelu, st)
+                   : launch_quant_kc<4096, CODE>(X, M, mult, q, scale, rot, gelu, st);
 }
 }  // namespace
 
 cudaError_t launch_quantize_rows(const uint16_t *X, int64_t M, int K, const float *mult,
-                                 uint8_t *q, float *scale, bool rot, bool gelu, int bits,
+                                 uint8_t *q, float *scale, bool rot, bool gelu, CodeFormat code,
                                  cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  if (bits == 8)
-    return K == 1024 ? launch_quant_kb<1024, 8>(X, M, mult, q, scale, rot, gelu, st)
-                     : launch_quant_kb<4096, 8>(X, M, mult, q, scale, rot, gelu, st);
-  return K == 1024 ? launch_quant_kb<1024, 4>(X, M, mult, q, scale, rot, gelu, st)
-                   : launch_quant_kb<4096, 4>(X, M, mult, q, scale, rot, gelu, st);
+  switch (code) {
+    case kCodeBytes4: return launch_quant_c<kCodeBytes4>(X, M, K, mult, q, scale, rot, gelu, st);
+    case kCodeBytes8: return launch_quant_c<kCodeBytes8>(X, M, K, mult, q, scale, rot, gelu, st);
+    default: return launch_quant_c<kCodePacked4>(X, M, K, mult, q, scale, rot, gelu, st);
+  }
 }
 
 cudaError_t launch_colmax(const uint16_t *X, int64_t M, int K, float *colmax, cudaStream_t st) {

@@ -28,6 +28,7 @@ W4A4_DEV_TIMEOUT = 0x1
 W4A4_FLAG_GELU = 0x1
 W4A4_FLAG_PLAIN = 0x2
 W4A4_FLAG_INT8 = 0x4
+W4A4_FLAG_UNPACKED = 0x8
 
 _vp, _i32, _i64, _u32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
                                     ctypes.c_float, ctypes.c_size_t)
@@ -46,11 +47,13 @@ def _sig(name, res, args):
 
 
 _workspace_bytes = _sig("w4a4_workspace_bytes", _sz, [_i64, _i32])
-_workspace_bytes_ex = _sig("w4a4_workspace_bytes_ex", _sz, [_i64, _i32, _u32])
+_workspace_bytes_min = _sig("w4a4_workspace_bytes_min", _sz, [_i64, _i32, _u32])
 _prepare = _sig("w4a4_prepare_weights", ctypes.c_int,
                 [_vp, _vp, _i32, _i32, _vp, _i64, _f32, _u32, ctypes.POINTER(W4A4WeightsT), _vp])
 _quantize = _sig("w4a4_quantize_act", ctypes.c_int, [_vp, _i64, _i32, _vp, _vp, _vp, _u32, _vp])
 _linear = _sig("w4a4_linear", ctypes.c_int, [_vp, _vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp])
+_linear_ex = _sig("w4a4_linear_ex", ctypes.c_int,
+                  [_vp, _vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _u32, _vp])
 _fused = _sig("w4a4_linear_fused", ctypes.c_int,
               [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp, _sz, _u32, _vp])
 _fused_noalloc = _sig("w4a4_linear_fused_noalloc", ctypes.c_int,
@@ -100,8 +103,8 @@ def w4a4_workspace_bytes(M: int, K: int) -> int:
     return int(_workspace_bytes(M, K))
 
 
-def w4a4_workspace_bytes_ex(M: int, K: int, flags: int) -> int:
-    return int(_workspace_bytes_ex(M, K, flags))
+def w4a4_workspace_bytes_min(M: int, K: int, flags: int) -> int:
+    return int(_workspace_bytes_min(M, K, flags))
 
 
 class PreparedWeights:
@@ -144,7 +147,7 @@ def w4a4_prepare_weights(W: torch.Tensor, bias, X_calib, alpha: float = 0.5, fla
 def w4a4_quantize_act(X: torch.Tensor, inv_smooth, flags: int = 0, qx=None, scale_tok=None,
                       stream=None):
     M, K = X.shape
-    width = K if flags & W4A4_FLAG_INT8 else K // 2
+    width = K if flags & (W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED) else K // 2
     qx = qx if qx is not None else torch.empty((M, width), dtype=torch.uint8, device=X.device)
     scale_tok = scale_tok if scale_tok is not None else torch.empty(M, dtype=torch.float32, device=X.device)
     _check(_quantize(_ptr(X), M, K, _ptr(inv_smooth), _ptr(qx), _ptr(scale_tok), flags,
@@ -160,11 +163,20 @@ def w4a4_linear(qx: torch.Tensor, scale_tok: torch.Tensor, w: PreparedWeights, Y
     return Y
 
 
+def w4a4_linear_ex(qx: torch.Tensor, scale_tok: torch.Tensor, w: PreparedWeights, flags: int = 0, Y=None,
+                   stream=None):
+    M = qx.shape[0]
+    Y = Y if Y is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=qx.device)
+    _check(_linear_ex(_ptr(qx), _ptr(scale_tok), M, ctypes.byref(w.struct), _ptr(Y), flags,
+                      _stream(stream)), "w4a4_linear_ex")
+    return Y
+
+
 def w4a4_linear_fused(X: torch.Tensor, w: PreparedWeights, Y=None, workspace=None, flags: int = 0,
                       stream=None):
     M = X.shape[0]
     Y = Y if Y is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
-    need = w4a4_workspace_bytes_ex(M, w.K, flags)
+    need = w4a4_workspace_bytes(M, w.K)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
     _check(_fused(_ptr(X), M, ctypes.byref(w.struct), _ptr(Y), _ptr(workspace),
