@@ -2,6 +2,7 @@
 include/w4a4.h declares, and rejects bad arguments on the host (before any
 CUDA call) with the documented status codes."""
 import ctypes
+import glob
 import os
 import re
 
@@ -21,15 +22,19 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(w4a4_[a-z0-9_]+)\s*\(", text)))
+    """Every function any include/*.h declares."""
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b((?:w4a4|tq)_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ["w4a4_prepare_weights", "w4a4_quantize_act", "w4a4_linear", "w4a4_linear_fused",
-              "w4a4_workspace_bytes", "w4a4_gemm_s32", "w4a4_get_device_status"]:
+              "w4a4_workspace_bytes", "w4a4_gemm_s32", "w4a4_get_device_status",
+              "tq_codebook", "tq_encode", "tq_decode"]:
         assert n in names
 
 
@@ -259,3 +264,34 @@ def test_host_pipeline_argument_checks(lib):
     assert f(None, 10, ctypes.byref(w), A, 128, A, need, fake_pipe, 0, None) == 1
     assert f(A, 10, ctypes.byref(w), A, 128, A + 4, need, fake_pipe, 0, None) == 3  # misaligned
     assert f(A, 10, ctypes.byref(w), A, 128, A, need - 1, fake_pipe, 0, None) == 2  # too small
+
+
+def test_tq_codebook_and_argument_checks(lib):
+    """The codec's host codebook (no GPU needed) matches the oracle's Lloyd-Max
+    to fp32 rounding; encode / decode reject bad arguments on the host."""
+    import numpy as np
+    from oracle import turboquant as tq
+    f32 = ctypes.POINTER(ctypes.c_float)
+    lib.tq_codebook.argtypes = [ctypes.c_int32, ctypes.c_int32, f32, f32]
+    c = np.empty(16, np.float32)
+    t = np.empty(15, np.float32)
+    assert lib.tq_codebook(1024, 4, c.ctypes.data_as(f32), t.ctypes.data_as(f32)) == 0
+    oc, ot = tq.lloyd_max(1024, 4)
+    np.testing.assert_allclose(c, oc, rtol=2 ** -23, atol=0)
+    np.testing.assert_allclose(t, ot, rtol=2 ** -23, atol=1e-30)
+    assert t[7] == 0.0 and np.array_equal(c, -c[::-1])
+    assert lib.tq_codebook(1024, 3, c.ctypes.data_as(f32), t.ctypes.data_as(f32)) == 4
+    assert lib.tq_codebook(512, 4, c.ctypes.data_as(f32), t.ctypes.data_as(f32)) == 4
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    lib.tq_encode.argtypes = [vp, i64, i32, vp, vp, vp, vp, vp]
+    lib.tq_decode.argtypes = [vp, vp, i64, i32, vp, vp, vp, vp]
+    E, D = lib.tq_encode, lib.tq_decode
+    assert E(A, 10, 512, A, A, A, A, None) == 4
+    assert E(A, -1, 1024, A, A, A, A, None) == 2
+    assert E(A, 0, 1024, A, A, A, A, None) == 0
+    assert E(None, 10, 1024, A, A, A, A, None) == 1
+    assert E(A + 4, 10, 1024, A, A, A, A, None) == 3
+    assert D(A, A, 10, 2048, A, A, A, None) == 4
+    assert D(A, A, 0, 1024, A, A, A, None) == 0
+    assert D(A, None, 10, 1024, A, A, A, None) == 1
+    assert D(A, A, 10, 1024, A, A, A + 8, None) == 3

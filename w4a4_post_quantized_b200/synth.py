@@ -103,3 +103,26 @@ CONFIGS = {
                           layers=[("qkv", 1024, 3072), ("proj", 1024, 1024),
                                   ("fc1", 1024, 4096), ("fc2", 4096, 1024)]),
 }
+
+
+# KV-cache vectors for the 3DTurboQuant codec (page "3DTurboQuant: Training-
+# Free Near-Optimal Quantization for 3D Reconstruction Models", section 4.2:
+# the DUSt3R KV cache, d = 1024, about 100 MB in fp32 = 24576 vectors).
+KV_DIM = 1024
+KV_VECTORS = 24576
+
+
+def kv_vectors(n: int, d: int, seed: int) -> np.ndarray:
+    """fp32 [n, d] KV-like vectors: N(0, 1) entries, 8 seeded outlier channels
+    x15, and a per-vector scale drawn log-uniformly from [0.25, 4]."""
+    rng = np.random.Generator(np.random.PCG64([seed, 0x4B56]))
+    x = rng.standard_normal((n, d), dtype=np.float32)
+    x[:, outlier_channels(d, seed)] *= np.float32(OUTLIER_SCALE)
+    x *= np.exp(rng.uniform(np.log(0.25), np.log(4.0), size=(n, 1))).astype(np.float32)
+    return x
+
+
+def random_signs(d: int, seed: int) -> np.ndarray:
+    """fp32 [d] of independent +-1 (the random sign vector of a rotation)."""
+    rng = np.random.Generator(np.random.PCG64([seed, 0x516E]))
+    return np.where(rng.random(d) < 0.5, np.float32(-1.0), np.float32(1.0)).astype(np.float32)

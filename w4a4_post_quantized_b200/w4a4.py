@@ -67,6 +67,9 @@ _fused_host = _sig("w4a4_linear_fused_host", ctypes.c_int,
 _expand = _sig("w4a4_expand_weights", ctypes.c_int, [ctypes.POINTER(W4A4WeightsT), _vp])
 _get_status = _sig("w4a4_get_device_status", ctypes.c_int, [_vp, ctypes.POINTER(_u32)])
 _clear_status = _sig("w4a4_clear_device_status", ctypes.c_int, [_vp])
+_tq_codebook = _sig("tq_codebook", ctypes.c_int, [_i32, _i32, _vp, _vp])
+_tq_encode = _sig("tq_encode", ctypes.c_int, [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp])
+_tq_decode = _sig("tq_decode", ctypes.c_int, [_vp, _vp, _i64, _i32, _vp, _vp, _vp, _vp])
 _status_string = _sig("w4a4_status_string", ctypes.c_char_p, [ctypes.c_int])
 _version = _sig("w4a4_version", ctypes.c_char_p, [])
 
@@ -267,3 +270,34 @@ def w4a4_get_device_status(stream=None) -> int:
 
 def w4a4_clear_device_status(stream=None) -> None:
     _check(_clear_status(_stream(stream)), "w4a4_clear_device_status")
+
+
+# ------------------------------------------------- 3DTurboQuant codec (include/tq.h)
+def tq_codebook(d: int = 1024, b: int = 4):
+    """Host Lloyd-Max codebook: (centroids [2^b], boundaries [2^b - 1]) as fp32 numpy arrays."""
+    import numpy as np
+    c = np.empty(1 << b, np.float32)
+    t = np.empty((1 << b) - 1, np.float32)
+    _check(_tq_codebook(d, b, c.ctypes.data_as(_vp), t.ctypes.data_as(_vp)), "tq_codebook")
+    return c, t
+
+
+def tq_encode(X: torch.Tensor, signs: torch.Tensor, boundaries: torch.Tensor, codes=None, norms=None,
+              stream=None):
+    """X [n, d] fp32 -> (codes uint8 [n, d/2], norms fp32 [n])."""
+    n, d = X.shape
+    codes = codes if codes is not None else torch.empty((n, d // 2), dtype=torch.uint8, device=X.device)
+    norms = norms if norms is not None else torch.empty(n, dtype=torch.float32, device=X.device)
+    _check(_tq_encode(_ptr(X), n, d, _ptr(signs), _ptr(boundaries), _ptr(codes), _ptr(norms),
+                      _stream(stream)), "tq_encode")
+    return codes, norms
+
+
+def tq_decode(codes: torch.Tensor, norms: torch.Tensor, signs: torch.Tensor, centroids: torch.Tensor,
+              Y=None, stream=None):
+    """(codes [n, d/2], norms [n]) -> Y [n, d] fp32."""
+    n, d = codes.shape[0], codes.shape[1] * 2
+    Y = Y if Y is not None else torch.empty((n, d), dtype=torch.float32, device=codes.device)
+    _check(_tq_decode(_ptr(codes), _ptr(norms), n, d, _ptr(signs), _ptr(centroids), _ptr(Y),
+                      _stream(stream)), "tq_decode")
+    return Y
