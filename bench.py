@@ -26,6 +26,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -640,13 +641,196 @@ def run_stack(args, st, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+TQ_WORKLOAD = "kv_turboquant"
+TQ_METRIC = "3DTurboQuant KV-cache codec GB/s (encode + decode, algorithmic bytes), % of HBM BW"
+
+
+def tq_bytes(n: int, d: int):
+    """Algorithmic bytes of one encode and one decode of n vectors (fp32 in and
+    out, 4-bit codes + fp32 norm)."""
+    packed = n * (d // 2 + 4)
+    return n * 4 * d + packed, packed + n * 4 * d
+
+
+def tq_oracle_sample(rows: int, seed: int = 0):
+    """The oracle's encode + decode on `rows` KV vectors (untimed setup)."""
+    from oracle import turboquant as tq
+    d = synth.KV_DIM
+    X = synth.kv_vectors(rows, d, seed=seed + 10)
+    s = synth.random_signs(d, seed=seed + 2)
+    c, t = tq.lloyd_max(d, 4)
+
+    def run():
+        codes, gamma, _ = tq.encode(X, s, t)
+        return tq.decode(codes, gamma, s, c)
+    import oracle
+    return run, rows, oracle.max_threads()
+
+
+def run_tq(args, world, rank, local):
+    """The 3DTurboQuant KV-cache codec on the page's DUSt3R case: 24576 vectors
+    of d = 1024 (100.7 MB of fp32), b = 4; a step encodes and decodes one batch."""
+    import torch
+    from w4a4_post_quantized_b200 import w4a4
+    n, d = synth.KV_VECTORS, synth.KV_DIM
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    c, t = w4a4.tq_codebook(d, 4)
+    cd, td = torch.from_numpy(c).to(dev), torch.from_numpy(t).to(dev)
+    seed = 1000 * rank
+    sg = torch.from_numpy(synth.random_signs(d, seed=seed + 2)).to(dev)
+    Xs = [torch.from_numpy(synth.kv_vectors(n, d, seed=seed + 10 + i)).to(dev) for i in range(NSETS)]
+    Cs = [torch.empty((n, d // 2), dtype=torch.uint8, device=dev) for _ in range(NSETS)]
+    Ns = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(NSETS)]
+    Ys = [torch.empty((n, d), dtype=torch.float32, device=dev) for _ in range(NSETS)]
+    enc = lambda j: w4a4.tq_encode(Xs[j], sg, td, codes=Cs[j], norms=Ns[j])
+    dec = lambda j: w4a4.tq_decode(Cs[j], Ns[j], sg, cd, Y=Ys[j])
+
+    def step(i):
+        enc(i % NSETS)
+        dec(i % NSETS)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    w4a4.w4a4_clear_device_status()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        iso = {}
+        n_iso = max(3, min(args.steps, 200))
+        for name, fn in (("encode", enc), ("decode", dec)):
+            for i in range(3):
+                fn(i % NSETS)
+            k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            k0.record(stream)
+            for i in range(n_iso):
+                fn(i % NSETS)
+            k1.record(stream)
+            torch.cuda.synchronize()
+            iso[name] = max_over_ranks(world, k0.elapsed_time(k1)) / n_iso
+    status = w4a4.w4a4_get_device_status()
+    elapsed_ms = max_over_ranks(world, t0.elapsed_time(t1))
+    ms_step = elapsed_ms / args.steps
+    be, bd = tq_bytes(n, d)
+    value = world * (be + bd) * args.steps / (elapsed_ms * 1e-3) / 1e9
+    # reconstruction quality of the timed batch 0 against the page's bound
+    step(0)
+    torch.cuda.synchronize()
+    X64 = Xs[0].double()
+    rel = (((X64 - Ys[0].double()) ** 2).sum(1) / (X64 ** 2).sum(1))
+    bound = math.sqrt(3.0) * math.pi / 2.0 * 4.0 ** -4
+    # end to end: X from pinned host memory, encode + decode, Y back to pinned host memory
+    Xh = Xs[0].cpu().pin_memory()
+    Yh = torch.empty((n, d), dtype=torch.float32, pin_memory=True)
+    Xd, Yd = torch.empty_like(Xs[0]), torch.empty_like(Ys[0])
+
+    def host_step():
+        Xd.copy_(Xh, non_blocking=True)
+        w4a4.tq_encode(Xd, sg, td, codes=Cs[0], norms=Ns[0])
+        w4a4.tq_decode(Cs[0], Ns[0], sg, cd, Y=Yd)
+        Yh.copy_(Yd, non_blocking=True)
+    for _ in range(3):
+        host_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        host_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / e2e_steps
+    peaks = load_peaks()
+    kern = "tq_encode_kernel" if iso["encode"] >= iso["decode"] else "tq_decode_kernel"
+    kb = be if kern == "tq_encode_kernel" else bd
+    kms = max(iso["encode"], iso["decode"])
+    ach = kb / (kms * 1e-3) / 1e9
+    line = {
+        "metric": TQ_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 in/out, u4 codes", "data": "synthetic",
+        "vectors_per_s": world * n * args.steps / (elapsed_ms * 1e-3),
+        "config": {"workload": "3DTurboQuant DUSt3R KV cache: 24576 x 1024 fp32 (100.7 MB), b = 4",
+                   "n": n, "d": d, "bits": 4, "per_rank_batch": n,
+                   "parallelism": f"dp{world} (independent replicas)",
+                   "l2": f"inputs/outputs rotated over {NSETS} buffer sets (~{(8 * n * d + n * d // 2) * NSETS / 1e6:.0f} MB > L2)"},
+        "clocks": clk.summary(),
+        "e2e": {"value": world * (be + bd) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 4 * n * d, "d2h_bytes_per_step": 4 * n * d,
+                "api": "tq_encode + tq_decode (C ABI) with X copied from and Y copied to pinned host memory"},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "kernel": kern, "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm"], "traffic": None,
+                     "ms_per_launch": kms, "algorithmic_bytes_per_launch": kb,
+                     "encode_ms": iso["encode"], "decode_ms": iso["decode"],
+                     "encode_gbs": be / (iso["encode"] * 1e-3) / 1e9,
+                     "decode_gbs": bd / (iso["decode"] * 1e-3) / 1e9,
+                     "timing": f"CUDA events around {n_iso} back-to-back launches of each kernel alone"},
+        "quality": {"mse_rel_mean": float(rel.mean()), "mse_rel_max": float(rel.max()),
+                    "page_bound": bound, "compression_vs_fp32": (4 * n * d) / (n * (d // 2) + 4 * n)},
+        "device_status": status,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        run, r, cores = tq_oracle_sample(256)
+        passes, tt = 0, 0.0
+        while passes < 2000 and tt < 10.0:  # about 10 s of CPU work
+            t_ = time.perf_counter()
+            run()
+            tt += time.perf_counter() - t_
+            passes += 1
+        dt = tt / passes
+        eb, db = tq_bytes(r, d)
+        line["cpu_baseline"] = {"value": (eb + db) / dt / 1e9, "unit": "GB/s", "cores": cores,
+                                "kind": "oracle", "sample": f"{r} of {n} vectors per pass, {passes} passes, "
+                                                            f"{dt:.2f} s per pass"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_tq_reference(args, world, rank):
+    if rank != 0:
+        return
+    d = synth.KV_DIM
+    probe, r0, _ = tq_oracle_sample(64)
+    t_ = time.perf_counter()
+    probe()
+    per_vec = (time.perf_counter() - t_) / r0
+    rows = int(min(1024, max(16, 120.0 / max(1, args.steps + args.warmup) / per_vec)))
+    run, r, cores = tq_oracle_sample(rows)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    eb, db = tq_bytes(r, d)
+    gbs = (eb + db) / dt / 1e9
+    line = {"impl": "reference", "metric": TQ_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "3DTurboQuant DUSt3R KV cache, d = 1024, b = 4", "n_sampled": r},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{r} of {synth.KV_VECTORS} vectors per step"},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(STACKS), default="c2_frame_qkv")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(STACKS) + [TQ_WORKLOAD],
+                    default="c2_frame_qkv")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--e2e-chunk", type=int, default=1408, help="row chunk of the host-buffer call")
     ap.add_argument("--cpu-rows", type=int, default=512)
@@ -656,6 +840,18 @@ def main():
         ap.error("--warmup must be at least 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.workload == TQ_WORKLOAD:
+        if args.impl == "reference":
+            run_tq_reference(args, world, rank)
+            return
+        world, rank, local = dist_setup()
+        try:
+            run_tq(args, world, rank, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     if args.workload in STACKS:
         if args.impl == "reference":
             if rank == 0:
