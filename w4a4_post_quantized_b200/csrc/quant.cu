@@ -165,11 +165,68 @@ __device__ __forceinline__ uint32_t low_bytes(uint32_t a, uint32_t b, uint32_t c
 // applied to the stored step only.  CODE (CodeFormat): kCodePacked4 codes in
 // [-7, 7] two per byte; kCodeBytes4 the same codes one per byte in operand
 // order; kCodeBytes8 codes in [-127, 127] one per byte.
-template <int K, bool ROT, int CODE>
-__device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], int lane, int64_t row,
-                                                   const float4 *__restrict__ mtab,
-                                                   uint8_t *__restrict__ q, float *__restrict__ scale) {
-  constexpr int V = RowShape<K>::V;
+// Bytes the codes of `elems` elements take in a code format.
+template <int CODE>
+constexpr int code_bytes_of(int elems) {
+  return CODE == kCodePacked4 ? elems / 2 : elems;
+}
+
+// Codes of V consecutive elements whose row absmax is amax, stored at dst
+// (16-byte aligned).  code = round-half-even(v * kQmax / amax); |v * inv| <=
+// kQmax (1 + 2^-24), so no clamp can ever act.  Adding 1.5 * 2^23 in the same
+// fused operation rounds the exact product to an integer whose low 8 bits are
+// the two's-complement code.
+template <int V, int CODE>
+__device__ __forceinline__ void store_codes(float (&v)[V], float amax, uint8_t *__restrict__ dst) {
+  constexpr float kQmax = CODE == kCodeBytes8 ? 127.0f : 7.0f;
+  if (amax < 0x1p-100f) {  // keep kQmax/amax finite: exact power-of-two rescale, same codes
+#pragma unroll
+    for (int r = 0; r < V; ++r) v[r] *= 0x1p+64f;
+    amax *= 0x1p+64f;
+  }
+  const float inv = (amax > 0.0f) ? kQmax / amax : 0.0f;
+  const unsigned long long inv2 = pack2(inv, inv), magic2 = pack2(12582912.0f, 12582912.0f);
+#pragma unroll
+  for (int k = 0; k < V; k += 2) fma_x2(v[k], v[k + 1], inv2, magic2);
+  uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+  if constexpr (CODE != kCodePacked4) {
+    // one byte per code.  Natural order: word w holds elements 4w .. 4w + 3.
+    // Operand order: the word pair (2g, 2g + 1) holds elements 8g + 0, 2, 4, 6
+    // and 8g + 1, 3, 5, 7.
+    uint32_t words[V / 4];
+#pragma unroll
+    for (int w = 0; w < V / 4; ++w) {
+      const int e0 = CODE == kCodeBytes8 ? 4 * w : 8 * (w >> 1) + (w & 1);
+      const int d = CODE == kCodeBytes8 ? 1 : 2;
+      words[w] = low_bytes(__float_as_uint(v[e0]), __float_as_uint(v[e0 + d]),
+                           __float_as_uint(v[e0 + 2 * d]), __float_as_uint(v[e0 + 3 * d]));
+    }
+#pragma unroll
+    for (int c = 0; c < V / 16; ++c)
+      d4[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+  } else {
+    // word w: codes of elements 8w .. 8w + 7, element 2i in the low nibble of byte i
+    uint32_t words[V / 8];
+#pragma unroll
+    for (int w = 0; w < V / 8; ++w) {
+      uint32_t b[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) b[e] = __float_as_uint(v[8 * w + e]);
+      const uint32_t even = low_bytes(b[0], b[2], b[4], b[6]);
+      const uint32_t odd = low_bytes(b[1], b[3], b[5], b[7]);
+      words[w] = (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
+    }
+#pragma unroll
+    for (int c = 0; c < V / 32; ++c)
+      d4[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+  }
+}
+
+// Per-channel multiplier (from the block's shared table) and this lane's
+// absmax of a phase-2 row (V values).
+template <int V, bool ROT>
+__device__ __forceinline__ float mult_lane_absmax(float (&v)[V], int lane,
+                                                  const float4 *__restrict__ mtab) {
   if (ROT) {
 #pragma unroll
     for (int c = 0; c < V / 4; ++c) {
@@ -183,57 +240,26 @@ __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], i
   for (int r = 0; r < V; r += 8)
 #pragma unroll
     for (int a = 0; a < 4; ++a) am[a] = fmax3(am[a], fabsf(v[r + 2 * a]), fabsf(v[r + 2 * a + 1]));
-  float amax = fmax3(am[0], am[1], fmaxf(am[2], am[3]));
+  return fmax3(am[0], am[1], fmaxf(am[2], am[3]));
+}
+
+// Per-channel multiplier, per-row absmax, codes, store for a phase-2 row.
+// The transform's 1/sqrt(K) is an exact power of two, so it changes neither
+// the absmax position nor any code: it is applied to the stored step only.
+// CODE (CodeFormat): kCodePacked4 codes in [-7, 7] two per byte; kCodeBytes4
+// the same codes one per byte in operand order; kCodeBytes8 codes in
+// [-127, 127] one per byte.
+template <int K, bool ROT, int CODE>
+__device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], int lane, int64_t row,
+                                                   const float4 *__restrict__ mtab,
+                                                   uint8_t *__restrict__ q, float *__restrict__ scale) {
+  constexpr int V = RowShape<K>::V;
+  float amax = mult_lane_absmax<V, ROT>(v, lane, mtab);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   constexpr float kQmax = CODE == kCodeBytes8 ? 127.0f : 7.0f;
   if (lane == 0) scale[row] = (ROT ? amax * RowShape<K>::kInvSqrtK : amax) / kQmax;
-  if (amax < 0x1p-100f) {  // keep kQmax/amax finite: exact power-of-two rescale, same codes
-#pragma unroll
-    for (int r = 0; r < V; ++r) v[r] *= 0x1p+64f;
-    amax *= 0x1p+64f;
-  }
-  const float inv = (amax > 0.0f) ? kQmax / amax : 0.0f;
-  // code = round-half-even(v * inv); |v * inv| <= kQmax (1 + 2^-24), so no
-  // clamp can ever act.  Adding 1.5 * 2^23 in the same fused operation rounds
-  // the exact product to an integer whose low 8 bits are the two's-complement
-  // code.
-  const unsigned long long inv2 = pack2(inv, inv), magic2 = pack2(12582912.0f, 12582912.0f);
-#pragma unroll
-  for (int k = 0; k < V; k += 2) fma_x2(v[k], v[k + 1], inv2, magic2);
-  if constexpr (CODE != kCodePacked4) {
-    // one byte per code.  Natural order: word w holds elements 4w .. 4w + 3.
-    // Operand order: the word pair (2g, 2g + 1) holds elements 8g + 0, 2, 4, 6
-    // and 8g + 1, 3, 5, 7.
-    uint32_t words[V / 4];
-#pragma unroll
-    for (int w = 0; w < V / 4; ++w) {
-      const int e0 = CODE == kCodeBytes8 ? 4 * w : 8 * (w >> 1) + (w & 1);
-      const int d = CODE == kCodeBytes8 ? 1 : 2;
-      words[w] = low_bytes(__float_as_uint(v[e0]), __float_as_uint(v[e0 + d]),
-                           __float_as_uint(v[e0 + 2 * d]), __float_as_uint(v[e0 + 3 * d]));
-    }
-    uint4 *dst = reinterpret_cast<uint4 *>(q + row * K + static_cast<int64_t>(lane) * V);
-#pragma unroll
-    for (int c = 0; c < V / 16; ++c)
-      dst[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
-    return;
-  }
-  // word w: codes of elements 8w .. 8w + 7, element 2i in the low nibble of byte i
-  uint32_t words[V / 8];
-#pragma unroll
-  for (int w = 0; w < V / 8; ++w) {
-    uint32_t b[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) b[e] = __float_as_uint(v[8 * w + e]);
-    const uint32_t even = low_bytes(b[0], b[2], b[4], b[6]);
-    const uint32_t odd = low_bytes(b[1], b[3], b[5], b[7]);
-    words[w] = (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
-  }
-  uint4 *dst = reinterpret_cast<uint4 *>(q + row * (K / 2) + static_cast<int64_t>(lane) * (V / 2));
-#pragma unroll
-  for (int c = 0; c < V / 32; ++c)
-    dst[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+  store_codes<V, CODE>(v, amax, q + row * code_bytes_of<CODE>(K) + lane * code_bytes_of<CODE>(V));
 }
 
 template <int K>
@@ -408,6 +434,7 @@ cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint
                            float *scale, cudaStream_t st) {
   auto kern = quantize_rows_kernel<K, ROT, GELU, CODE>;
   constexpr int smem = QuantStaging<K>::SMEM;
+  constexpr int kRowsPerBlock = kQuantWarps;  // one warp per row
   static int per_sm_dev[64] = {};  // per device: attribute set and occupancy known
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -421,7 +448,7 @@ cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kQuantWarps * 32, smem);
     per_sm = n < 1 ? 1 : n;
   }
-  const int64_t need = (M + kQuantWarps - 1) / kQuantWarps;
+  const int64_t need = (M + kRowsPerBlock - 1) / kRowsPerBlock;
   const int64_t g = static_cast<int64_t>(num_sms()) * per_sm;
   const int grid = static_cast<int>(need < g ? need : g);
   // programmatic stream serialization: the block setup may overlap the
