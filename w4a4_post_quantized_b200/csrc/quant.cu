@@ -265,7 +265,9 @@ __device__ __forceinline__ void quantize_store_row(float (&v)[RowShape<K>::V], i
 template <int K>
 struct QuantStaging {
   static constexpr int ROWB = 2 * K;                 // bf16 row bytes
-  static constexpr int NS = 2;                        // rows in flight per warp
+  // rows in flight per warp: K = 1024 uses one slot, refilled as soon as the
+  // row has been read into registers (measured faster than two slots)
+  static constexpr int NS = K == 1024 ? 1 : 2;
   static constexpr int WARP_BYTES = NS * ROWB + 32 * 32 * 4;
   static constexpr int OFF_TAB = kQuantWarps * WARP_BYTES;        // multiplier table, K floats
   static constexpr int OFF_BAR = OFF_TAB + 4 * K;
@@ -329,8 +331,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
   for (int64_t row = r0; row < M; row += G, ++i) {
     const int s = static_cast<int>(i % S::NS);
     if (!mbar_wait_drain(&bars[s], static_cast<uint32_t>((i / S::NS) & 1), status)) break;
-    static_assert(S::NS == 2, "the ring's second slot is filled here");
-    if (i == 0 && lane == 0) {
+    if (S::NS == 2 && i == 0 && lane == 0) {  // the ring's second slot
       const int64_t r = r0 + G;
       if (r < M) {
         mbar_arrive_expect_tx(&bars[1], S::ROWB);
@@ -340,8 +341,20 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     }
     float u[V], v[V];
     load_phase1<K, GELU, true>(reinterpret_cast<const unsigned short *>(ring + s * S::ROWB), lane, u);
+    if constexpr (S::NS == 1) {
+      __syncwarp();  // every lane has read the slot: the next row may land there
+      if (lane == 0) {
+        const int64_t rn = row + G;
+        if (rn < M) {
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&bars[0], S::ROWB);
+          bulk_load(ring, X + rn * K, S::ROWB, &bars[0]);
+          ++issued;
+        }
+      }
+    }
     transform_row<K, ROT>(u, lane, tile, v);  // ends with __syncwarp: slot s is no longer read
-    if (lane == 0) {
+    if (S::NS == 2 && lane == 0) {
       const int64_t rn = row + S::NS * G;
       if (rn < M) {
         mbar_arrive_expect_tx(&bars[s], S::ROWB);
