@@ -768,7 +768,8 @@ def run_tq(args, world, rank, local):
                 "api": "tq_encode + tq_decode (C ABI) with X copied from and Y copied to pinned host memory"},
         "gpu_launches": 2 * args.steps,
         "roofline": {"bound": "hbm", "kernel": kern, "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": ach / peaks["hbm"], "traffic": None,
+                     "frac": ach / peaks["hbm"],
+                     "traffic": profile_traffic("tq.cu", f"{kern.split('_kernel')[0]}_kv_turboquant"),
                      "ms_per_launch": kms, "algorithmic_bytes_per_launch": kb,
                      "encode_ms": iso["encode"], "decode_ms": iso["decode"],
                      "encode_gbs": be / (iso["encode"] * 1e-3) / 1e9,
