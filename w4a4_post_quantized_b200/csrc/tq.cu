@@ -29,13 +29,21 @@ constexpr int kTqLevels = 16;     // 2^b, b = 4
 constexpr int kTqWarps = 8;       // warps (vectors in flight) per block
 constexpr float kTqSqrtD = 32.0f;
 
+// The code decision by table: a uniform grid over |y| with cells narrower
+// than the smallest gap between consecutive boundaries holds at most one
+// boundary per cell, so m(|y|) = #{positive boundaries < |y|} = base[cell] +
+// (|y| > boundary in the cell).  kTqCells bounds the grid: 1 / width cells
+// cover |y| <= 1 (|y| <= 1 for a unit vector).
+constexpr int kTqCells = 1024;
+
 struct TqEncodeStaging {
   static constexpr int ROWB = 4 * kTqD;                 // fp32 vector bytes
   static constexpr int NS = 2;                          // vectors in flight per warp
   static constexpr int WARP_BYTES = NS * ROWB + 32 * 32 * 4;
   static constexpr int OFF_SIGN = kTqWarps * WARP_BYTES;  // 32 sign masks
-  static constexpr int OFF_BND = OFF_SIGN + 32 * 4;       // 15 boundaries
-  static constexpr int OFF_BAR = OFF_BND + 64;
+  static constexpr int OFF_BND = OFF_SIGN + 32 * 4;       // 15 boundaries + the cell width
+  static constexpr int OFF_CELL = OFF_BND + 64;           // [kTqCells] (base, boundary in cell units)
+  static constexpr int OFF_BAR = OFF_CELL + kTqCells * 8;
   static constexpr int SMEM = OFF_BAR + kTqWarps * NS * 8;
 };
 
@@ -48,12 +56,28 @@ __device__ __forceinline__ void load_sign_masks(const float *__restrict__ signs,
   }
 }
 
-// Number of the 7 positive boundaries p[0..6] (increasing) strictly below a >= 0.
-__device__ __forceinline__ int count_below(float a, const float (&p)[7]) {
-  int m = a > p[3] ? 4 : 0;
-  m += a > (m ? p[5] : p[1]) ? 2 : 0;
-  const float q = m >= 4 ? (m == 6 ? p[6] : p[4]) : (m == 2 ? p[2] : p[0]);
-  return m + (a > q ? 1 : 0);
+// Fills the block's cell table from the 7 positive boundaries p (increasing):
+// width w = 0.9 x the smallest gap; entry j describes cell c = max(j - 1, 0)
+// (index j = floor(t) + 1 of t = |y| / w, with the index -1 of tiny t folded
+// into cell 0): base = #{p_k < c w}, and the boundary inside [c w, (c + 1) w)
+// in cell units (t units), or +inf.  Returns 1 / w.
+__device__ __forceinline__ float fill_cells(const float *bnd, float2 *cells) {
+  const float *p = bnd + 8;
+  float gap = p[0];
+  for (int k = 1; k < 7; ++k) gap = fminf(gap, p[k] - p[k - 1]);
+  const float w = 0.9f * gap;
+  for (int j = threadIdx.x; j < kTqCells; j += blockDim.x) {
+    const int c = j > 0 ? j - 1 : 0;
+    const float lo = c * w, hi = (c + 1) * w;
+    int base = 0;
+    float inside = __int_as_float(0x7F800000);  // +inf
+    for (int k = 0; k < 7; ++k) {
+      if (p[k] < lo) ++base;
+      else if (p[k] < hi) inside = p[k] / w;
+    }
+    cells[j] = make_float2(__int_as_float(base), inside);
+  }
+  return 1.0f / w;
 }
 
 __global__ void __launch_bounds__(kTqWarps * 32)
@@ -69,6 +93,7 @@ __global__ void __launch_bounds__(kTqWarps * 32)
   float *tile = reinterpret_cast<float *>(ring + S::NS * S::ROWB);
   uint32_t *masks = reinterpret_cast<uint32_t *>(tsmem + S::OFF_SIGN);
   float *bnd = reinterpret_cast<float *>(tsmem + S::OFF_BND);
+  float2 *cells = reinterpret_cast<float2 *>(tsmem + S::OFF_CELL);
   uint64_t *bars = reinterpret_cast<uint64_t *>(tsmem + S::OFF_BAR) + warp * S::NS;
   const int64_t G = static_cast<int64_t>(gridDim.x) * kTqWarps;
   const int64_t r0 = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x;
@@ -93,10 +118,10 @@ __global__ void __launch_bounds__(kTqWarps * 32)
   load_sign_masks(signs, masks);
   if (threadIdx.x < kTqLevels - 1) bnd[threadIdx.x] = __ldg(boundaries + threadIdx.x);
   __syncthreads();
+  // (the codebook is odd-symmetric: boundary 7 is 0, boundaries 8..14 positive)
+  const float inv_w = fill_cells(bnd, cells);
+  __syncthreads();
   const uint32_t smask = masks[lane];
-  float pb[7];  // the positive boundaries (the codebook is odd-symmetric; boundary 7 is 0)
-#pragma unroll
-  for (int k = 0; k < 7; ++k) pb[k] = bnd[8 + k];
   int64_t i = 0;
   for (int64_t row = r0; row < n; row += G, ++i) {
     const int s = static_cast<int>(i % S::NS);
@@ -124,17 +149,21 @@ __global__ void __launch_bounds__(kTqWarps * 32)
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float gamma = sqrtf(sum);
     if (lane == 0) norms[row] = gamma;
-    // y_j > t_k  <=>  (H diag(s) theta)_j > t_k * gamma * sqrt(d)
+    // |y_j| = |(H diag(s) theta)_j| / (gamma sqrt(d)), in cell units t = |y_j| / w
     const float g = gamma * kTqSqrtD;
-    float p[7];
-#pragma unroll
-    for (int k = 0; k < 7; ++k) p[k] = pb[k] * g;
+    const float tscale = g > 0.0f ? inv_w / g : 0.0f;
     // codes of elements 32 lane + r: 8 per 32-bit word, element 2i in the low nibble
     uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int r = 0; r < V; ++r) {
-      const float a = fabsf(v[r]);
-      const int m = count_below(a, p);
+      const float t = fabsf(v[r]) * tscale;
+      // 2^23 - 0.5 + t rounds to 2^23 + floor(t) (or one less at an exact
+      // integer, where the cell below gives the same count); entry = that + 1,
+      // clamped (unsigned) into the table for any input
+      const uint32_t j = min(static_cast<uint32_t>(__float_as_int(t + 8388607.5f) - 0x4AFFFFFF),
+                             static_cast<uint32_t>(kTqCells - 1));
+      const float2 cell = cells[j];
+      const int m = __float_as_int(cell.x) + (t > cell.y ? 1 : 0);
       const int code = v[r] > 0.0f ? 8 + m : 7 - m;  // odd symmetry around boundary 7 = 0
       w[r >> 3] |= static_cast<uint32_t>(code) << (4 * (r & 7));
     }
