@@ -195,9 +195,21 @@ __global__ void __launch_bounds__(kTqWarps * 32)
   __syncthreads();
   const uint32_t smask = masks[lane];
   const int64_t G = static_cast<int64_t>(gridDim.x) * kTqWarps;
-  for (int64_t row = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; row < n; row += G) {
-    const uint4 cw = __ldcs(reinterpret_cast<const uint4 *>(codes + row * (kTqD / 2)) + lane);
-    const float gamma = __ldg(norms + row);
+  const int64_t r0 = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x;
+  // the next vector's codes and norm are loaded while this one is transformed
+  uint4 cw_next = make_uint4(0u, 0u, 0u, 0u);
+  float gamma_next = 0.0f;
+  if (r0 < n) {
+    cw_next = __ldcs(reinterpret_cast<const uint4 *>(codes + r0 * (kTqD / 2)) + lane);
+    gamma_next = __ldg(norms + r0);
+  }
+  for (int64_t row = r0; row < n; row += G) {
+    const uint4 cw = cw_next;
+    const float gamma = gamma_next;
+    if (row + G < n) {
+      cw_next = __ldcs(reinterpret_cast<const uint4 *>(codes + (row + G) * (kTqD / 2)) + lane);
+      gamma_next = __ldg(norms + row + G);
+    }
     const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
     float v[32], u[32];
 #pragma unroll
