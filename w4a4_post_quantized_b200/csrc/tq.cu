@@ -135,15 +135,17 @@ __global__ void __launch_bounds__(kTqWarps * 32)
       u[j] = __uint_as_float(__float_as_uint(xv) ^ (((smask >> j) & 1u) << 31));  // diag(s) theta
       ss[j & 3] = fmaf(xv, xv, ss[j & 3]);
     }
-    transform_row<kTqD, true>(u, lane, tile, v);  // H diag(s) theta; ends with __syncwarp
-    if (lane == 0) {  // slot s is no longer read: the vector after next may land there
+    __syncwarp();  // every lane has read slot s: the vector after next may land there
+    if (lane == 0) {
       const int64_t rn = row + S::NS * G;
       if (rn < n) {
+        fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[s], S::ROWB);
         bulk_load(ring + s * S::ROWB, X + rn * kTqD, S::ROWB, &bars[s]);
         ++issued;
       }
     }
+    transform_row<kTqD, true>(u, lane, tile, v);  // H diag(s) theta
     float sum = (ss[0] + ss[1]) + (ss[2] + ss[3]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
