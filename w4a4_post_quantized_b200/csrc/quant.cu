@@ -339,29 +339,30 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         ++issued;
       }
     }
-    float u[V], v[V];
+    float u[V];
     load_phase1<K, GELU, true>(reinterpret_cast<const unsigned short *>(ring + s * S::ROWB), lane, u);
-    if constexpr (S::NS == 1) {
-      __syncwarp();  // every lane has read the slot: the next row may land there
+    // slot s is refilled with the row NS rounds ahead as soon as every lane has
+    // read it (one slot; GELU rows, whose long compute covers the copy), or
+    // after the transform (K = 4096 without GELU, measured 2 % faster so)
+    constexpr bool kEarly = S::NS == 1 || GELU;
+    auto refill = [&]() {
       if (lane == 0) {
-        const int64_t rn = row + G;
+        const int64_t rn = row + S::NS * G;
         if (rn < M) {
           fence_proxy_async_smem();
-          mbar_arrive_expect_tx(&bars[0], S::ROWB);
-          bulk_load(ring, X + rn * K, S::ROWB, &bars[0]);
+          mbar_arrive_expect_tx(&bars[s], S::ROWB);
+          bulk_load(ring + s * S::ROWB, X + rn * K, S::ROWB, &bars[s]);
           ++issued;
         }
       }
+    };
+    if (kEarly) {
+      __syncwarp();
+      refill();
     }
+    float v[V];
     transform_row<K, ROT>(u, lane, tile, v);  // ends with __syncwarp: slot s is no longer read
-    if (S::NS == 2 && lane == 0) {
-      const int64_t rn = row + S::NS * G;
-      if (rn < M) {
-        mbar_arrive_expect_tx(&bars[s], S::ROWB);
-        bulk_load(ring + s * S::ROWB, X + rn * K, S::ROWB, &bars[s]);
-        ++issued;
-      }
-    }
+    if (!kEarly) refill();
     quantize_store_row<K, ROT, CODE>(v, lane, row, mtab, q, scale);
   }
   // after a timed-out wait, let the copies still in flight land before exiting
