@@ -14,7 +14,8 @@
 //     smoothing factors are computed from).
 //   * smooth_factors, bias conversion, fill: small offline helpers.
 //
-// Row layout (one warp per row of K = 32*V values):
+// Row layout (one warp per row of K = 32*V values; the transform routine,
+// transform_row, is in fwht.cuh):
 //   phase 1: lane l holds x[l + 32 j], j < V: 16-bit loads, every warp-wide
 //            load instruction covers 64 contiguous bytes.  The butterflies over
 //            the bits of j (index bits 5 .. log2 K - 1) run in registers.
@@ -26,8 +27,8 @@
 //            16-byte store takes four consecutive slots.
 //   phase 2: lane l holds x[V l + r], r < V: the butterflies over index bits
 //            0..4 run in registers; each lane then owns V consecutive outputs,
-//            i.e. V/2 consecutive bytes of packed codes, stored with 16-byte
-//            stores.
+//            i.e. V/2 (packed) or V (one per byte) consecutive code bytes,
+//            stored with 16-byte stores.
 // Packed fp32x2 instructions do two butterflies, products or fused
 // multiply-adds at once; adjacent register slots (2m, 2m + 1) form the pairs.
 // The transform is the Sylvester (natural-order) Hadamard product x H, scaled
