@@ -68,6 +68,22 @@ def test_gemm_s32_int8_bit_exact(w4, M, N, K):
     assert np.array_equal(acc.astype(np.int64), oracle.int_gemm(A, B))
 
 
+def test_gemm_s32_int8_many_tiles_per_cta(w4):
+    """Byte-operand GEMM with several tiles per CTA: M = 8229 (65 row blocks,
+    the last one ragged) x N = 3072 is 780 tiles of 128 x 256, 5-6 per
+    persistent CTA, so every CTA cycles both accumulator buffers and the TMA
+    ring several times; rows sampled from every row block, all columns,
+    bit-exact against the oracle's int64 GEMM."""
+    M, N, K = 8229, 3072, 1024
+    rng = np.random.default_rng(77)
+    A = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    B = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    acc = host(w4.w4a4_gemm_s32(dev(A.view(np.uint8)), _raw_int8_weights(w4, B)))
+    rows = np.unique(np.concatenate([np.arange(0, M, 53), np.arange(M - 40, M)]))
+    assert np.array_equal(acc[rows].astype(np.int64), oracle.int_gemm(A[rows], B))
+    assert w4.w4a4_get_device_status() == 0
+
+
 def test_gemm_int8_extreme_accumulators(w4):
     """Every product 127 * +-127 over K = 4096: |acc| = 66 064 384 > 2^24.  The
     s32 path is exact; the bf16 path converts with one rounding (relative
