@@ -599,6 +599,33 @@ def run_stack(args, st, world, rank, local):
         t = per[name] / st["blocks"]
         per_layer[name] = {"K": K, "N": N, "ms_per_layer": t,
                            "tops": 2.0 * M * N * K / (t * 1e-3) / 1e12}
+    # each kernel alone, per layer shape (block 0's weights and the step's
+    # inputs): the quantize kernel (codes one per byte, the fused call's route)
+    # and the GEMM, n_iso back-to-back launches each between CUDA events
+    n_iso = 10
+    for i, (b, name, K, N) in enumerate(layers[:len(st["layers"])]):
+        x = Ys["fc1"] if name == "fc2" else Xp[b % 2]
+        fl = (w4a4.W4A4_FLAG_GELU if name == "fc2" else 0) | w4a4.W4A4_FLAG_UNPACKED
+        q, sq = w4a4.w4a4_quantize_act(x, pws[i].inv_smooth, fl)
+        Yk = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        times = []
+        for fn in (lambda: w4a4.w4a4_quantize_act(x, pws[i].inv_smooth, fl, qx=q, scale_tok=sq),
+                   lambda: w4a4.w4a4_linear_ex(q, sq, pws[i], flags=w4a4.W4A4_FLAG_UNPACKED, Y=Yk)):
+            fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n_iso):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(max_over_ranks(world, e0.elapsed_time(e1)) / n_iso)
+        tq_ms, tg_ms = times
+        gtops = 2.0 * M * N * K / (tg_ms * 1e-3) / 1e12
+        per_layer[name].update({
+            "quantize_us": tq_ms * 1e3, "quantize_gbs": (2.5 * M * K + 4 * M) / (tq_ms * 1e-3) / 1e9,
+            "gemm_us": tg_ms * 1e3, "gemm_tops": gtops, "gemm_frac": gtops / int8_peak})
+        del q, sq, Yk
     # end to end: the first layer's input from pinned host memory, the last
     # layer's output back, around one whole step
     Xh = torch.empty((M, 1024), dtype=torch.bfloat16, pin_memory=True)
@@ -634,7 +661,9 @@ def run_stack(args, st, world, rank, local):
         "per_layer": per_layer,
         "roofline": {"bound": "tensor", "kernel": "w4a4_gemm_kernel + quantize_rows_kernel (whole stack)",
                      "achieved": value / world, "peak": int8_peak, "unit": "TOPS",
-                     "frac": value / world / int8_peak, "traffic": None},
+                     "frac": value / world / int8_peak, "traffic": None,
+                     "per_layer_kernels": "per_layer.*.gemm_frac: the GEMM alone per layer shape "
+                                          f"({n_iso} back-to-back launches, int8 peak = 2 x measured bf16 burst)"},
         "device_status": status,
     }
     if rank == 0:
