@@ -7,9 +7,9 @@
 // 4-bit codes; section 细粒度量化粒度 read as per-token x per-channel steps).
 // tcgen05 has no 4-bit integer MMA, so the int4 codes are widened to 8 bits
 // and multiplied with tcgen05.mma kind::i8 (s32 accumulators in tensor
-// memory).  Two ways of feeding B (the weights):
+// memory).  Three ways of feeding the operands:
 //
-//   * expanded B (default, when the prepared weights carry qw8): the weights
+//   * expanded B (packed activation codes, weights that carry qw8): the weights
 //     are static, so their int4 codes are widened once, at preparation time,
 //     into qw8 [N, K] int8 in exactly the order the kernel widens A.  The
 //     kernel TMA-loads B tiles straight into the 128-byte swizzled operand
@@ -26,11 +26,12 @@
 //   * packed B (qw8 == NULL): both operands are TMA-staged packed and
 //     sign-extended to int8 in shared memory on every tile (no extra weight
 //     memory, more shared-memory traffic and integer work); tiles 128 x 256.
-//   * int8 (the W8A8 setting): activations and weights carry one 8-bit code
-//     per byte in natural order; TMA loads both straight into the 128-byte
-//     swizzled operand layout and the MMA reads them there (signed x signed).
-//     No widening at all, so comparing it with the expanded path isolates
-//     what the 4-bit codes cost; tiles 128 x 256.
+//   * bytes (a8): activations and weights carry one code per byte in the
+//     same order: the int4 codes the quantize kernel writes one per byte in
+//     qw8's operand order (the fused call's default route), or the W8A8
+//     setting's 8-bit codes in natural order.  TMA loads both straight into
+//     the 128-byte swizzled operand layout and the MMA reads them there
+//     (signed x signed); no widening at all; tiles 128 x 256.
 //
 // Warp roles (one persistent CTA per SM, tiles round-robin, M-major):
 //   warp 0      TMA producer (one thread)
