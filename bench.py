@@ -49,9 +49,9 @@ WORKLOADS = {
                    desc="VGGT MLP fc2 (GELU on input), 8 frames: M=10992, K=4096, N=1024", gelu=True),
 }
 # Multi-layer workloads: the four linears of a transformer block (fc2 takes
-# fc1's output through GELU, folded into its quantize kernel; the other
-# layers take synthetic activations, since attention and normalisation sit
-# between them), repeated over `blocks` blocks with fresh weights per layer.
+# fc1's output through GELU, applied by fc1's GEMM epilogue; the other layers
+# take synthetic activations, since attention and normalisation sit between
+# them), repeated over `blocks` blocks with fresh weights per layer.
 STACKS = {
     "c3_mlp_pair": dict(frames=8, blocks=1, layers=[("fc1", 1024, 4096), ("fc2", 4096, 1024)],
                         desc="VGGT MLP pair, 8 frames: fc1 1024->4096, GELU, fc2 4096->1024, M=10992"),
@@ -555,10 +555,12 @@ def run_stack(args, st, world, rank, local):
     torch.cuda.synchronize()
     ops_step = sum(2.0 * M * N * K for (_, _, K, N) in layers)
 
+    # the MLP's GELU is applied by fc1's GEMM epilogue to its output (the same
+    # bf16 values as applying it in fc2's quantize kernel to its input)
     def run_layer(i, b, name, K, N):
         x = Ys["fc1"] if name == "fc2" else Xp[b % 2]
         w4a4.w4a4_linear_fused(x, pws[i], Y=Ys[name], workspace=ws,
-                               flags=w4a4.W4A4_FLAG_GELU if name == "fc2" else 0)
+                               flags=w4a4.W4A4_FLAG_GELU_OUT if name == "fc1" else 0)
 
     def step():
         for i, (b, name, K, N) in enumerate(layers):
@@ -605,12 +607,13 @@ def run_stack(args, st, world, rank, local):
     n_iso = 10
     for i, (b, name, K, N) in enumerate(layers[:len(st["layers"])]):
         x = Ys["fc1"] if name == "fc2" else Xp[b % 2]
-        fl = (w4a4.W4A4_FLAG_GELU if name == "fc2" else 0) | w4a4.W4A4_FLAG_UNPACKED
+        fl = w4a4.W4A4_FLAG_UNPACKED
+        gfl = fl | (w4a4.W4A4_FLAG_GELU_OUT if name == "fc1" else 0)
         q, sq = w4a4.w4a4_quantize_act(x, pws[i].inv_smooth, fl)
         Yk = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         times = []
         for fn in (lambda: w4a4.w4a4_quantize_act(x, pws[i].inv_smooth, fl, qx=q, scale_tok=sq),
-                   lambda: w4a4.w4a4_linear_ex(q, sq, pws[i], flags=w4a4.W4A4_FLAG_UNPACKED, Y=Yk)):
+                   lambda: w4a4.w4a4_linear_ex(q, sq, pws[i], flags=gfl, Y=Yk)):
             fn()
             torch.cuda.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

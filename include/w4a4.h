@@ -99,6 +99,15 @@ typedef enum {
                                  no widening in the GEMM (which otherwise widens
                                  every activation tile once per output tile).
                                  Not with W4A4_FLAG_INT8. */
+#define W4A4_FLAG_GELU_OUT 0x10u  /* linear_ex / linear_fused: Y = bf16(GELU(y)) of
+                                 the bf16-rounded output y, the same exact-erf GELU
+                                 as W4A4_FLAG_GELU, applied by the GEMM epilogue
+                                 to the output of an MLP's first linear instead of
+                                 by the quantize kernel to the input of its second
+                                 (both give the same bf16 values: the MLP block of
+                                 page "十亿参数的三维重建模型，能塞进手机吗？",
+                                 section 视觉几何基础 Transformer（VGGT）, with its
+                                 activation placed where it costs least). */
 
 /* Prepared weights of one linear layer.  The caller allocates every array
  * (device memory) with the sizes given and keeps ownership. */
@@ -181,8 +190,8 @@ w4a4_status w4a4_linear(const uint8_t *qx, const float *scale_tok, int64_t M,
 /* w4a4_linear with the code layout of qx given by flags: 0 (as w4a4_linear)
  * or W4A4_FLAG_UNPACKED for 4-bit weights that carry qw8 (then qx [M, K] holds
  * the int4 codes one per byte in operand order, as w4a4_quantize_act writes
- * them with that flag; W4A4_ERR_ARG without qw8).  Other flags:
- * W4A4_ERR_UNSUPPORTED. */
+ * them with that flag; W4A4_ERR_ARG without qw8); W4A4_FLAG_GELU_OUT may be
+ * added (the GELU on the output).  Other flags: W4A4_ERR_UNSUPPORTED. */
 w4a4_status w4a4_linear_ex(const uint8_t *qx, const float *scale_tok, int64_t M,
                            const w4a4_weights_t *w, uint16_t *Y, uint32_t flags, void *stream);
 
@@ -195,8 +204,9 @@ w4a4_status w4a4_linear_ex(const uint8_t *qx, const float *scale_tok, int64_t M,
  * reads them without widening; otherwise they are packed two per byte.  The
  * workspace afterwards holds those codes, then (at the next 256-byte boundary)
  * the steps.  flags must carry the same W4A4_FLAG_PLAIN and W4A4_FLAG_INT8
- * bits as w->flags (W4A4_ERR_ARG otherwise); W4A4_FLAG_UNPACKED is not a flag
- * of this call (W4A4_ERR_UNSUPPORTED). */
+ * bits as w->flags (W4A4_ERR_ARG otherwise); W4A4_FLAG_GELU applies the GELU
+ * to X, W4A4_FLAG_GELU_OUT to Y (both may be given); W4A4_FLAG_UNPACKED is not
+ * a flag of this call (W4A4_ERR_UNSUPPORTED). */
 w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t *w, uint16_t *Y,
                               void *workspace, size_t workspace_bytes, uint32_t flags,
                               void *stream);

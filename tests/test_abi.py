@@ -159,6 +159,24 @@ def test_unpacked_codes_argument_checks(lib):
     assert F(A, 100, ctypes.byref(w), A, A, lib.w4a4_workspace_bytes_min(100, 1024, 0) - 1, 0, None) == 2
 
 
+def test_gelu_out_argument_checks(lib):
+    """W4A4_FLAG_GELU_OUT (0x10): the GELU on a linear's output; a flag of
+    linear_ex and linear_fused, not of the activation quantizer; the workspace
+    sizes do not depend on it."""
+    _setup(lib)
+    q, LX, F = lib.w4a4_quantize_act, lib.w4a4_linear_ex, lib.w4a4_linear_fused
+    GOUT = 0x10
+    assert q(A, 10, 1024, A, A, A, GOUT, None) == 4
+    w = _weights()
+    assert LX(A, A, 0, ctypes.byref(w), A, GOUT, None) == 0
+    assert LX(A, A, 0, ctypes.byref(w), A, GOUT | UNPACKED, None) == 0
+    assert LX(A, A, 10, ctypes.byref(w), A, GOUT | 0x20, None) == 4
+    assert F(A, 0, ctypes.byref(w), A, A, 0, GOUT | 0x1, None) == 0          # with the input GELU too
+    assert F(A, 100, ctypes.byref(w), A, A, 16, GOUT, None) == 2              # workspace too small
+    for K in (1024, 4096):
+        assert lib.w4a4_workspace_bytes_min(100, K, GOUT) == lib.w4a4_workspace_bytes_min(100, K, 0)
+
+
 def test_quantize_act_argument_checks(lib):
     _setup(lib)
     q = lib.w4a4_quantize_act

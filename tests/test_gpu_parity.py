@@ -307,3 +307,41 @@ def test_unpacked_route_matches_packed_route(w4, M, N, K):
     assert torch.equal(Yf_small.view(torch.int16), Yp.view(torch.int16))
     assert torch.equal(Yf_full.view(torch.int16), Yp.view(torch.int16))
     assert w4.w4a4_get_device_status() == 0
+
+
+# ------------------------------------------------- GELU on the output (W4A4_FLAG_GELU_OUT)
+GELU_OUT = 0x10
+
+
+@pytest.mark.parametrize("route", ["fused", "bytes", "expanded", "packed"])
+def test_gelu_on_output(w4, route):
+    """W4A4_FLAG_GELU_OUT gives, element by element, the oracle's GELU (exact
+    erf in fp64, rounded to bf16) of the same call's output without the flag,
+    on an fc1-shaped layer (K = 1024, N = 4096), through every GEMM route.
+    Below -5.9 the kernel's GELU returns -0 (or the exact value): the exact
+    GELU there is below 1e-8 of the input in magnitude."""
+    M, N, K = 300, 4096, 1024
+    X = synth.activations(M, K, seed=820)
+    W, b = synth.weights(N, K, seed=821), synth.bias(N, seed=822)
+    pw = w4.w4a4_prepare_weights(bf16_dev(W), bf16_dev(b), bf16_dev(X[:synth.calibration_rows(M)]),
+                                 expanded=(route != "packed"))
+    Xd = bf16_dev(X)
+    if route == "fused":
+        Y0 = w4.w4a4_linear_fused(Xd, pw)
+        Y1 = w4.w4a4_linear_fused(Xd, pw, flags=GELU_OUT)
+    else:
+        fl = UNPACKED if route == "bytes" else 0
+        q, s = w4.w4a4_quantize_act(Xd, pw.inv_smooth, fl)
+        Y0 = w4.w4a4_linear_ex(q, s, pw, flags=fl)
+        Y1 = w4.w4a4_linear_ex(q, s, pw, flags=fl | GELU_OUT)
+    y0 = host(Y0.view(torch.int16)).view(np.uint16)
+    y1 = host(Y1.view(torch.int16)).view(np.uint16)
+    want = oracle.gelu_bf16(y0)
+    f0 = synth.bf16_bits_to_f32(y0).astype(np.float64)
+    far = f0 < -5.9
+    assert far.sum() > 0 and (~far).sum() > 0.9 * f0.size   # both branches exercised
+    assert np.array_equal(y1[~far], want[~far])
+    f1 = synth.bf16_bits_to_f32(y1[far]).astype(np.float64)
+    assert np.all((y1[far] == 0x8000) | (y1[far] == want[far]))
+    assert np.all(np.abs(f1) <= 1e-8 * np.abs(f0[far]))
+    assert w4.w4a4_get_device_status() == 0

@@ -11,7 +11,10 @@
 
 namespace {
 
-constexpr uint32_t kKnownFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED;
+constexpr uint32_t kKnownFlags =
+    W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED | W4A4_FLAG_GELU_OUT;
+// flags of the activation quantizer (w4a4_quantize_act and the workspace sizes)
+constexpr uint32_t kActFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED;
 constexpr uint32_t kWeightFlags = W4A4_FLAG_PLAIN | W4A4_FLAG_INT8;  // fixed at preparation
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -57,7 +60,7 @@ w4a4::CodeFormat code_format(uint32_t flags) {
 
 w4a4_status check_act(const void *X, int64_t M, int32_t K, const float *inv_smooth, const void *qx,
                       const float *scale_tok, uint32_t flags) {
-  if (flags & ~kKnownFlags) return W4A4_ERR_UNSUPPORTED;
+  if (flags & ~kActFlags) return W4A4_ERR_UNSUPPORTED;
   if (!k_ok(K)) return W4A4_ERR_UNSUPPORTED;
   if (!m_ok(M)) return W4A4_ERR_SHAPE;
   if (M == 0) return W4A4_OK;
@@ -158,7 +161,7 @@ w4a4_status w4a4_linear_ex(const uint8_t *qx, const float *scale_tok, int64_t M,
                            const w4a4_weights_t *w, uint16_t *Y, uint32_t flags, void *stream) {
   w4a4_status s = check_weights(w);
   if (s != W4A4_OK) return s;
-  if (flags & ~W4A4_FLAG_UNPACKED) return W4A4_ERR_UNSUPPORTED;
+  if (flags & ~(W4A4_FLAG_UNPACKED | W4A4_FLAG_GELU_OUT)) return W4A4_ERR_UNSUPPORTED;
   // one-per-byte 4-bit codes pair with the expanded weight codes
   if ((flags & W4A4_FLAG_UNPACKED) && (int8_weights(w) || !w->qw8)) return W4A4_ERR_ARG;
   if (!m_ok(M)) return W4A4_ERR_SHAPE;
@@ -166,7 +169,8 @@ w4a4_status w4a4_linear_ex(const uint8_t *qx, const float *scale_tok, int64_t M,
   if (!qx || !scale_tok || !Y) return W4A4_ERR_ARG;
   if (!aligned16(qx) || !aligned16(scale_tok) || !aligned16(Y)) return W4A4_ERR_ALIGN;
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, scale_tok, w->scale_ch, w->bias, Y, nullptr,
-                   M, w->N, w->K, int8_weights(w) || (flags & W4A4_FLAG_UNPACKED) != 0};
+                   M, w->N, w->K, int8_weights(w) || (flags & W4A4_FLAG_UNPACKED) != 0,
+                   (flags & W4A4_FLAG_GELU_OUT) != 0};
   return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
 }
 
@@ -203,7 +207,7 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
                                              (flags & W4A4_FLAG_GELU) != 0, code_format(cf), cs);
   if (e != cudaSuccess) return cuda_status(e);
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, st, w->scale_ch, w->bias, Y, nullptr,
-                   M, w->N, w->K, one_per_byte(cf)};
+                   M, w->N, w->K, one_per_byte(cf), (flags & W4A4_FLAG_GELU_OUT) != 0};
   return cuda_status(w4a4::launch_gemm(a, cs));
 }
 

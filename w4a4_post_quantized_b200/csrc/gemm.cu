@@ -66,6 +66,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "gelu.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -234,7 +235,14 @@ __device__ __forceinline__ uint32_t dequant2_bf16_cvt(int32_t a0, int32_t a1, fl
   return pack_bf16x2(y0, y1);
 }
 
-template <int MODE, bool OUT_S32>
+// GELU of the two bf16 values of a packed pair (bf16 in, bf16 out).
+__device__ __forceinline__ uint32_t gelu_pair_bf16(uint32_t w) {
+  float a = __uint_as_float(w << 16), b = __uint_as_float(w & 0xFFFF0000u);
+  gelu2_bf16(a, b);
+  return (__float_as_uint(b) & 0xFFFF0000u) | (__float_as_uint(a) >> 16);
+}
+
+template <int MODE, bool OUT_S32, bool GELU_OUT = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmY, const float *__restrict__ scale_tok,
@@ -273,7 +281,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], NUM_EPI_WARPS);
+      mbar_init(&acc_empty[b], (GELU_OUT && P::A8 ? 2 : 1) * NUM_EPI_WARPS);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -478,9 +486,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (warp >= W_EPI0) {
+  } else if (warp >= W_EPI0 || (GELU_OUT && P::A8 && warp >= W_UNPACK0 && warp < W_UNPACK0 + 4)) {
     // ---------------------------------------------------------------- epilogue
-    const int ew = warp - W_EPI0;  // == warp % 4: owns TMEM lanes 32 ew .. 32 ew + 31
+    const int ew = warp & 3;  // owns TMEM lanes 32 ew .. 32 ew + 31
+    // With the GELU on the output (the epilogue's ALU work then exceeds the
+    // main loop's time) the byte-operand mode's idle warps 4..7 join in: the
+    // two warps of a lane quadrant take half of the tile's columns each, with
+    // one staging buffer each.
+    constexpr bool EPI8 = GELU_OUT && P::A8;
+    const int half = (EPI8 && warp < W_EPI0) ? 1 : 0;
+    constexpr int SC_PER = EPI8 ? P::TN / EPI_COLS / 2 : P::TN / EPI_COLS;
     // this warp's copy of the tile's per-column constants:
     //   off[n] = 0x4B400000 - 8 colsum[n] (the code-offset correction folded
     //   into the exact int -> float bias), sc[n], bias[n]
@@ -521,12 +536,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + b * TN;
 #pragma unroll 1
-        for (int sc = 0; sc < TN / EPI_COLS; ++sc) {
+        for (int sc = half * SC_PER; sc < (half + 1) * SC_PER; ++sc) {
           uint32_t r[2][32];  // [16-row half][4 j + k]
           tmem_ld_16x256b_x8(tbase + sc * EPI_COLS, r[0]);
           tmem_ld_16x256b_x8(tbase + (16u << 16) + sc * EPI_COLS, r[1]);
           tmem_wait_ld();
-          if (sc == TN / EPI_COLS - 1) {
+          if (sc == (half + 1) * SC_PER - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
@@ -559,8 +574,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                           static_cast<int32_t>(r[h][4 * j + 2 * u + 1]) + o.y,
                                           st4[2 * h + u], scl.x, scl.y, bi.x, bi.y);
           }
-          uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (sc & 1)) * EPI_BYTES;
-          if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
+          if constexpr (GELU_OUT) {
+            // the MLP's activation on the rounded output (bf16 in, bf16 out)
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) pk[h][u][j] = gelu_pair_bf16(pk[h][u][j]);
+          }
+          uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (EPI8 ? half : (sc & 1))) * EPI_BYTES;
+          if (lane == 0) {  // the store that last read this buffer is done
+            if constexpr (EPI8)
+              bulk_wait_read<0>();
+            else
+              bulk_wait_read<1>();
+          }
           __syncwarp();
           // staging tile: 32 rows of 128 bytes, 16-byte chunk k of row R at k ^ (R % 8);
           // stmatrix x4 #(h, jp): matrices (u, j) = (0, 2jp), (1, 2jp), (0, 2jp+1), (1, 2jp+1)
@@ -627,6 +656,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             pk[2 * c + 1] = dequant2_bf16(static_cast<int32_t>(r[4 * c + 2]) + o.z,
                                           static_cast<int32_t>(r[4 * c + 3]) + o.w, st, scl.z, scl.w,
                                           bi.z, bi.w);
+          }
+          if constexpr (GELU_OUT) {
+#pragma unroll
+            for (int c = 0; c < EPI_COLS / 2; ++c) pk[c] = gelu_pair_bf16(pk[c]);
           }
           uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (sc & 1)) * EPI_BYTES;
           if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
@@ -711,10 +744,10 @@ bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, bool OUT_S32>
+template <int MODE, bool OUT_S32, bool GELU_OUT = false>
 cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   using P = Plan<MODE>;
-  auto kern = w4a4_gemm_kernel<MODE, OUT_S32>;
+  auto kern = w4a4_gemm_kernel<MODE, OUT_S32, GELU_OUT>;
   static bool attr_set[64] = {};  // per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -770,6 +803,11 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
 
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st) {
   if (a.M <= 0) return cudaSuccess;
+  if (a.gelu_out) {
+    if (a.acc) return cudaErrorInvalidValue;
+    if (a.a8) return launch_t<kInt8, false, true>(a, st);
+    return a.qw8 ? launch_t<kExpanded, false, true>(a, st) : launch_t<kPacked, false, true>(a, st);
+  }
   if (a.a8) return a.acc ? launch_t<kInt8, true>(a, st) : launch_t<kInt8, false>(a, st);
   const bool packed = (a.qw8 == nullptr);
   if (a.acc) return packed ? launch_t<kPacked, true>(a, st) : launch_t<kExpanded, true>(a, st);

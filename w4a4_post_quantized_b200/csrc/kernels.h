@@ -40,6 +40,7 @@ struct GemmArgs {
   int N, K;
   bool a8;                  // qx and qw8 hold one code per byte in the same order (int8 codes,
                             // or int4 codes in operand order): no widening
+  bool gelu_out = false;    // y = bf16(GELU(bf16 result)) (an MLP's first linear)
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,

@@ -1,5 +1,6 @@
-"""Coefficients of the GELU the quantize kernel evaluates (csrc/quant.cu,
-gelu2_bf16), and a check of how its bf16 results compare with the exact GELU.
+"""Coefficients of the GELU the kernels evaluate (csrc/gelu.cuh, gelu2_bf16:
+the quantize kernel on an MLP's fc2 input, or the GEMM epilogue on its fc1
+output), and a check of how its bf16 results compare with the exact GELU.
 
 The kernel computes Phi(-|x|) = erfc(z) / 2, z = |x| / sqrt 2, as
 exp2(log2(e) (-z^2) + c(u)) with u = z / (Z/2) - 1 on 0 <= z <= Z = 4.2

@@ -29,6 +29,7 @@ W4A4_FLAG_GELU = 0x1
 W4A4_FLAG_PLAIN = 0x2
 W4A4_FLAG_INT8 = 0x4
 W4A4_FLAG_UNPACKED = 0x8
+W4A4_FLAG_GELU_OUT = 0x10
 
 _vp, _i32, _i64, _u32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
                                     ctypes.c_float, ctypes.c_size_t)
