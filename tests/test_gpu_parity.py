@@ -345,3 +345,24 @@ def test_gelu_on_output(w4, route):
     assert np.all((y1[far] == 0x8000) | (y1[far] == want[far]))
     assert np.all(np.abs(f1) <= 1e-8 * np.abs(f0[far]))
     assert w4.w4a4_get_device_status() == 0
+
+
+def test_mlp_gelu_placements_agree(w4):
+    """An MLP pair (fc1 1024 -> 4096, GELU, fc2 4096 -> 1024): the GELU in
+    fc1's epilogue (W4A4_FLAG_GELU_OUT) or in fc2's quantize kernel
+    (W4A4_FLAG_GELU) gives the same fc2 output bits, since both apply the same
+    function to the same bf16 values."""
+    M = 700
+    X = synth.activations(M, 1024, seed=830)
+    W1, b1 = synth.weights(4096, 1024, seed=831), synth.bias(4096, seed=832)
+    W2, b2 = synth.weights(1024, 4096, seed=833), synth.bias(1024, seed=834)
+    C = synth.calibration_rows(M)
+    Xd = bf16_dev(X)
+    pw1 = w4.w4a4_prepare_weights(bf16_dev(W1), bf16_dev(b1), bf16_dev(X[:C]))
+    Y1 = w4.w4a4_linear_fused(Xd, pw1)
+    G1 = w4.w4a4_linear_fused(Xd, pw1, flags=GELU_OUT)
+    pw2 = w4.w4a4_prepare_weights(bf16_dev(W2), bf16_dev(b2), G1[:C].contiguous())
+    Ya = w4.w4a4_linear_fused(Y1, pw2, flags=w4.W4A4_FLAG_GELU)
+    Yb = w4.w4a4_linear_fused(G1, pw2)
+    assert torch.equal(Ya.view(torch.int16), Yb.view(torch.int16))
+    assert w4.w4a4_get_device_status() == 0
