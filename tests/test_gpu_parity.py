@@ -313,22 +313,24 @@ def test_unpacked_route_matches_packed_route(w4, M, N, K):
 GELU_OUT = 0x10
 
 
-@pytest.mark.parametrize("route", ["fused", "bytes", "expanded", "packed"])
+@pytest.mark.parametrize("route", ["fused", "bytes", "expanded", "packed", "w8a8"])
 def test_gelu_on_output(w4, route):
     """W4A4_FLAG_GELU_OUT gives, element by element, the oracle's GELU (exact
     erf in fp64, rounded to bf16) of the same call's output without the flag,
-    on an fc1-shaped layer (K = 1024, N = 4096), through every GEMM route.
+    on an fc1-shaped layer (K = 1024, N = 4096), through every GEMM route and
+    the W8A8 setting.
     Below -5.9 the kernel's GELU returns -0 (or the exact value): the exact
     GELU there is below 1e-8 of the input in magnitude."""
     M, N, K = 300, 4096, 1024
     X = synth.activations(M, K, seed=820)
     W, b = synth.weights(N, K, seed=821), synth.bias(N, seed=822)
+    i8 = w4.W4A4_FLAG_INT8 if route == "w8a8" else 0
     pw = w4.w4a4_prepare_weights(bf16_dev(W), bf16_dev(b), bf16_dev(X[:synth.calibration_rows(M)]),
-                                 expanded=(route != "packed"))
+                                 flags=i8, expanded=(route != "packed"))
     Xd = bf16_dev(X)
-    if route == "fused":
-        Y0 = w4.w4a4_linear_fused(Xd, pw)
-        Y1 = w4.w4a4_linear_fused(Xd, pw, flags=GELU_OUT)
+    if route in ("fused", "w8a8"):
+        Y0 = w4.w4a4_linear_fused(Xd, pw, flags=i8)
+        Y1 = w4.w4a4_linear_fused(Xd, pw, flags=i8 | GELU_OUT)
     else:
         fl = UNPACKED if route == "bytes" else 0
         q, s = w4.w4a4_quantize_act(Xd, pw.inv_smooth, fl)
