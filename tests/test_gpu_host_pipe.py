@@ -22,12 +22,14 @@ def bf16(bits, device):
 
 
 @pytest.mark.parametrize("M,N,K,chunk,gelu", [(10992, 3072, 1024, 2816, False), (1000, 512, 1024, 384, False),
-                                              (100, 256, 4096, 2816, True), (1374, 1024, 1024, 128, False)])
+                                              (100, 256, 4096, 2816, True), (1374, 1024, 1024, 128, False),
+                                              (1000, 4096, 1024, 384, "out")])
 def test_host_pipeline_matches_device_call(w4, M, N, K, chunk, gelu):
     X = synth.activations(M, K, seed=M + K)
     W, b = synth.weights(N, K, seed=5), synth.bias(N, seed=6)
     pw = w4.w4a4_prepare_weights(bf16(W, "cuda"), bf16(b, "cuda"), bf16(X[:synth.calibration_rows(M)], "cuda"))
-    flags = w4.W4A4_FLAG_GELU if gelu else 0
+    # gelu: on the input (True), on the output ("out", an MLP's fc1), or none
+    flags = {False: 0, True: w4.W4A4_FLAG_GELU, "out": w4.W4A4_FLAG_GELU_OUT}[gelu]
     want = w4.w4a4_linear_fused(bf16(X, "cuda"), pw, flags=flags).cpu()
     Xh = bf16(X, "cpu").pin_memory()
     pipe = w4.HostPipe()
