@@ -101,17 +101,20 @@ constexpr uint32_t TMEM_COLS = 512;     // the whole tensor memory of the SM
 //   packed B: A and B are widened into a ring of shared-memory slots; tiles
 //     are 128 x 256.
 //   int8: A and B arrive as int8 operand tiles; tiles are 128 x 256, two
-//     256-column accumulators.
-enum : int { kExpanded = 0, kPacked = 1, kInt8 = 2 };
+//     256-column accumulators.  The narrow variant (128 x 128 tiles, 6 stages
+//     of 32 KB) serves shapes whose 128 x 256 tiles would leave more than
+//     half of the SMs idle (a single frame: 44 tiles), doubling the tiles.
+enum : int { kExpanded = 0, kPacked = 1, kInt8 = 2, kInt8Narrow = 3 };
 
 template <int MODE>
 struct Plan {
   static constexpr bool B_PACKED = MODE == kPacked;
   static constexpr bool A_TMEM = MODE == kExpanded;
-  static constexpr bool A8 = MODE == kInt8;
+  static constexpr bool NARROW = MODE == kInt8Narrow;
+  static constexpr bool A8 = MODE == kInt8 || NARROW;  // both operands one code per byte
   static constexpr bool EPI16 = !B_PACKED;           // 16x256b epilogue fragments
-  static constexpr int TN = A_TMEM ? 192 : BN;       // tile columns
-  static constexpr int STAGES = B_PACKED ? 3 : (A8 ? 4 : 5);  // TMA stages
+  static constexpr int TN = A_TMEM ? 192 : (NARROW ? 128 : BN);  // tile columns
+  static constexpr int STAGES = B_PACKED ? 3 : (NARROW ? 6 : (A8 ? 4 : 5));  // TMA stages
   static constexpr int KG = A_TMEM ? 2 : 1;          // k-blocks per widen -> MMA handshake
   static constexpr int WSLOTS = A8 ? 0 : 2;          // widened operand slots
   static constexpr int A_ST = A8 ? A_UN : A_PK;      // A bytes of a stage
@@ -803,11 +806,16 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
 
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st) {
   if (a.M <= 0) return cudaSuccess;
+  // byte operands: 128 x 128 tiles when 128 x 256 ones would fill at most half of the SMs
+  const int64_t wide_tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  const bool narrow = a.a8 && 2 * wide_tiles <= device_sm_count();
   if (a.gelu_out) {
     if (a.acc) return cudaErrorInvalidValue;
-    if (a.a8) return launch_t<kInt8, false, true>(a, st);
+    if (a.a8)
+      return narrow ? launch_t<kInt8Narrow, false, true>(a, st) : launch_t<kInt8, false, true>(a, st);
     return a.qw8 ? launch_t<kExpanded, false, true>(a, st) : launch_t<kPacked, false, true>(a, st);
   }
+  if (narrow) return a.acc ? launch_t<kInt8Narrow, true>(a, st) : launch_t<kInt8Narrow, false>(a, st);
   if (a.a8) return a.acc ? launch_t<kInt8, true>(a, st) : launch_t<kInt8, false>(a, st);
   const bool packed = (a.qw8 == nullptr);
   if (a.acc) return packed ? launch_t<kPacked, true>(a, st) : launch_t<kExpanded, true>(a, st);
