@@ -131,6 +131,33 @@ typedef struct {
                              8-bit codes */
 } w4a4_weights_t;
 
+/* Bytes of one device allocation that holds every array of a prepared layer
+ * [PTQ][GRAN] (what w4a4_weights_bind lays out in it), each array starting at
+ * a 256-byte boundary:
+ *   flags 0:                    qw [N, K/2] packed int4 codes, scale_ch [N],
+ *                               bias [N], smooth [K], inv_smooth [K];
+ *   + W4A4_FLAG_UNPACKED:       also qw8 [N, K] (the codes widened to one per
+ *                               byte in operand order, w4a4_expand_weights) and
+ *                               colsum [N] (the tensor-core GEMM's fast route);
+ *   W4A4_FLAG_INT8:             qw8 [N, K] 8-bit codes, scale_ch, bias, smooth,
+ *                               inv_smooth (no qw, no colsum).
+ * W4A4_FLAG_PLAIN may be given and changes nothing.  About N*K/2 + 12 N + 8 K
+ * bytes for packed int4 weights, against 2 N K + 2 N for bf16 weights and bias.
+ * Returns 0 for an unsupported K, an N that is not a positive multiple of 256,
+ * or another flag. */
+size_t w4a4_weights_bytes(int32_t N, int32_t K, uint32_t flags);
+
+/* Points out's arrays into `base` (device memory of at least
+ * w4a4_weights_bytes(N, K, flags) bytes, 16-byte aligned, owned by the caller)
+ * in the layout w4a4_weights_bytes describes and sets out->N, out->K; pointers
+ * the layout does not use are set to NULL, out->flags to 0.  Reads and writes
+ * no device memory: fill the arrays with w4a4_prepare_weights (same flags
+ * minus W4A4_FLAG_UNPACKED).  W4A4_ERR_ARG for NULL base or out,
+ * W4A4_ERR_ALIGN for a misaligned base, W4A4_ERR_SHAPE when `bytes` is too
+ * small or N, K are not accepted, W4A4_ERR_UNSUPPORTED for another flag. */
+w4a4_status w4a4_weights_bind(void *base, size_t bytes, int32_t N, int32_t K, uint32_t flags,
+                              w4a4_weights_t *out);
+
 /* Bytes of workspace that let w4a4_linear_fused take its fastest route for M
  * tokens of width K, whatever the weights and flags: activation codes one per
  * byte (M*K, rounded up to 256) followed by the per-token steps (4*M).
@@ -231,7 +258,9 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
  *     per byte (the faster route of w4a4_linear_fused).
  *   - The first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept per CUDA context: after
+ *     cudaDeviceReset, or under another context of the same device, the next
+ *     call looks it up again (make that call, too, outside a capture).
  *   - Every call on a device shares the one scratch array, which keeps the
  *     last call's contents: calls that may overlap on the GPU (different
  *     streams without ordering between them) race on it and must not be
@@ -295,6 +324,21 @@ w4a4_status w4a4_linear_fused_host(const uint16_t *X_host, int64_t M, const w4a4
  * exact. */
 w4a4_status w4a4_gemm_s32(const uint8_t *qx, int64_t M, const w4a4_weights_t *w, int32_t *acc,
                           void *stream);
+
+/* Failure-path test of the bounded waits (include/w4a4.h conventions): with
+ * this bit, w4a4_gemm_s32_ex launches the GEMM with its TMA producer issuing
+ * no copy and every bounded wait limited to 1 ms, so the consumers' waits run
+ * out: the kernel sets W4A4_DEV_TIMEOUT in the device status word, drains,
+ * frees its tensor memory and returns, leaving acc undefined.  Not for
+ * computing anything. */
+#define W4A4_DEBUG_STALL 0x80000000u
+
+/* w4a4_gemm_s32 with flags: 0; W4A4_FLAG_UNPACKED (qx [M, K] holds the int4
+ * codes one per byte in operand order, the layout w4a4_quantize_act writes with
+ * that flag; the weights must carry qw8); W4A4_DEBUG_STALL may be added.
+ * Other flags: W4A4_ERR_UNSUPPORTED. */
+w4a4_status w4a4_gemm_s32_ex(const uint8_t *qx, int64_t M, const w4a4_weights_t *w, int32_t *acc,
+                             uint32_t flags, void *stream);
 
 /* Synchronizes `stream`, then copies the device status word (bits
  * W4A4_DEV_*) of the current device into *status.  Returns W4A4_ERR_TIMEOUT

@@ -1,21 +1,35 @@
 """Comparison rules shared by the GPU parity tests.
 
-Integer codes.  Both sides take the rounding decision in binary32 (the
-oracle's decision="f32" quantizer), but the CUDA path reaches its binary32
-values through an fp32 fast Walsh-Hadamard transform while the oracle rounds
-its exact fp64 values once.  Where the exact ratio value/step lies within the
-fp32 error bound of a rounding boundary (x.5), both codes are correct.  So a
-code may differ from the oracle's only
+Integer codes.  The CUDA path forms each rotated value in binary32 (an fp32
+transform of the bf16 inputs), multiplies it by the binary32 reciprocal step
+qmax/absmax and rounds the exact product half to even.  The oracle is compared
+in two modes:
+  * decision="f64" -- the method as the pages define it: exact fp64 rotation,
+    fp64 step absmax/qmax, round(value/step);
+  * decision="f32" -- the same quantizer with the rounding decision taken in
+    binary32 (the oracle's fp64 values rounded to binary32, the binary32
+    reciprocal step).
+Where the exact ratio value/step lies within the GPU's error bound of a
+rounding boundary (x.5), both codes are correct.  So a code may differ from
+the oracle's only
   * by +-1,
   * at an element whose fp64 ratio is within `tie_bound` of a half-integer,
   * on at most 1e-4 of the elements (checked on the large cases).
 Everything else must be bit-exact.
 
-tie_bound: each rotated value is a +-sum of K inputs formed through log2(K)
-rounding levels, so its absolute error is at most log2(K) * u * sum_i |x_i| /
-sqrt(K) (u = 2^-24); the smoothing multiply, the reciprocal step and the
-absmax add a few relative u.  The bound below takes that, times the
-multiplier and 7/absmax, with a factor 4 of margin.
+tie_bound, the bound on |ratio_gpu - ratio_oracle| (u = 2^-24):
+  * the rotated value: a +-sum of K inputs formed through log2(K) rounding
+    levels, so its absolute error is at most e_val = log2(K) u sum_i|x_i| /
+    sqrt(K), times the largest multiplier; in the ratio that is
+    e_ratio = qmax e_val / absmax;
+  * the absmax is one of those values, so it carries the same absolute error
+    e_val; through the reciprocal step it moves every ratio of the row by at
+    most |ratio| e_val / absmax <= e_ratio;
+  * relative roundings: the smoothing multiply (1 u), the binary32 reciprocal
+    (1 u) and, against the fp64 oracle, the binary32 rounding of the value
+    and of the absmax (2 u): at most 4 u |ratio|, plus the 8 u qmax slack kept
+    from the binary32 comparison;
+and the sum is taken with a factor 4 of margin.
 """
 import numpy as np
 
@@ -31,7 +45,8 @@ def tie_bound(x_in: np.ndarray, mult: np.ndarray, ratio: np.ndarray, amax: np.nd
     e_val = np.log2(K) * U * l1 / np.sqrt(K) * np.max(np.abs(mult))
     with np.errstate(divide="ignore", invalid="ignore"):
         e_ratio = np.where(amax > 0, qmax * e_val / amax, 0.0)
-    return 4.0 * (e_ratio + 8 * U * qmax * (1 + np.max(np.abs(ratio), axis=1) / qmax))
+    rmax = np.max(np.abs(ratio), axis=1)
+    return 4.0 * (2.0 * e_ratio + 4 * U * rmax + 8 * U * qmax * (1 + rmax / qmax))
 
 
 def compare_codes(got: np.ndarray, want: np.ndarray, ratio: np.ndarray, bound_row: np.ndarray,

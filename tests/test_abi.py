@@ -313,3 +313,94 @@ def test_tq_codebook_and_argument_checks(lib):
     assert D(A, A, 0, 1024, A, A, A, None) == 0
     assert D(A, None, 10, 1024, A, A, A, None) == 1
     assert D(A, A, 10, 1024, A, A, A + 8, None) == 3
+
+
+def test_weights_layout(lib):
+    """w4a4_weights_bytes / w4a4_weights_bind: one allocation holding every
+    array of a prepared layer, each at a 256-byte boundary, in the order qw,
+    qw8, scale_ch, bias, smooth, inv_smooth, colsum; the arrays the layout
+    leaves out are NULL.  (Sizes from the weight side of the linear: packed
+    int4 codes, per-channel steps and bias, smoothing factors and their
+    reciprocals.)"""
+    vp, i32, u32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t
+    lib.w4a4_weights_bytes.restype = sz
+    lib.w4a4_weights_bytes.argtypes = [i32, i32, u32]
+    lib.w4a4_weights_bind.restype = ctypes.c_int
+    lib.w4a4_weights_bind.argtypes = [vp, sz, i32, i32, u32, ctypes.POINTER(WeightsT)]
+    WB, BIND = lib.w4a4_weights_bytes, lib.w4a4_weights_bind
+    r = lambda b: (b + 255) // 256 * 256
+    for N, K in [(256, 1024), (3072, 1024), (1024, 4096), (4096, 1024)]:
+        packed = r(N * K // 2) + 2 * r(4 * N) + 2 * r(4 * K)
+        assert WB(N, K, 0) == WB(N, K, 2) == packed
+        assert WB(N, K, UNPACKED) == packed + r(N * K) + r(4 * N)
+        assert WB(N, K, INT8) == r(N * K) + 2 * r(4 * N) + 2 * r(4 * K)
+        for flags in (0, UNPACKED, INT8, INT8 | 2):
+            need = WB(N, K, flags)
+            w = WeightsT()
+            assert BIND(A, need, N, K, flags, ctypes.byref(w)) == 0
+            assert (w.N, w.K, w.flags) == (N, K, 0)
+            ptrs = {f: getattr(w, f) for f in ("qw", "qw8", "scale_ch", "bias", "smooth", "inv_smooth",
+                                               "colsum")}
+            size = {"qw": N * K // 2, "qw8": N * K, "scale_ch": 4 * N, "bias": 4 * N, "smooth": 4 * K,
+                    "inv_smooth": 4 * K, "colsum": 4 * N}
+            present = [f for f, p in ptrs.items() if p]
+            want = {0: ["qw", "scale_ch", "bias", "smooth", "inv_smooth"],
+                    UNPACKED: ["qw", "qw8", "scale_ch", "bias", "smooth", "inv_smooth", "colsum"]}
+            want[INT8] = want[INT8 | 2] = ["qw8", "scale_ch", "bias", "smooth", "inv_smooth"]
+            assert present == want[flags]
+            off = A
+            for f in present:                      # consecutive, 256-byte aligned, inside the buffer
+                assert ptrs[f] == off and ptrs[f] % 256 == 0
+                off += r(size[f])
+            assert off == A + need
+            # the bound struct passes the library's own weight checks (M = 0: no launch)
+            w.flags = flags & (INT8 | 2)
+            _setup(lib)
+            assert lib.w4a4_linear(A, A, 0, ctypes.byref(w), A, None) == 0
+    assert WB(1000, 1024, 0) == 0 and WB(256, 2048, 0) == 0 and WB(256, 1024, 0x10) == 0
+    w = WeightsT()
+    assert BIND(A, WB(256, 1024, 0) - 1, 256, 1024, 0, ctypes.byref(w)) == 2   # too small
+    assert BIND(A + 8, 1 << 30, 256, 1024, 0, ctypes.byref(w)) == 3            # misaligned
+    assert BIND(None, 1 << 30, 256, 1024, 0, ctypes.byref(w)) == 1
+    assert BIND(A, 1 << 30, 256, 1024, 0, None) == 1
+    assert BIND(A, 1 << 30, 100, 1024, 0, ctypes.byref(w)) == 2                 # N
+    assert BIND(A, 1 << 30, 256, 1000, 0, ctypes.byref(w)) == 4                 # K
+    assert BIND(A, 1 << 30, 256, 1024, 0x1, ctypes.byref(w)) == 4               # flag
+
+
+STALL = 0x80000000
+
+
+def test_gemm_s32_ex_argument_checks(lib):
+    """w4a4_gemm_s32_ex: flags 0, W4A4_FLAG_UNPACKED (one-per-byte codes, with
+    the expanded weights) and the failure-path test bit W4A4_DEBUG_STALL."""
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    G = lib.w4a4_gemm_s32_ex
+    G.restype = ctypes.c_int
+    G.argtypes = [vp, i64, ctypes.POINTER(WeightsT), vp, ctypes.c_uint32, vp]
+    w = _weights()
+    assert G(A, 0, ctypes.byref(w), A, 0, None) == 0
+    assert G(A, 0, ctypes.byref(w), A, UNPACKED | STALL, None) == 0
+    assert G(A, 10, ctypes.byref(w), A, 0x1, None) == 4                         # GELU: no
+    assert G(A, 10, ctypes.byref(w), A, INT8, None) == 4                        # a weight flag
+    assert G(A, 10, ctypes.byref(_weights(expanded=False)), A, UNPACKED, None) == 1
+    assert G(A, 10, ctypes.byref(_weights8()), A, UNPACKED, None) == 1
+    assert G(A, 10, ctypes.byref(w), None, STALL, None) == 1
+
+
+def test_noalloc_argument_order(lib):
+    """w4a4_linear_fused_noalloc refuses the flags w4a4_linear_fused refuses
+    (W4A4_FLAG_UNPACKED among them) with the same status whatever M is, and
+    sizes beyond its scratch with W4A4_ERR_SHAPE, before any CUDA call."""
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    f = lib.w4a4_linear_fused_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [vp, i64, ctypes.POINTER(WeightsT), vp, ctypes.c_uint32, vp]
+    w = _weights()
+    for M in (10, 1 << 20):
+        assert f(A, M, ctypes.byref(w), A, UNPACKED, None) == 4
+        assert f(A, M, ctypes.byref(w), A, 0x40, None) == 4
+    assert f(A, 16257, ctypes.byref(w), A, 0, None) == 2         # one token past the scratch
+    assert f(A, 4089, ctypes.byref(_weights(K=4096)), A, 0, None) == 2
+    assert f(A, -1, ctypes.byref(w), A, 0, None) == 2
+    assert f(A, 10, None, A, 0, None) == 1

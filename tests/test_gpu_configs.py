@@ -8,9 +8,10 @@ launch configuration the benchmark uses; the oracle recomputes sampled rows
 the bar is the end-to-end one: relative Frobenius error of the sampled rows at
 most 2e-3, and the same SQNR against the unquantized product on both sides.
 The MLP pair is also run as a chain (fc1's bf16 output, through GELU, is fc2's
-input on the GPU; the oracle runs its own chain on the sampled rows and the
-calibration rows): quantization noise compounds along the chain, so there
-the check is on the SQNR of the final output, which must agree within 0.3 dB.
+input on the GPU).  Against the oracle's own chain (its own fc1 output feeding
+its fc2) quantization noise compounds, so there the SQNR of the final output
+must agree within 0.3 dB; fc2 fed the GPU's own fc1 output is held to the
+2e-3 bar.
 """
 import numpy as np
 import pytest
@@ -103,8 +104,8 @@ def test_mlp_pair_chain_8_frames(w4):
     # GPU chain; fc2's calibration input is GELU of the GPU's own fc1 output
     p1 = w4.w4a4_prepare_weights(bf16_dev(W1), bf16_dev(b1), bf16_dev(X[:C]))
     Y1 = w4.w4a4_linear_fused(bf16_dev(X), p1)
-    G1 = torch.nn.functional.gelu(Y1[:C].float()).to(torch.bfloat16)
-    p2 = w4.w4a4_prepare_weights(bf16_dev(W2), bf16_dev(b2), G1)
+    G1c = oracle.gelu_bf16(y_bits(Y1)[:C])           # exact GELU of the GPU's calibration rows
+    p2 = w4.w4a4_prepare_weights(bf16_dev(W2), bf16_dev(b2), bf16_dev(G1c))
     Y2 = w4.w4a4_linear_fused(Y1, p2, flags=w4.W4A4_FLAG_GELU)
     assert w4.w4a4_get_device_status() == 0
     got = synth.bf16_bits_to_f32(y_bits(Y2)[rows]).astype(np.float64)
@@ -113,4 +114,13 @@ def test_mlp_pair_chain_8_frames(w4):
     ref = oracle.reference_fp(oracle.f64_to_bf16(r1), W2, b2, gelu=True)
     sq_gpu, sq_or = oracle.sqnr_db(ref, got), oracle.sqnr_db(ref, Y2o)
     assert abs(sq_gpu - sq_or) < 0.3, (sq_gpu, sq_or)
-    assert rel_fro(got, Y2o) < 0.05
+    # fc2 on its own, held to the end-to-end bar: the oracle's fc2 takes the
+    # GPU's bf16 fc1 output (as the accumulator check takes the GPU's codes),
+    # its smoothing factors calibrated on GELU of the same rows
+    Y1b = y_bits(Y1)
+    o2g = oracle.prepare_weights(W2, b2, G1c, decision="f32")
+    Y2g = oracle.linear(Y1b[rows], o2g, gelu=True, decision="f32")[0]
+    err = rel_fro(got, Y2g)
+    print(f"MLP chain: fc2 on the GPU's fc1 output rel_fro {err:.3e}; chain SQNR gpu {sq_gpu:.2f} "
+          f"oracle {sq_or:.2f} dB")
+    assert err <= 2e-3, err

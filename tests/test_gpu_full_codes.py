@@ -3,9 +3,11 @@
 The oracle's rotation is a dense d x d product, too slow for every row of a
 32-frame batch; here every row is rotated with the Kronecker-factored product
 H_n R H_n (K = n^2, numpy fp64 matrix products; pinned to the oracle's dense
-rotation on sampled rows), and the oracle's binary32-decision quantizer forms
+rotation on sampled rows), and the oracle's quantizer forms
 the exact codes of
-all M x K elements, compared code by code with the GPU's (bit-exact except
+all M x K elements, in both of its decision modes (the fp64 quantizer the
+pages define, and the binary32 decision), compared code by code with the
+GPU's (bit-exact except
 +-1 flips within the fp32 rounding-tie bound of tests/parity.py, at most 1e-4
 of the codes).  Page "十亿参数的三维重建模型，能塞进手机吗？", sections
 预全局旋转 / 后局部平滑 / 训练后量化（PTQ）.
@@ -58,14 +60,17 @@ def test_every_code_of_a_large_batch(w4, frames, K, gelu):
     del qx, Xd
     xin = oracle.bf16_to_f64(oracle.gelu_bf16(X) if gelu else X)
     hat = fwht_rows(xin) * (inv_s.astype(np.float64) / np.sqrt(K))[None, :]
-    want_q, want_d = oracle.quantize_rows(hat, 4, "f32")
-    np.testing.assert_allclose(st, want_d, rtol=2e-5, atol=0)
     amax = np.max(np.abs(hat), axis=1)
     with np.errstate(divide="ignore", invalid="ignore"):
         ratio = np.where(amax[:, None] > 0, hat * 7.0 / amax[:, None], 0.0)
     bound = tie_bound(xin, inv_s.astype(np.float64), ratio, amax, K)
     if gelu:  # GELU in fp32 may land one bf16 step away from the fp64 GELU
         bound = bound + 4.0 * 2.0 ** -8 * np.max(np.abs(xin), axis=1) * np.max(inv_s) / np.sqrt(K) * 7.0 / np.maximum(amax, 1e-300)
-    flips = compare_codes(got, want_q, ratio, bound, 1e-4)
-    print(f"M={M} K={K} gelu={gelu}: {flips} flips of {got.size}")
+    # the method as defined (fp64 decision), then the binary32 decision
+    for decision in ("f64", "f32"):
+        want_q, want_d = oracle.quantize_rows(hat, 4, decision)
+        np.testing.assert_allclose(st, want_d, rtol=2e-5, atol=0)
+        flips = compare_codes(got, want_q, ratio, bound, 1e-4)
+        print(f"M={M} K={K} gelu={gelu}: {flips} flips of {got.size} against the {decision} decision")
+        del want_q
     assert w4.w4a4_get_device_status() == 0

@@ -81,6 +81,67 @@ size_t w4a4_workspace_bytes_min(int64_t M, int32_t K, uint32_t flags) {
   return round256(code_bytes(M, K, flags)) + sizeof(float) * static_cast<size_t>(M);
 }
 
+namespace {
+// The arrays of a prepared layer in one allocation: byte offsets (each a
+// multiple of 256) and sizes; SIZE_MAX marks an array the layout leaves out.
+struct WeightsLayout {
+  size_t qw, qw8, scale_ch, bias, smooth, inv_smooth, colsum, total;
+};
+constexpr size_t kAbsent = ~size_t(0);
+constexpr uint32_t kLayoutFlags = W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED;
+
+bool weights_layout(int32_t N, int32_t K, uint32_t flags, WeightsLayout *L) {
+  if (!k_ok(K) || !n_ok(N) || (flags & ~kLayoutFlags)) return false;
+  const bool int8 = (flags & W4A4_FLAG_INT8) != 0;
+  const bool expanded = int8 || (flags & W4A4_FLAG_UNPACKED) != 0;
+  const size_t n = static_cast<size_t>(N), k = static_cast<size_t>(K);
+  size_t off = 0;
+  auto place = [&](bool present, size_t bytes) {
+    if (!present) return kAbsent;
+    const size_t at = off;
+    off += round256(bytes);
+    return at;
+  };
+  L->qw = place(!int8, n * k / 2);
+  L->qw8 = place(expanded, n * k);
+  L->scale_ch = place(true, 4 * n);
+  L->bias = place(true, 4 * n);
+  L->smooth = place(true, 4 * k);
+  L->inv_smooth = place(true, 4 * k);
+  L->colsum = place(expanded && !int8, 4 * n);
+  L->total = off;
+  return true;
+}
+}  // namespace
+
+size_t w4a4_weights_bytes(int32_t N, int32_t K, uint32_t flags) {
+  WeightsLayout L;
+  return weights_layout(N, K, flags, &L) ? L.total : 0;
+}
+
+w4a4_status w4a4_weights_bind(void *base, size_t bytes, int32_t N, int32_t K, uint32_t flags,
+                              w4a4_weights_t *out) {
+  if (!base || !out) return W4A4_ERR_ARG;
+  if (flags & ~kLayoutFlags) return W4A4_ERR_UNSUPPORTED;
+  if (!aligned16(base)) return W4A4_ERR_ALIGN;
+  WeightsLayout L;
+  if (!weights_layout(N, K, flags, &L)) return k_ok(K) ? W4A4_ERR_SHAPE : W4A4_ERR_UNSUPPORTED;
+  if (bytes < L.total) return W4A4_ERR_SHAPE;
+  uint8_t *b = static_cast<uint8_t *>(base);
+  auto at = [&](size_t off) { return off == kAbsent ? nullptr : b + off; };
+  out->N = N;
+  out->K = K;
+  out->qw = at(L.qw);
+  out->qw8 = reinterpret_cast<int8_t *>(at(L.qw8));
+  out->scale_ch = reinterpret_cast<float *>(at(L.scale_ch));
+  out->bias = reinterpret_cast<float *>(at(L.bias));
+  out->smooth = reinterpret_cast<float *>(at(L.smooth));
+  out->inv_smooth = reinterpret_cast<float *>(at(L.inv_smooth));
+  out->colsum = reinterpret_cast<int32_t *>(at(L.colsum));
+  out->flags = 0;
+  return W4A4_OK;
+}
+
 size_t w4a4_workspace_bytes(int64_t M, int32_t K) {
   return w4a4_workspace_bytes_min(M, K, W4A4_FLAG_UNPACKED);
 }
@@ -211,22 +272,31 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
   return cuda_status(w4a4::launch_gemm(a, cs));
 }
 
-w4a4_status w4a4_gemm_s32(const uint8_t *qx, int64_t M, const w4a4_weights_t *w, int32_t *acc,
-                          void *stream) {
+w4a4_status w4a4_gemm_s32_ex(const uint8_t *qx, int64_t M, const w4a4_weights_t *w, int32_t *acc,
+                             uint32_t flags, void *stream) {
   if (!w) return W4A4_ERR_ARG;
+  if (flags & ~(W4A4_FLAG_UNPACKED | W4A4_DEBUG_STALL)) return W4A4_ERR_UNSUPPORTED;
   if (!k_ok(w->K)) return W4A4_ERR_UNSUPPORTED;
   if (!n_ok(w->N) || !m_ok(M)) return W4A4_ERR_SHAPE;
   if (w->flags & ~kWeightFlags) return W4A4_ERR_UNSUPPORTED;
   const bool int8 = int8_weights(w);
   if (int8 ? !w->qw8 : ((w->qw8 == nullptr) != (w->colsum == nullptr))) return W4A4_ERR_ARG;
+  const bool unpacked = (flags & W4A4_FLAG_UNPACKED) != 0;
+  if (unpacked && (int8 || !w->qw8)) return W4A4_ERR_ARG;
   if (M == 0) return W4A4_OK;
   if (!qx || !acc || (!w->qw && !w->qw8)) return W4A4_ERR_ARG;
   if (!aligned16(qx) || !aligned16(acc) || !aligned16(w->qw) || !aligned16(w->qw8) ||
       !aligned16(w->colsum))
     return W4A4_ERR_ALIGN;
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, nullptr, nullptr, nullptr, nullptr, acc,
-                   M, w->N, w->K, int8};
+                   M, w->N, w->K, int8 || unpacked};
+  a.stall = (flags & W4A4_DEBUG_STALL) != 0;
   return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
+}
+
+w4a4_status w4a4_gemm_s32(const uint8_t *qx, int64_t M, const w4a4_weights_t *w, int32_t *acc,
+                          void *stream) {
+  return w4a4_gemm_s32_ex(qx, M, w, acc, 0, stream);
 }
 
 w4a4_status w4a4_get_device_status(void *stream, uint32_t *status) {

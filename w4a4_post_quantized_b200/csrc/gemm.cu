@@ -66,6 +66,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "ctxcache.h"
 #include "gelu.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -251,7 +252,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      const __grid_constant__ CUtensorMap tmY, const float *__restrict__ scale_tok,
                      const float *__restrict__ scale_ch, const float *__restrict__ bias,
                      const int32_t *__restrict__ colsum, int32_t *__restrict__ acc_out, int M, int N,
-                     int num_n_tiles, int num_tiles, int num_kb) {
+                     int num_n_tiles, int num_tiles, int num_kb, uint32_t stall,
+                     unsigned long long wait_ns) {
   using P = Plan<MODE>;
   constexpr bool B_PACKED = P::B_PACKED;
   constexpr int ST = P::STAGES;
@@ -314,11 +316,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------------------------------------------------------- producer
       uint32_t issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      // stall (a test of the failure path, w4a4_gemm_s32_ex with W4A4_DEBUG_STALL):
+      // no copy is ever issued, so the consumers' first waits run out
+      for (int tile = blockIdx.x; tile < num_tiles && ok && !stall; tile += gridDim.x) {
         const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
         for (int kb = 0; kb < num_kb; ++kb) {
           const uint32_t s = issued % ST, ph = (issued / ST) & 1u;
-          if (!mbar_wait(&freed[s], ph ^ 1u, abort_flag, &g_status)) {
+          if (!mbar_wait(&freed[s], ph ^ 1u, abort_flag, &g_status, wait_ns)) {
             ok = false;
             break;
           }
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // let every issued copy land before the CTA can exit
       for (uint32_t t = (issued > ST ? issued - ST : 0); t < issued; ++t)
-        mbar_wait_drain(&full[t % ST], (t / ST) & 1u, &g_status);
+        mbar_wait_drain(&full[t % ST], (t / ST) & 1u, &g_status, wait_ns);
     }
   } else if (warp == W_MMA) {
     if (lane == 0) {
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
         const uint32_t b = it & 1, pb = (it >> 1) & 1;
-        if (!mbar_wait(&acc_empty[b], pb ^ 1u, abort_flag, &g_status)) break;
+        if (!mbar_wait(&acc_empty[b], pb ^ 1u, abort_flag, &g_status, wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * P::TN;
         if constexpr (P::A_TMEM) {
@@ -349,7 +353,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // slot u, B of each k-block in its TMA stage
           for (int kb = 0; kb < num_kb; kb += P::KG, ++group) {
             const uint32_t u = group % WS, pu = (group / WS) & 1u;
-            if (!mbar_wait(&wready[u], pu, abort_flag, &g_status)) {
+            if (!mbar_wait(&wready[u], pu, abort_flag, &g_status, wait_ns)) {
               ok = false;
               break;
             }
@@ -372,7 +376,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // both operands straight from the TMA stage
           for (int kb = 0; kb < num_kb; ++kb) {
             const uint32_t s = consumed % ST, ps = (consumed / ST) & 1u;
-            if (!mbar_wait(&full[s], ps, abort_flag, &g_status)) {
+            if (!mbar_wait(&full[s], ps, abort_flag, &g_status, wait_ns)) {
               ok = false;
               break;
             }
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t s = consumed % ST;
             const uint32_t u = consumed % WS, pu = (consumed / WS) & 1u;
             // the widen warps waited for the stage's TMA bytes before signalling wready
-            if (!mbar_wait(&wready[u], pu, abort_flag, &g_status)) {
+            if (!mbar_wait(&wready[u], pu, abort_flag, &g_status, wait_ns)) {
               ok = false;
               break;
             }
@@ -412,7 +416,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // every MMA issued must finish before tensor memory is freed
       tc_commit(mma_done);
-      mbar_wait_drain(mma_done, 0, &g_status);
+      mbar_wait_drain(mma_done, 0, &g_status, wait_ns);
     }
   } else if (!P::A8 && warp >= W_UNPACK0 && warp < W_UNPACK0 + 4) {
     // ------------------------------------------------------------------ widen
@@ -426,7 +430,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         for (int kb = 0; kb < num_kb && ok; kb += P::KG, ++grp) {
           const uint32_t u = grp % WS, pu = (grp / WS) & 1u;
-          if (!mbar_wait(&wfree[u], pu ^ 1u, abort_flag, &g_status)) {
+          if (!mbar_wait(&wfree[u], pu ^ 1u, abort_flag, &g_status, wait_ns)) {
             ok = false;
             break;
           }
@@ -434,7 +438,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
           for (int j = 0; j < P::KG; ++j, ++n) {
             const uint32_t s = n % ST, ps = (n / ST) & 1u;
-            if (!mbar_wait(&full[s], ps, abort_flag, &g_status)) {
+            if (!mbar_wait(&full[s], ps, abort_flag, &g_status, wait_ns)) {
               ok = false;
               break;
             }
@@ -474,8 +478,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kb = 0; kb < num_kb; ++kb, ++n) {
           const uint32_t s = n % ST, ps = (n / ST) & 1u;
           const uint32_t u = n % WS, pu = (n / WS) & 1u;
-          if (!mbar_wait(&full[s], ps, abort_flag, &g_status) ||
-              !mbar_wait(&wfree[u], pu ^ 1u, abort_flag, &g_status)) {
+          if (!mbar_wait(&full[s], ps, abort_flag, &g_status, wait_ns) ||
+              !mbar_wait(&wfree[u], pu ^ 1u, abort_flag, &g_status, wait_ns)) {
             ok = false;
             break;
           }
@@ -522,7 +526,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       __syncwarp();
-      if (!mbar_wait(&acc_full[b], pb, abort_flag, &g_status)) break;
+      if (!mbar_wait(&acc_full[b], pb, abort_flag, &g_status, wait_ns)) break;
       tc_fence_after();
       const int row0 = mb * BM + ew * 32;
       if constexpr (!OUT_S32 && P::EPI16) {
@@ -751,16 +755,13 @@ template <int MODE, bool OUT_S32, bool GELU_OUT = false>
 cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   using P = Plan<MODE>;
   auto kern = w4a4_gemm_kernel<MODE, OUT_S32, GELU_OUT>;
-  static bool attr_set[64] = {};  // per device
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static ContextCache<bool> attr_set;  // the shared-memory attribute, per context
+  bool done = false;
+  cudaError_t e = attr_set.get(&done, [&](bool *v) {
+    *v = true;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES);
+  });
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
   CUtensorMap tmA, tmB, tmY;
   const uint64_t kp = static_cast<uint64_t>(a.K / 2);
   const bool okA = P::A8 ? make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qx, a.K, a.M, a.K, BK,
@@ -796,8 +797,11 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // a stalled launch (failure-path test) gives every bounded wait 1 ms
+  const unsigned long long wait_ns = a.stall ? 1000000ull : kWaitLimitNs;
   e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmY, a.scale_tok, a.scale_ch, a.bias, a.colsum, a.acc,
-                         static_cast<int>(a.M), a.N, num_n, tiles, a.K / BK);
+                         static_cast<int>(a.M), a.N, num_n, tiles, a.K / BK,
+                         static_cast<uint32_t>(a.stall ? 1u : 0u), wait_ns);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -828,15 +832,41 @@ cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, 
   return cudaGetLastError();
 }
 
-unsigned int *status_word() {
-  static unsigned int *addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
+cudaError_t status_word(unsigned int **out) {
+  static ContextCache<unsigned int *> cache;
+  const cudaError_t e = cache.get(out, [](unsigned int **p) {
+    void *a = nullptr;
+    const cudaError_t r = cudaGetSymbolAddress(&a, g_status);
+    *p = static_cast<unsigned int *>(a);
+    return r;
+  });
+  if (e == cudaSuccess && *out == nullptr) return cudaErrorInvalidSymbol;
+  return e;
+}
+
+unsigned long long current_context_id() {
+  using GetCurrentFn = CUresult (*)(CUcontext *);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) == cudaSuccess) addr[dev] = static_cast<unsigned int *>(p);
-  }
-  return addr[dev];
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
 }
 
 cudaError_t read_status(unsigned int *out, cudaStream_t st) {

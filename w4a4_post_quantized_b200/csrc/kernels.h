@@ -41,13 +41,16 @@ struct GemmArgs {
   bool a8;                  // qx and qw8 hold one code per byte in the same order (int8 codes,
                             // or int4 codes in operand order): no widening
   bool gelu_out = false;    // y = bf16(GELU(bf16 result)) (an MLP's first linear)
+  bool stall = false;       // failure-path test: the TMA producer issues nothing and every
+                            // bounded wait gives up after 1 ms (sets the status word)
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,
                                   cudaStream_t st);
 
-// status word (device address of the current device's word, for kernel arguments)
-unsigned int *status_word();
+// status word: *out = its device address in the current context (for kernel
+// arguments); an error when the lookup fails (nothing may then be launched)
+cudaError_t status_word(unsigned int **out);
 cudaError_t read_status(unsigned int *out, cudaStream_t st);
 cudaError_t clear_status(cudaStream_t st);
 

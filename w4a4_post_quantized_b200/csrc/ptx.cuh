@@ -61,17 +61,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase of `bar` with the given parity has completed.  Gives up
 // (returns false, sets bit 0 (W4A4_DEV_TIMEOUT) of *status, raises *abort)
-// after kWaitLimitNs, and returns false early when another role of the CTA has
-// raised *abort.
+// after limit_ns of %globaltimer, and returns false early when another role of
+// the CTA has raised *abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          unsigned int *status) {
+                                          unsigned int *status,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (;;) {
     if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(status, 1u);
       *abort = 1;
       return false;
@@ -82,12 +83,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 // Same as mbar_wait but ignores *abort: used on the exit path to let copies
 // that are already in flight land before the CTA leaves.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
-                                                unsigned int *status) {
+                                                unsigned int *status,
+                                                unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(a, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(status, 1u);
       return false;
     }

@@ -38,6 +38,7 @@
 
 #include <cstdint>
 
+#include "ctxcache.h"
 #include "fwht.cuh"
 #include "gelu.cuh"
 #include "kernels.h"
@@ -363,15 +364,16 @@ __global__ void fill_kernel(float *__restrict__ out, int n, float v) {
 }
 
 int num_sms() {
-  static int sms[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (sms[dev] == 0) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    sms[dev] = n > 0 ? n : 148;
-  }
-  return sms[dev];
+  static ContextCache<int> sms;
+  int n = 0;
+  if (sms.get(&n, [](int *v) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev);
+        return e;
+      }) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
 }
 
 template <typename Kern>
@@ -390,19 +392,19 @@ cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint
   auto kern = quantize_rows_kernel<K, ROT, GELU, CODE>;
   constexpr int smem = QuantStaging<K>::SMEM;
   constexpr int kRowsPerBlock = kQuantWarps;  // one warp per row
-  static int per_sm_dev[64] = {};  // per device: attribute set and occupancy known
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  int &per_sm = per_sm_dev[dev];
-  if (per_sm == 0) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
+  static ContextCache<int> occupancy;  // per context: attribute set, resident blocks per SM
+  int per_sm = 0;
+  cudaError_t e = occupancy.get(&per_sm, [&](int *v) {
+    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (r != cudaSuccess) return r;
     int n = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kQuantWarps * 32, smem);
-    per_sm = n < 1 ? 1 : n;
-  }
+    r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kQuantWarps * 32, smem);
+    *v = n < 1 ? 1 : n;
+    return r;
+  });
+  if (e != cudaSuccess) return e;
+  unsigned int *status = nullptr;
+  if ((e = status_word(&status)) != cudaSuccess) return e;
   const int64_t need = (M + kRowsPerBlock - 1) / kRowsPerBlock;
   const int64_t g = static_cast<int64_t>(num_sms()) * per_sm;
   const int grid = static_cast<int>(need < g ? need : g);
@@ -418,7 +420,7 @@ cudaError_t launch_quant_k(const uint16_t *X, int64_t M, const float *mult, uint
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, X, M, mult, q, scale, status_word());
+  e = cudaLaunchKernelEx(&cfg, kern, X, M, mult, q, scale, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

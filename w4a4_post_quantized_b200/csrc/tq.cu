@@ -16,6 +16,7 @@
 #include <cmath>
 #include <cstdint>
 
+#include "ctxcache.h"
 #include "fwht.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -253,7 +254,10 @@ cudaError_t launch_pdl(void (*kern)(const float *, int64_t, const float *, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, X, n, signs, bnd, codes, norms, status_word());
+  unsigned int *status = nullptr;
+  const cudaError_t e = status_word(&status);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, kern, X, n, signs, bnd, codes, norms, status);
 }
 
 // ---------------------------------------------------------------- codebook
@@ -339,17 +343,17 @@ w4a4_status tq_encode(const float *X, int64_t n, int32_t d, const float *signs,
       !tq_aligned16(boundaries))
     return W4A4_ERR_ALIGN;
   using S = w4a4::TqEncodeStaging;
-  static int per_sm_dev[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4A4_ERR_CUDA;
-  if (per_sm_dev[dev] == 0) {
-    if (cudaFuncSetAttribute(w4a4::tq_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             S::SMEM) != cudaSuccess)
-      return W4A4_ERR_CUDA;
-    per_sm_dev[dev] = w4a4::blocks_per_sm(w4a4::tq_encode_kernel, S::SMEM);
-  }
+  static w4a4::ContextCache<int> occupancy;  // per context: attribute set, blocks per SM
+  int per_sm = 0;
+  if (occupancy.get(&per_sm, [](int *v) {
+        const cudaError_t r = cudaFuncSetAttribute(
+            w4a4::tq_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        if (r == cudaSuccess) *v = w4a4::blocks_per_sm(w4a4::tq_encode_kernel, S::SMEM);
+        return r;
+      }) != cudaSuccess)
+    return W4A4_ERR_CUDA;
   const int64_t need = (n + w4a4::kTqWarps - 1) / w4a4::kTqWarps;
-  const int64_t g = static_cast<int64_t>(w4a4::device_sm_count()) * per_sm_dev[dev];
+  const int64_t g = static_cast<int64_t>(w4a4::device_sm_count()) * per_sm;
   const int grid = static_cast<int>(need < g ? need : g);
   cudaError_t e = w4a4::launch_pdl(w4a4::tq_encode_kernel, grid, S::SMEM,
                                    static_cast<cudaStream_t>(stream), X, n, signs, boundaries, codes,
@@ -367,12 +371,15 @@ w4a4_status tq_decode(const uint8_t *codes, const float *norms, int64_t n, int32
   if (!tq_aligned16(codes) || !tq_aligned16(Y) || !tq_aligned16(signs) || !tq_aligned16(norms) ||
       !tq_aligned16(centroids))
     return W4A4_ERR_ALIGN;
-  static int per_sm_dev[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4A4_ERR_CUDA;
-  if (per_sm_dev[dev] == 0) per_sm_dev[dev] = w4a4::blocks_per_sm(w4a4::tq_decode_kernel, 0);
+  static w4a4::ContextCache<int> occupancy;  // per context: blocks per SM
+  int per_sm = 0;
+  if (occupancy.get(&per_sm, [](int *v) {
+        *v = w4a4::blocks_per_sm(w4a4::tq_decode_kernel, 0);
+        return cudaSuccess;
+      }) != cudaSuccess)
+    return W4A4_ERR_CUDA;
   const int64_t need = (n + w4a4::kTqWarps - 1) / w4a4::kTqWarps;
-  const int64_t g = static_cast<int64_t>(w4a4::device_sm_count()) * per_sm_dev[dev];
+  const int64_t g = static_cast<int64_t>(w4a4::device_sm_count()) * per_sm;
   const int grid = static_cast<int>(need < g ? need : g);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);

@@ -30,6 +30,7 @@ W4A4_FLAG_PLAIN = 0x2
 W4A4_FLAG_INT8 = 0x4
 W4A4_FLAG_UNPACKED = 0x8
 W4A4_FLAG_GELU_OUT = 0x10
+W4A4_DEBUG_STALL = 0x80000000
 
 _vp, _i32, _i64, _u32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
                                     ctypes.c_float, ctypes.c_size_t)
@@ -60,6 +61,11 @@ _fused = _sig("w4a4_linear_fused", ctypes.c_int,
 _fused_noalloc = _sig("w4a4_linear_fused_noalloc", ctypes.c_int,
                       [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _u32, _vp])
 _gemm_s32 = _sig("w4a4_gemm_s32", ctypes.c_int, [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _vp])
+_gemm_s32_ex = _sig("w4a4_gemm_s32_ex", ctypes.c_int,
+                    [_vp, _i64, ctypes.POINTER(W4A4WeightsT), _vp, _u32, _vp])
+_weights_bytes = _sig("w4a4_weights_bytes", _sz, [_i32, _i32, _u32])
+_weights_bind = _sig("w4a4_weights_bind", ctypes.c_int,
+                     [_vp, _sz, _i32, _i32, _u32, ctypes.POINTER(W4A4WeightsT)])
 _pipe_create = _sig("w4a4_host_pipe_create", ctypes.c_int, [ctypes.POINTER(_vp)])
 _pipe_destroy = _sig("w4a4_host_pipe_destroy", ctypes.c_int, [_vp])
 _host_ws_bytes = _sig("w4a4_host_workspace_bytes", _sz, [_i64, _i32, _i32])
@@ -111,26 +117,46 @@ def w4a4_workspace_bytes_min(M: int, K: int, flags: int) -> int:
     return int(_workspace_bytes_min(M, K, flags))
 
 
+def w4a4_weights_bytes(N: int, K: int, flags: int = 0) -> int:
+    return int(_weights_bytes(N, K, flags))
+
+
 class PreparedWeights:
-    """Device arrays of one prepared layer (owned by torch) and the C struct
-    that points at them.  expanded=True also allocates the widened int8 copy
-    of the codes (qw8, N*K bytes) and the per-row code sums the fast GEMM
-    path uses; expanded=False keeps only the packed int4 codes.  int8=True
-    (the W8A8 setting) allocates only qw8, which then holds the 8-bit codes."""
+    """Device arrays of one prepared layer and the C struct that points at
+    them: one torch-owned allocation of w4a4_weights_bytes(N, K, layout) bytes,
+    laid out by w4a4_weights_bind; the attributes (qw, scale_ch, ...) are typed
+    views into it.  expanded=True also holds the widened int8 copy of the codes
+    (qw8, N*K bytes) and the per-row code sums the fast GEMM path uses;
+    expanded=False keeps only the packed int4 codes.  int8=True (the W8A8
+    setting) holds qw8 with the 8-bit codes and no packed codes."""
 
     def __init__(self, N: int, K: int, device="cuda", expanded: bool = True, int8: bool = False):
         self.N, self.K = N, K
         self.device = torch.device(device)
-        self.qw = None if int8 else torch.empty((N, K // 2), dtype=torch.uint8, device=device)
-        self.scale_ch = torch.empty(N, dtype=torch.float32, device=device)
-        self.bias = torch.empty(N, dtype=torch.float32, device=device)
-        self.smooth = torch.empty(K, dtype=torch.float32, device=device)
-        self.inv_smooth = torch.empty(K, dtype=torch.float32, device=device)
-        self.qw8 = torch.empty((N, K), dtype=torch.int8, device=device) if (expanded or int8) else None
-        self.colsum = torch.empty(N, dtype=torch.int32, device=device) if (expanded and not int8) else None
-        self.struct = W4A4WeightsT(N, K, _ptr(self.qw), self.scale_ch.data_ptr(),
-                                   self.bias.data_ptr(), self.smooth.data_ptr(),
-                                   self.inv_smooth.data_ptr(), _ptr(self.qw8), _ptr(self.colsum), 0)
+        layout = W4A4_FLAG_INT8 if int8 else (W4A4_FLAG_UNPACKED if expanded else 0)
+        nbytes = w4a4_weights_bytes(N, K, layout)
+        if nbytes == 0:
+            raise W4A4Error(W4A4_ERR_SHAPE, "w4a4_weights_bytes")
+        self.storage = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.struct = W4A4WeightsT()
+        _check(_weights_bind(_ptr(self.storage), nbytes, N, K, layout, ctypes.byref(self.struct)),
+               "w4a4_weights_bind")
+        base = self.storage.data_ptr()
+
+        def view(addr, count, dtype, shape):
+            if not addr:
+                return None
+            off = addr - base
+            nb = count * torch.empty((), dtype=dtype).element_size()
+            return self.storage[off:off + nb].view(dtype).view(shape)
+        st = self.struct
+        self.qw = view(st.qw, N * K // 2, torch.uint8, (N, K // 2))
+        self.scale_ch = view(st.scale_ch, N, torch.float32, (N,))
+        self.bias = view(st.bias, N, torch.float32, (N,))
+        self.smooth = view(st.smooth, K, torch.float32, (K,))
+        self.inv_smooth = view(st.inv_smooth, K, torch.float32, (K,))
+        self.qw8 = view(st.qw8, N * K, torch.int8, (N, K))
+        self.colsum = view(st.colsum, N, torch.int32, (N,))
 
     @property
     def flags(self) -> int:
@@ -258,6 +284,14 @@ def w4a4_gemm_s32(qx: torch.Tensor, w: PreparedWeights, acc=None, stream=None):
     M = qx.shape[0]
     acc = acc if acc is not None else torch.empty((M, w.N), dtype=torch.int32, device=qx.device)
     _check(_gemm_s32(_ptr(qx), M, ctypes.byref(w.struct), _ptr(acc), _stream(stream)), "w4a4_gemm_s32")
+    return acc
+
+
+def w4a4_gemm_s32_ex(qx: torch.Tensor, w: PreparedWeights, flags: int = 0, acc=None, stream=None):
+    M = qx.shape[0]
+    acc = acc if acc is not None else torch.empty((M, w.N), dtype=torch.int32, device=qx.device)
+    _check(_gemm_s32_ex(_ptr(qx), M, ctypes.byref(w.struct), _ptr(acc), flags, _stream(stream)),
+           "w4a4_gemm_s32_ex")
     return acc
 
 
