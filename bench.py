@@ -4,14 +4,21 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
 
-Workload (default): the frame-attention QKV linear of a VGGT-style 1024-wide
-transformer at 8 frames: X [10992, 1024] bf16 -> Y [10992, 3072] bf16, one
-"step" = the whole hot path on one batch: rotate + smooth + per-token int4
-quantize + pack (kernel 1), integer GEMM on the tensor cores + dequant/bias
-epilogue (kernel 2).  Weight preparation is offline and untimed.
+Workload (default, c5_full_stack): the full-depth linear stack of a VGGT-style
+1024-wide transformer at 64 frames (M = 87936 tokens): 48 blocks x the four
+linears (QKV 1024->3072, proj 1024->1024, fc1 1024->4096 with the GELU on its
+output, fc2 4096->1024), fresh seeded weights per layer and a fresh seeded
+heavy-tailed activation batch for every layer that reads the block's input
+(fc2 reads its block's GELU(fc1) output).  One "step" = every layer once:
+rotate + smooth + per-token int4 quantize (kernel 1), integer GEMM on the
+tensor cores + dequant/bias epilogue (kernel 2).  Weight preparation is
+offline and untimed.  Other workloads (--workload): the single linear, the
+frame-attention QKV at 8 frames, the MLP pair, the global-attention block and
+the 3DTurboQuant KV-cache codec.
 
-Metric: W4A4 linear throughput in TOPS (2*M*N*K integer ops per step), with
-tokens/s alongside; roofline fractions against the measured peaks.
+Metric: W4A4 linear throughput in TOPS (2*M*N*K integer ops per layer, summed
+over the step), with tokens/s alongside; roofline fractions of the GEMM
+against the int8 tensor peak and of the quantize kernel against HBM bandwidth.
 
 Under torchrun each rank runs an independent replica on its own GPU (token
 batches are independent: weak scaling, no data-path collective); the timed
@@ -521,6 +528,124 @@ def run_ours(args, wl, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def stack_layers(st):
+    """(block, name, K, N) of every layer of a multi-layer workload, in order."""
+    return [(b, name, K, N) for b in range(st["blocks"]) for (name, K, N) in st["layers"]]
+
+
+def stack_ops(st, M):
+    return sum(2.0 * M * N * K for (_, _, K, N) in stack_layers(st))
+
+
+def stack_oracle_sample(st, rows: int, seed: int = 0):
+    """Prepare (untimed) the oracle's weights for one block's layer shapes and
+    return a closure that runs the oracle's hot path on `rows` token rows of
+    each (special-token rows first, then a regular stride of patch tokens;
+    fc2's input through the GELU, as the block's MLP feeds it).  One block
+    stands for every block of the stack: they share the four layer shapes."""
+    import oracle
+    M = st["frames"] * synth.FRAME_TOKENS
+    sel = np.concatenate([synth.special_rows(M), np.arange(5, M, max(1, M // rows))])[:rows]
+    cases = []
+    for j, (name, K, N) in enumerate(st["layers"]):
+        W = synth.weights(N, K, seed=seed + 10 * j + 1)
+        b = synth.bias(N, seed=seed + 10 * j + 2)
+        Xc = synth.activations(synth.calibration_rows(M), K, seed=seed + 10 * j + 3)
+        gelu = name == "fc2"
+        pw = oracle.prepare_weights(W, b, oracle.gelu_bf16(Xc) if gelu else Xc)
+        # the sampled rows of a full-size batch, drawn directly (the generator's
+        # special rows sit at the frame starts, so sel's first rows are those)
+        X = synth.activations(len(sel), K, seed=seed + 10 * j + 4)
+        cases.append((X, pw, gelu))
+
+    def run():
+        for X, pw, gelu in cases:
+            oracle.linear(X, pw, gelu=gelu)
+    return run, len(sel), oracle.max_threads()
+
+
+def time_stack_oracle(st, rows: int, budget_s: float, max_passes: int = 8):
+    """The oracle's per-token rate on the stack: one block's four layer shapes
+    on `rows` rows per pass, repeated until about budget_s of CPU time; the
+    stack's time per token is 48 blocks' worth of that block's."""
+    run, r, cores = stack_oracle_sample(st, rows)
+    passes, t_total = 0, 0.0
+    while passes < max_passes and (passes == 0 or t_total < budget_s):
+        t = time.perf_counter()
+        run()
+        t_total += time.perf_counter() - t
+        passes += 1
+    t_block = t_total / passes
+    M = st["frames"] * synth.FRAME_TOKENS
+    sec_per_token = t_block * st["blocks"] / r
+    tops = stack_ops(st, M) / M / sec_per_token / 1e12
+    return tops, 1.0 / sec_per_token, r, passes, t_block, cores
+
+
+def run_stack_reference(args, st, world, rank):
+    """The reference arm on a multi-layer workload: the CPU oracle on a
+    bounded row sample of one block's four layer shapes per step (the stack's
+    rate is 48 blocks of that), sized so the whole run takes a few minutes."""
+    if rank != 0:
+        return
+    run, r0, _ = stack_oracle_sample(st, 64)
+    t = time.perf_counter()
+    run()
+    per_row = (time.perf_counter() - t) / r0
+    rows = int(min(args.cpu_rows * 2, max(32, 150.0 / max(1, args.steps + args.warmup) / per_row)))
+    run, r, cores = stack_oracle_sample(st, rows)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    t_block = (time.perf_counter() - t0) / args.steps
+    M = st["frames"] * synth.FRAME_TOKENS
+    sec_per_token = t_block * st["blocks"] / r
+    tops = stack_ops(st, M) / M / sec_per_token / 1e12
+    sample = (f"{r} of {M} token rows (special tokens included) through one block's four layer "
+              f"shapes per step; the stack's rate is {st['blocks']} blocks of it (sampled, per-token rate)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_block * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/int64",
+        "data": "synthetic", "tokens_per_s": 1.0 / sec_per_token,
+        "config": {"workload": st["desc"], "M": M, "blocks": st["blocks"], "M_sampled": r,
+                   "layers": [f"{n} {K}->{N}" for (n, K, N) in st["layers"]]},
+        "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def int8_ceiling(dev, stream):
+    """Dense int8 tensor-core throughput measured on this GPU by a library
+    GEMM (cuBLASLt through torch._int_mm, 8192^3, s8 x s8 -> s32): the
+    measured ceiling the GEMM's roofline fraction is also reported against.
+    None when the library call is not available here."""
+    import torch
+    try:
+        n = 8192
+        a = torch.randint(-8, 8, (n, n), dtype=torch.int8, device=dev)
+        b = torch.randint(-8, 8, (n, n), dtype=torch.int8, device=dev).t()
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        e0.record(stream)
+        for _ in range(reps):
+            torch._int_mm(a, b)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        del a, b
+        return {"tops": 2.0 * n ** 3 / (ms * 1e-3) / 1e12, "ms": ms,
+                "how": "torch._int_mm (cuBLASLt) s8 x s8 -> s32, 8192^3, 20 back-to-back calls"}
+    except Exception as e:  # noqa: BLE001
+        return {"tops": None, "why": f"{type(e).__name__}: {e}"[:200]}
+
+
 def run_stack(args, st, world, rank, local):
     """A block (or stack of blocks) of quantized linears: one step = every
     layer once, in order, on one batch of M tokens."""
@@ -529,38 +654,41 @@ def run_stack(args, st, world, rank, local):
     M = st["frames"] * synth.FRAME_TOKENS
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
-    layers = [(b, name, K, N) for b in range(st["blocks"]) for (name, K, N) in st["layers"]]
-
-    def bf16(bits):
-        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
-
-    # inputs: two synthetic activation sets (K = 1024) rotate over the blocks;
-    # weights: fresh per layer (seeded normal(0, 0.02^2) / (0, 0.01^2) drawn on
-    # the device: a stack holds up to 192 of them), prepared untimed
-    Xp = [bf16(synth.activations(M, 1024, seed=1000 * rank + 10 + i)) for i in range(2)]
+    layers = stack_layers(st)
     C = synth.calibration_rows(M)
-    gen = torch.Generator(device=dev)
+    GOUT, UNP = w4a4.W4A4_FLAG_GELU_OUT, w4a4.W4A4_FLAG_UNPACKED
+
+    # ------------------------------------------------------------ inputs (untimed)
+    # every layer that reads the block's input stream (qkv, proj, fc1) gets a
+    # fresh seeded heavy-tailed activation batch of its own, drawn on the
+    # device; fc2 reads GELU(fc1's output) of its block (the MLP's own data
+    # flow; fc1's GEMM epilogue applies the GELU).  Weights: fresh seeded
+    # normal(0, 0.02^2) per layer, bias normal(0, 0.01^2), prepared untimed.
+    seed0 = 100000 * rank
+    X = {i: synth.activations_device(M, K, seed0 + i, dev)
+         for i, (_, name, K, _) in enumerate(layers) if name != "fc2"}
+    Ys = {name: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (name, K, N) in st["layers"]}
     pws = []
     for i, (b, name, K, N) in enumerate(layers):
-        gen.manual_seed(1000 * rank + 7 * i + 1)
-        W = (torch.randn((N, K), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
-        bias = (torch.randn(N, generator=gen, device=dev) * 0.01).to(torch.bfloat16)
-        Xc = Xp[b % 2][:C] if K == 1024 else torch.nn.functional.gelu(
-            (torch.randn((C, K), generator=gen, device=dev))).to(torch.bfloat16)
+        W = synth.weights_device(N, K, seed0 + 7 * i + 1, dev)
+        bias = synth.bias_device(N, seed0 + 7 * i + 2, dev)
+        if name == "fc2":   # calibration: the block's fc1 output (with its GELU) on the first frame
+            Xc = w4a4.w4a4_linear_fused(X[i - 1][:C], pws[i - 1], flags=GOUT)
+        else:
+            Xc = X[i][:C]
         pws.append(w4a4.w4a4_prepare_weights(W, bias, Xc))
-        del W
-    Ys = {name: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (name, K, N) in st["layers"]}
+        del W, bias, Xc
     ws = torch.empty(max(w4a4.w4a4_workspace_bytes(M, K) for (_, _, K, _) in layers), dtype=torch.uint8,
                      device=dev)
     torch.cuda.synchronize()
-    ops_step = sum(2.0 * M * N * K for (_, _, K, N) in layers)
+    ops_step = stack_ops(st, M)
 
-    # the MLP's GELU is applied by fc1's GEMM epilogue to its output (the same
-    # bf16 values as applying it in fc2's quantize kernel to its input)
+    def layer_input(i, name):
+        return Ys["fc1"] if name == "fc2" else X[i]
+
     def run_layer(i, b, name, K, N):
-        x = Ys["fc1"] if name == "fc2" else Xp[b % 2]
-        w4a4.w4a4_linear_fused(x, pws[i], Y=Ys[name], workspace=ws,
-                               flags=w4a4.W4A4_FLAG_GELU_OUT if name == "fc1" else 0)
+        w4a4.w4a4_linear_fused(layer_input(i, name), pws[i], Y=Ys[name], workspace=ws,
+                               flags=GOUT if name == "fc1" else 0)
 
     def step():
         for i, (b, name, K, N) in enumerate(layers):
@@ -570,6 +698,8 @@ def run_stack(args, st, world, rank, local):
         step()
     torch.cuda.synchronize()
     w4a4.w4a4_clear_device_status()
+
+    # ---------------------------------------------------------------- timed region
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
@@ -580,40 +710,51 @@ def run_stack(args, st, world, rank, local):
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        # per-layer-shape attribution: events around each layer of one step
-        per = {name: 0.0 for (name, _, _) in st["layers"]}
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+        # attribution step (not part of `value`): the same work as a step, the
+        # fused call's two kernels launched separately (the quantize kernel's
+        # one-per-byte codes into the workspace, then the GEMM) with CUDA
+        # events on the launching stream around each, for every layer
+        ws_q = ws[:M * 4096]
+        st_off = ((M * 4096 + 255) // 256) * 256
+        ws_s = ws[st_off:st_off + 4 * M].view(torch.float32)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layers]
         for i, (b, name, K, N) in enumerate(layers):
+            q = ws_q[:M * K].view(M, K)
             ev[i][0].record(stream)
-            run_layer(i, b, name, K, N)
+            w4a4.w4a4_quantize_act(layer_input(i, name), pws[i].inv_smooth, UNP, qx=q, scale_tok=ws_s)
             ev[i][1].record(stream)
+            w4a4.w4a4_linear_ex(q, ws_s, pws[i], flags=UNP | (GOUT if name == "fc1" else 0), Y=Ys[name])
+            ev[i][2].record(stream)
         torch.cuda.synchronize()
-        for (e0, e1), (b, name, K, N) in zip(ev, layers):
-            per[name] += e0.elapsed_time(e1)
     status = w4a4.w4a4_get_device_status()
     elapsed_ms = max_over_ranks(world, t0.elapsed_time(t1))
     ms_step = elapsed_ms / args.steps
     value = world * ops_step * args.steps / (elapsed_ms * 1e-3) / 1e12
+    q_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    g_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    q_bytes = [2.0 * M * K + M * K + 4.0 * M for (_, _, K, _) in layers]   # X in, one-per-byte codes, steps
+    g_ops = [2.0 * M * N * K for (_, _, K, N) in layers]
     peaks = load_peaks()
-    int8_peak = peaks["bf16"] * INT8_PER_BF16
-    per_layer = {}
-    for (name, K, N) in st["layers"]:
-        t = per[name] / st["blocks"]
-        per_layer[name] = {"K": K, "N": N, "ms_per_layer": t,
-                           "tops": 2.0 * M * N * K / (t * 1e-3) / 1e12}
-    # each kernel alone, per layer shape (block 0's weights and the step's
-    # inputs): the quantize kernel (codes one per byte, the fused call's route)
-    # and the GEMM, n_iso back-to-back launches each between CUDA events
+    int8_peak_burst = peaks["bf16"] * INT8_PER_BF16
+    int8_peak = (peaks["bf16_sus"] or peaks["bf16"]) * INT8_PER_BF16   # kernels timed inside a long step
+    per = {name: {"quantize_ms": 0.0, "gemm_ms": 0.0, "count": 0} for (name, _, _) in st["layers"]}
+    for (b, name, K, N), tq_, tg_ in zip(layers, q_ms, g_ms):
+        per[name]["quantize_ms"] += tq_
+        per[name]["gemm_ms"] += tg_
+        per[name]["count"] += 1
+
+    # each kernel alone, per layer shape (block 0's weights and inputs): 10
+    # back-to-back launches between CUDA events
     n_iso = 10
+    per_layer = {}
     for i, (b, name, K, N) in enumerate(layers[:len(st["layers"])]):
-        x = Ys["fc1"] if name == "fc2" else Xp[b % 2]
-        fl = w4a4.W4A4_FLAG_UNPACKED
-        gfl = fl | (w4a4.W4A4_FLAG_GELU_OUT if name == "fc1" else 0)
-        q, sq = w4a4.w4a4_quantize_act(x, pws[i].inv_smooth, fl)
-        Yk = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        x = layer_input(i, name)
+        gfl = UNP | (GOUT if name == "fc1" else 0)
+        q = ws_q[:M * K].view(M, K)
+        Yk = Ys[name]
         times = []
-        for fn in (lambda: w4a4.w4a4_quantize_act(x, pws[i].inv_smooth, fl, qx=q, scale_tok=sq),
-                   lambda: w4a4.w4a4_linear_ex(q, sq, pws[i], flags=gfl, Y=Yk)):
+        for fn in (lambda: w4a4.w4a4_quantize_act(x, pws[i].inv_smooth, UNP, qx=q, scale_tok=ws_s),
+                   lambda: w4a4.w4a4_linear_ex(q, ws_s, pws[i], flags=gfl, Y=Yk)):
             fn()
             torch.cuda.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -625,50 +766,135 @@ def run_stack(args, st, world, rank, local):
             times.append(max_over_ranks(world, e0.elapsed_time(e1)) / n_iso)
         tq_ms, tg_ms = times
         gtops = 2.0 * M * N * K / (tg_ms * 1e-3) / 1e12
-        per_layer[name].update({
-            "quantize_us": tq_ms * 1e3, "quantize_gbs": (2.5 * M * K + 4 * M) / (tq_ms * 1e-3) / 1e9,
-            "gemm_us": tg_ms * 1e3, "gemm_tops": gtops, "gemm_frac": gtops / int8_peak})
-        del q, sq, Yk
-    # end to end: the first layer's input from pinned host memory, the last
-    # layer's output back, around one whole step
-    Xh = torch.empty((M, 1024), dtype=torch.bfloat16, pin_memory=True)
-    Xh.copy_(Xp[0].cpu())
-    last = st["layers"][-1]
-    Yh = torch.empty((M, last[2]), dtype=torch.bfloat16, pin_memory=True)
+        c = per[name]["count"]
+        per_layer[name] = {
+            "K": K, "N": N, "layers": c,
+            "in_step_quantize_us": per[name]["quantize_ms"] / c * 1e3,
+            "in_step_gemm_us": per[name]["gemm_ms"] / c * 1e3,
+            "alone_quantize_us": tq_ms * 1e3, "alone_quantize_gbs": (3.0 * M * K + 4 * M) / (tq_ms * 1e-3) / 1e9,
+            "alone_gemm_us": tg_ms * 1e3, "alone_gemm_tops": gtops,
+            "alone_gemm_frac_burst": gtops / int8_peak_burst}
+    # M7 (the pages' +0.2 % for DSFQ over plain quantization): the fused call per
+    # layer shape with the rotation and smoothing skipped (weights of the same
+    # layers prepared plain), 10 calls each, summed over the stack's layers
+    m7 = {"dsfq": 0.0, "plain": 0.0}
+    for i, (b, name, K, N) in enumerate(layers[:len(st["layers"])]):
+        x = layer_input(i, name)
+        W = synth.weights_device(N, K, seed0 + 7 * i + 1, dev)
+        bias = synth.bias_device(N, seed0 + 7 * i + 2, dev)
+        pplain = w4a4.w4a4_prepare_weights(W, bias, None, flags=w4a4.W4A4_FLAG_PLAIN)
+        for mode, p, fl in (("dsfq", pws[i], 0), ("plain", pplain, w4a4.W4A4_FLAG_PLAIN)):
+            fl |= GOUT if name == "fc1" else 0
+            fn = lambda: w4a4.w4a4_linear_fused(x, p, Y=Ys[name], workspace=ws, flags=fl)
+            fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n_iso):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            m7[mode] += st["blocks"] * max_over_ranks(world, e0.elapsed_time(e1)) / n_iso
+        del W, bias, pplain
+    ceiling = int8_ceiling(dev, stream)
+
+    # ------------------------------------------------------------- end to end
+    # through the C ABI's host-buffer call: the stack's input comes from pinned
+    # host memory into the first layer (w4a4_linear_fused_host, X on the host,
+    # Y left on the device) and the last layer's output goes back to pinned host
+    # memory (X on the device, Y on the host); the layers between run on the
+    # device.  Copies overlap those two layers' kernels chunk by chunk.
+    chunk = args.e2e_chunk
+    Xh = torch.empty((M, layers[0][2]), dtype=torch.bfloat16, pin_memory=True)
+    Xh.copy_(X[0].cpu())
+    last = len(layers) - 1
+    Yh = torch.empty((M, layers[last][3]), dtype=torch.bfloat16, pin_memory=True)
+    pipe = w4a4.HostPipe()
+    hws = torch.empty(max(w4a4.w4a4_host_workspace_bytes(chunk, K, N) for (_, _, K, N) in layers),
+                      dtype=torch.uint8, device=dev)
+
+    def host_step():
+        for i, (b, name, K, N) in enumerate(layers):
+            fl = GOUT if name == "fc1" else 0
+            if i == 0:
+                w4a4.w4a4_linear_fused_host(Xh, pws[i], Y_host=Ys[name], chunk_rows=chunk, workspace=hws,
+                                            pipe=pipe, flags=fl | w4a4.W4A4_FLAG_Y_DEVICE)
+            elif i == last:
+                w4a4.w4a4_linear_fused_host(layer_input(i, name), pws[i], Y_host=Yh, chunk_rows=chunk,
+                                            workspace=hws, pipe=pipe, flags=fl | w4a4.W4A4_FLAG_X_DEVICE)
+            else:
+                run_layer(i, b, name, K, N)
     n_e2e = max(3, min(args.steps, args.e2e_steps))
+    host_step()
+    torch.cuda.synchronize()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     a0.record(stream)
     for _ in range(n_e2e):
-        Xp[0].copy_(Xh, non_blocking=True)
-        step()
-        Yh.copy_(Ys[last[0]], non_blocking=True)
+        host_step()
     a1.record(stream)
     torch.cuda.synchronize()
+    barrier(world)
+    pipe.close()
     e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / n_e2e
+
+    # ------------------------------------------------------------- roofline
+    g_total_ms, q_total_ms = sum(g_ms), sum(q_ms)
+    g_ach = sum(g_ops) / (g_total_ms * 1e-3) / 1e12
+    q_ach = sum(q_bytes) / (q_total_ms * 1e-3) / 1e9
+    nominal_int8 = 4500.0
+    roofline = {
+        "bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": g_ach, "peak": int8_peak,
+        "unit": "TOPS", "frac": g_ach / int8_peak,
+        "traffic": profile_traffic("gemm.cu", f"gemm_{args.workload}"),
+        "peak_note": f"int8 = {INT8_PER_BF16:g} x {peaks['src']} sustained bf16 {peaks['bf16_sus']} TFLOP/s "
+                     "(the kernel runs inside an 80 ms step under the power cap)",
+        "frac_of_nominal_4500": g_ach / nominal_int8,
+        "frac_of_measured_int8_ceiling": (g_ach / ceiling["tops"]) if ceiling.get("tops") else None,
+        "measured_int8_ceiling": ceiling,
+        "ms_per_launch": g_total_ms / len(layers), "launches_per_step": len(layers),
+        "algorithmic_ops_per_launch": sum(g_ops) / len(layers),
+        "timing": "CUDA events on the launching stream around each GEMM launch of one step "
+                  "(time-weighted: sum of ops / sum of launch durations)"}
+    roofline_q = {
+        "bound": "hbm", "kernel": "quantize_rows_kernel", "achieved": q_ach, "peak": peaks["hbm"],
+        "unit": "GB/s", "frac": q_ach / peaks["hbm"],
+        "traffic": profile_traffic("quant.cu", f"quant_{args.workload}"),
+        "ms_per_launch": q_total_ms / len(layers), "algorithmic_bytes_per_launch": sum(q_bytes) / len(layers)}
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "s4xs4->s32 (bf16 in/out, fp32 transform)",
-        "data": "synthetic (activations: seeded heavy-tailed generator; weights: seeded normal on device)",
+        "data": "synthetic (seeded heavy-tailed activations, a fresh batch per layer; seeded normal weights "
+                "per layer; drawn on the device)",
         "tokens_per_s": world * M * args.steps / (elapsed_ms * 1e-3),
         "config": {"workload": st["desc"], "M": M, "blocks": st["blocks"],
                    "layers": [f"{n} {K}->{N}" for (n, K, N) in st["layers"]],
-                   "parallelism": f"dp{world} (independent replicas)"},
+                   "parallelism": f"dp{world} (independent replicas)",
+                   "l2": "every layer reads its own input batch (>= 180 MB, larger than L2)"},
         "clocks": clk.summary(),
         "e2e": {"value": world * ops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": 2 * M * 1024, "d2h_bytes_per_step": 2 * M * last[2],
-                "api": "w4a4_linear_fused per layer; input copied in, last output copied out, same stream"},
+                "h2d_bytes_per_step": 2 * M * layers[0][2], "d2h_bytes_per_step": 2 * M * layers[last][3],
+                "api": f"w4a4_linear_fused_host (C ABI) for the first layer (X from pinned host memory) and "
+                       f"the last (Y to pinned host memory), {chunk}-row chunks; w4a4_linear_fused between"},
         "gpu_launches": 2 * len(layers) * args.steps,
+        "roofline": roofline,
+        "roofline_quantize": roofline_q,
         "per_layer": per_layer,
-        "roofline": {"bound": "tensor", "kernel": "w4a4_gemm_kernel + quantize_rows_kernel (whole stack)",
-                     "achieved": value / world, "peak": int8_peak, "unit": "TOPS",
-                     "frac": value / world / int8_peak, "traffic": None,
-                     "per_layer_kernels": "per_layer.*.gemm_frac: the GEMM alone per layer shape "
-                                          f"({n_iso} back-to-back launches, int8 peak = 2 x measured bf16 burst)"},
+        "dsfq_overhead": {"dsfq_ms_per_step": m7["dsfq"], "plain_ms_per_step": m7["plain"],
+                          "overhead_pct": 100.0 * (m7["dsfq"] - m7["plain"]) / m7["plain"],
+                          "pages_figure_pct": 0.2,
+                          "how": f"fused call per layer shape, {n_iso} calls each, x {st['blocks']} blocks"},
         "device_status": status,
     }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        tops, tps, r, passes, t_block, cores = time_stack_oracle(st, 1024, budget_s=10.0)
+        line["cpu_baseline"] = {
+            "value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle", "tokens_per_s": tps,
+            "sample": f"sampled, per-token rate: {r} token rows (special tokens included) through one "
+                      f"block's four layer shapes, {passes} passes, {t_block:.2f} s per pass; the stack is "
+                      f"{st['blocks']} blocks of it"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -859,16 +1085,22 @@ def run_tq_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 20 for the multi-layer workloads, 2000 otherwise)")
+    ap.add_argument("--warmup", type=int, default=None, help="warm-up steps (default: 3 / 20)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(STACKS) + [TQ_WORKLOAD],
-                    default="c2_frame_qkv")
+                    default="c5_full_stack")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--e2e-chunk", type=int, default=1408, help="row chunk of the host-buffer call")
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    multi = args.workload in STACKS
+    if args.steps is None:
+        args.steps = 20 if multi else 2000
+    if args.warmup is None:
+        args.warmup = 3 if multi else 20
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -887,10 +1119,7 @@ def main():
         return
     if args.workload in STACKS:
         if args.impl == "reference":
-            if rank == 0:
-                print(json.dumps({"impl": "reference", "unavailable":
-                                  "multi-layer workloads are timed on the GPU only; the oracle "
-                                  "reference arm covers the single-layer workloads"}), flush=True)
+            run_stack_reference(args, STACKS[args.workload], world, rank)
             return
         world, rank, local = dist_setup()
         try:

@@ -301,15 +301,23 @@ w4a4_status w4a4_host_pipe_destroy(w4a4_host_pipe_t *pipe);
  * aligned. */
 size_t w4a4_host_workspace_bytes(int64_t chunk_rows, int32_t K, int32_t N);
 
+/* Flags of w4a4_linear_fused_host only: X_host (W4A4_FLAG_X_DEVICE) or Y_host
+ * (W4A4_FLAG_Y_DEVICE) is a device pointer (16-byte aligned) instead, read or
+ * written in place without copies -- the first or last layer of a stack whose
+ * other layers run on the device. */
+#define W4A4_FLAG_X_DEVICE 0x20u
+#define W4A4_FLAG_Y_DEVICE 0x40u
+
 /* Y_host [M, N] bf16 = w4a4_linear_fused(X_host [M, K] bf16) with X_host and
  * Y_host in host memory (page-locked memory for the copies to overlap; pageable
- * memory works but serializes).  workspace: device memory of at least
+ * memory works but serializes), unless flagged as device memory above.  workspace: device memory of at least
  * w4a4_host_workspace_bytes(chunk_rows, w->K, w->N) bytes, 16-byte aligned;
  * chunk_rows > 0 (a multiple of 128 uses whole GEMM tiles).  The call enqueues
  * the work and returns; `stream` (the compute stream; NULL = legacy default
  * stream) is made to wait for the last copy, so work enqueued on it afterwards,
  * or a synchronize of it, sees Y_host complete.  Flags and errors as
- * w4a4_linear_fused; M = 0 is a no-op. */
+ * w4a4_linear_fused, plus W4A4_FLAG_X_DEVICE / W4A4_FLAG_Y_DEVICE; M = 0 is a
+ * no-op. */
 w4a4_status w4a4_linear_fused_host(const uint16_t *X_host, int64_t M, const w4a4_weights_t *w,
                                    uint16_t *Y_host, int64_t chunk_rows, void *workspace,
                                    size_t workspace_bytes, w4a4_host_pipe_t *pipe,

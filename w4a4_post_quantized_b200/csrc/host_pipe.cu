@@ -98,6 +98,14 @@ extern "C" w4a4_status w4a4_linear_fused_host(const uint16_t *X_host, int64_t M,
   if (workspace_bytes < w4a4_host_workspace_bytes(chunk_rows, w->K, w->N)) return W4A4_ERR_SHAPE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != pipe->device) return W4A4_ERR_ARG;
+  // X or Y may stay in device memory (the first or last layer of a stack run
+  // on the device): that side's copies are skipped and the kernels read X /
+  // write Y in place
+  const bool x_dev = (flags & W4A4_FLAG_X_DEVICE) != 0, y_dev = (flags & W4A4_FLAG_Y_DEVICE) != 0;
+  flags &= ~(W4A4_FLAG_X_DEVICE | W4A4_FLAG_Y_DEVICE);
+  if ((x_dev && (reinterpret_cast<uintptr_t>(X_host) & 15) != 0) ||
+      (y_dev && (reinterpret_cast<uintptr_t>(Y_host) & 15) != 0))
+    return W4A4_ERR_ALIGN;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int64_t nchunks = (M + chunk_rows - 1) / chunk_rows;
   // the copy-in stream starts after everything already enqueued on `stream`
@@ -112,30 +120,37 @@ extern "C" w4a4_status w4a4_linear_fused_host(const uint16_t *X_host, int64_t M,
     const int64_t r0 = c * chunk_rows;
     const int64_t rows = (M - r0 < chunk_rows) ? M - r0 : chunk_rows;
     const Slot sl = slot_of(workspace, chunk_rows, w->K, w->N, i);
-    // X chunk in: its slot's X buffer was last read by compute of chunk c - DEPTH
-    if (c >= W4A4_PIPE_DEPTH && cudaStreamWaitEvent(pipe->copy_in, pipe->ev_done[i], 0) != cudaSuccess)
+    const uint16_t *x = x_dev ? X_host + r0 * w->K : sl.x;
+    uint16_t *y = y_dev ? Y_host + r0 * w->N : sl.y;
+    if (!x_dev) {
+      // X chunk in: its slot's X buffer was last read by compute of chunk c - DEPTH
+      if (c >= W4A4_PIPE_DEPTH && cudaStreamWaitEvent(pipe->copy_in, pipe->ev_done[i], 0) != cudaSuccess)
+        return W4A4_ERR_CUDA;
+      if (cudaMemcpyAsync(sl.x, X_host + r0 * w->K, static_cast<size_t>(rows) * w->K * 2,
+                          cudaMemcpyHostToDevice, pipe->copy_in) != cudaSuccess ||
+          cudaEventRecord(pipe->ev_in[i], pipe->copy_in) != cudaSuccess)
+        return W4A4_ERR_CUDA;
+      // compute needs the X chunk
+      if (cudaStreamWaitEvent(cs, pipe->ev_in[i], 0) != cudaSuccess) return W4A4_ERR_CUDA;
+    }
+    // ... and the slot's Y buffer drained by copy-out of chunk c - DEPTH
+    if (!y_dev && c >= W4A4_PIPE_DEPTH && cudaStreamWaitEvent(cs, pipe->ev_out[i], 0) != cudaSuccess)
       return W4A4_ERR_CUDA;
-    if (cudaMemcpyAsync(sl.x, X_host + r0 * w->K, static_cast<size_t>(rows) * w->K * 2,
-                        cudaMemcpyHostToDevice, pipe->copy_in) != cudaSuccess ||
-        cudaEventRecord(pipe->ev_in[i], pipe->copy_in) != cudaSuccess)
-      return W4A4_ERR_CUDA;
-    // compute: needs the X chunk, and the slot's Y buffer drained by copy-out of chunk c - DEPTH
-    if (cudaStreamWaitEvent(cs, pipe->ev_in[i], 0) != cudaSuccess) return W4A4_ERR_CUDA;
-    if (c >= W4A4_PIPE_DEPTH && cudaStreamWaitEvent(cs, pipe->ev_out[i], 0) != cudaSuccess)
-      return W4A4_ERR_CUDA;
-    const w4a4_status s = w4a4_linear_fused(sl.x, rows, w, sl.y, sl.ws, sl.ws_bytes, flags, cs);
+    const w4a4_status s = w4a4_linear_fused(x, rows, w, y, sl.ws, sl.ws_bytes, flags, cs);
     if (s != W4A4_OK) return s;
     if (cudaEventRecord(pipe->ev_done[i], cs) != cudaSuccess) return W4A4_ERR_CUDA;
     // Y chunk out
-    if (cudaStreamWaitEvent(pipe->copy_out, pipe->ev_done[i], 0) != cudaSuccess ||
-        cudaMemcpyAsync(Y_host + r0 * w->N, sl.y, static_cast<size_t>(rows) * w->N * 2,
-                        cudaMemcpyDeviceToHost, pipe->copy_out) != cudaSuccess ||
-        cudaEventRecord(pipe->ev_out[i], pipe->copy_out) != cudaSuccess)
+    if (!y_dev &&
+        (cudaStreamWaitEvent(pipe->copy_out, pipe->ev_done[i], 0) != cudaSuccess ||
+         cudaMemcpyAsync(Y_host + r0 * w->N, sl.y, static_cast<size_t>(rows) * w->N * 2,
+                         cudaMemcpyDeviceToHost, pipe->copy_out) != cudaSuccess ||
+         cudaEventRecord(pipe->ev_out[i], pipe->copy_out) != cudaSuccess))
       return W4A4_ERR_CUDA;
   }
   // `stream` sees the call complete once the last copy-out has finished (the
-  // copy-out stream is in order, so its latest event covers every chunk)
+  // copy-out stream is in order, so its latest event covers every chunk); with
+  // Y in device memory the kernels on `stream` are the last work
   const int last = static_cast<int>((nchunks - 1) % W4A4_PIPE_DEPTH);
-  if (cudaStreamWaitEvent(cs, pipe->ev_out[last], 0) != cudaSuccess) return W4A4_ERR_CUDA;
+  if (!y_dev && cudaStreamWaitEvent(cs, pipe->ev_out[last], 0) != cudaSuccess) return W4A4_ERR_CUDA;
   return W4A4_OK;
 }

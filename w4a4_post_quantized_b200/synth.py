@@ -64,6 +64,38 @@ def activations(M: int, K: int, seed: int, heavy_tailed: bool = True) -> np.ndar
     return to_bf16_bits(x)
 
 
+def activations_device(M: int, K: int, seed: int, device, heavy_tailed: bool = True):
+    """The same recipe as activations() drawn on a CUDA device with torch's
+    generator (other random numbers, same distribution and structure): a
+    torch.bfloat16 tensor [M, K].  For workloads whose inputs are too large to
+    draw on the host (a fresh activation batch for each of a stack's layers)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 7919 + 0xA11)
+    x = torch.randn((M, K), generator=g, device=device, dtype=torch.float32)
+    if heavy_tailed:
+        rows = torch.from_numpy(special_rows(M)).to(device)
+        x[rows] *= SPECIAL_SCALE
+        x[:, torch.from_numpy(outlier_channels(K, seed)).to(device)] *= OUTLIER_SCALE
+    return x.to(torch.bfloat16)
+
+
+def weights_device(N: int, K: int, seed: int, device, std: float = 0.02):
+    """weights() drawn on a CUDA device (torch's generator): bf16 [N, K]."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 7919 + 0x3E1)
+    return (torch.randn((N, K), generator=g, device=device) * std).to(torch.bfloat16)
+
+
+def bias_device(N: int, seed: int, device, std: float = 0.01):
+    """bias() drawn on a CUDA device (torch's generator): bf16 [N]."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 7919 + 0xB1A5)
+    return (torch.randn(N, generator=g, device=device) * std).to(torch.bfloat16)
+
+
 def weights(N: int, K: int, seed: int, std: float = 0.02) -> np.ndarray:
     rng = np.random.Generator(np.random.PCG64([seed, 0x3E1]))
     return to_bf16_bits(rng.standard_normal((N, K), dtype=np.float32) * np.float32(std))

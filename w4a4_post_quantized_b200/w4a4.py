@@ -30,6 +30,8 @@ W4A4_FLAG_PLAIN = 0x2
 W4A4_FLAG_INT8 = 0x4
 W4A4_FLAG_UNPACKED = 0x8
 W4A4_FLAG_GELU_OUT = 0x10
+W4A4_FLAG_X_DEVICE = 0x20
+W4A4_FLAG_Y_DEVICE = 0x40
 W4A4_DEBUG_STALL = 0x80000000
 
 _vp, _i32, _i64, _u32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
@@ -264,7 +266,9 @@ def w4a4_linear_fused_host(X_host: torch.Tensor, w: PreparedWeights, Y_host=None
     concurrently.  Returns Y_host (enqueued: synchronize `stream` before reading)."""
     M = X_host.shape[0]
     if Y_host is None:  # a convenience of this binding only
-        Y_host = torch.empty((M, w.N), dtype=torch.bfloat16, pin_memory=True)
+        Y_host = (torch.empty((M, w.N), dtype=torch.bfloat16, device=w.device)
+                  if flags & W4A4_FLAG_Y_DEVICE else
+                  torch.empty((M, w.N), dtype=torch.bfloat16, pin_memory=True))
     if workspace is None:
         workspace = torch.empty(w4a4_host_workspace_bytes(chunk_rows, w.K, w.N), dtype=torch.uint8,
                                 device=w.device)
