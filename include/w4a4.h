@@ -109,6 +109,19 @@ typedef enum {
                                  section 视觉几何基础 Transformer（VGGT）, with its
                                  activation placed where it costs least). */
 
+#define W4A4_FLAG_FWHT 0x100u  /* quantize_act / linear_fused: rotate the activations
+                                 with the CUDA-core fast Walsh-Hadamard transform
+                                 instead of the tensor cores.  The same method either
+                                 way ([ROT]: x H / sqrt(K)); the two differ only in
+                                 fp32 rounding, so codes may differ at rounding ties.
+                                 By default the DSFQ path (no W4A4_FLAG_PLAIN, no
+                                 W4A4_FLAG_GELU) uses the tensor cores, via
+                                 H_K = H_R (x) H_R with R = sqrt(K): a bf16 product
+                                 (exact inputs, fp32 sums) then a tf32 product of the
+                                 fp32 intermediate split into two tf32 terms;
+                                 W4A4_FLAG_PLAIN has no rotation and W4A4_FLAG_GELU
+                                 inputs use the CUDA-core transform. */
+
 /* Prepared weights of one linear layer.  The caller allocates every array
  * (device memory) with the sizes given and keeps ownership. */
 typedef struct {

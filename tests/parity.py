@@ -1,7 +1,8 @@
 """Comparison rules shared by the GPU parity tests.
 
 Integer codes.  The CUDA path forms each rotated value in binary32 (an fp32
-transform of the bf16 inputs), multiplies it by the binary32 reciprocal step
+transform of the bf16 inputs, on the tensor cores or the CUDA cores: see
+tie_bound), multiplies it by the binary32 reciprocal step
 qmax/absmax and rounds the exact product half to even.  The oracle is compared
 in two modes:
   * decision="f64" -- the method as the pages define it: exact fp64 rotation,
@@ -18,10 +19,20 @@ the oracle's only
 Everything else must be bit-exact.
 
 tie_bound, the bound on |ratio_gpu - ratio_oracle| (u = 2^-24):
-  * the rotated value: a +-sum of K inputs formed through log2(K) rounding
-    levels, so its absolute error is at most e_val = log2(K) u sum_i|x_i| /
-    sqrt(K), times the largest multiplier; in the ratio that is
-    e_ratio = qmax e_val / absmax;
+  * the rotated value, e_val = c * sum_i|x_i| / sqrt(K) times the largest
+    multiplier, with c fixed by the transform that formed it:
+      - "fwht", the CUDA-core fast Walsh-Hadamard transform: a +-sum of K
+        inputs formed through log2(K) round-to-nearest levels, c = log2(K) u;
+      - "tc", the tensor-core product through H_K = H_R (x) H_R (R = sqrt K):
+        stage 1 sums R exact products in fp32 on the tensor cores, stage 2
+        sums 2R products of the two tf32 terms of each intermediate value,
+        whose sum is within 2^-22 of it.  The summation order and rounding
+        inside the tensor core are not specified, so each sum of n terms is
+        bounded as n sequential additions that may each lose a full unit in
+        the last place (2u) of the running sum: c = (R + 2R) 2u + 2^-22, i.e.
+        (3R + 1/2) 2^-23 (stage-1 errors pass through stage 2 unchanged in
+        size: its coefficients are +-1);
+    in the ratio that is e_ratio = qmax e_val / absmax;
   * the absmax is one of those values, so it carries the same absolute error
     e_val; through the reciprocal step it moves every ratio of the row by at
     most |ratio| e_val / absmax <= e_ratio;
@@ -36,13 +47,24 @@ import numpy as np
 U = 2.0 ** -24
 
 
+def transform_error_coefficient(K: int, transform: str) -> float:
+    """c in e_val = c * sum|x| / sqrt(K) (module docstring)."""
+    if transform == "fwht":
+        return np.log2(K) * U
+    if transform == "tc":
+        R = int(round(np.sqrt(K)))
+        return (3 * R + 0.5) * 2.0 ** -23
+    raise ValueError(transform)
+
+
 def tie_bound(x_in: np.ndarray, mult: np.ndarray, ratio: np.ndarray, amax: np.ndarray, K: int,
-              qmax: float = 7.0) -> np.ndarray:
+              qmax: float = 7.0, transform: str = "fwht") -> np.ndarray:
     """Per-row bound on |ratio_cuda - ratio_exact| (rows of x_in are the
     transform's inputs, mult the per-channel multipliers, qmax the largest
-    code: 7 for int4, 127 for int8)."""
+    code: 7 for int4, 127 for int8; transform: "fwht" or "tc", the kernel
+    that rotated the values)."""
     l1 = np.sum(np.abs(x_in), axis=1)
-    e_val = np.log2(K) * U * l1 / np.sqrt(K) * np.max(np.abs(mult))
+    e_val = transform_error_coefficient(K, transform) * l1 / np.sqrt(K) * np.max(np.abs(mult))
     with np.errstate(divide="ignore", invalid="ignore"):
         e_ratio = np.where(amax > 0, qmax * e_val / amax, 0.0)
     rmax = np.max(np.abs(ratio), axis=1)
@@ -73,3 +95,11 @@ def rel_fro(got, want) -> float:
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
     return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
+
+
+def act_transform(flags: int) -> str:
+    """Which kernel rotated the activations for these w4a4_quantize_act /
+    w4a4_linear_fused flags: the tensor cores for DSFQ without GELU, unless
+    W4A4_FLAG_FWHT (0x100); the CUDA-core transform otherwise."""
+    plain, gelu, fwht = flags & 0x2, flags & 0x1, flags & 0x100
+    return "tc" if not (plain or gelu or fwht) else "fwht"

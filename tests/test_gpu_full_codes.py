@@ -19,7 +19,7 @@ import torch
 
 import oracle
 from w4a4_post_quantized_b200 import synth
-from parity import compare_codes, tie_bound
+from parity import act_transform, compare_codes, tie_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -47,7 +47,7 @@ def test_fwht_helper_matches_the_oracle_rotation():
     np.testing.assert_allclose(fwht_rows(X) / 32.0, oracle.rotate(X), rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("frames,K,gelu", [(32, 1024, False), (8, 4096, True)])
+@pytest.mark.parametrize("frames,K,gelu", [(32, 1024, False), (8, 4096, True), (8, 4096, False)])
 def test_every_code_of_a_large_batch(w4, frames, K, gelu):
     M = frames * synth.FRAME_TOKENS
     X = synth.activations(M, K, seed=900 + K)
@@ -63,7 +63,7 @@ def test_every_code_of_a_large_batch(w4, frames, K, gelu):
     amax = np.max(np.abs(hat), axis=1)
     with np.errstate(divide="ignore", invalid="ignore"):
         ratio = np.where(amax[:, None] > 0, hat * 7.0 / amax[:, None], 0.0)
-    bound = tie_bound(xin, inv_s.astype(np.float64), ratio, amax, K)
+    bound = tie_bound(xin, inv_s.astype(np.float64), ratio, amax, K, transform=act_transform(flags))
     if gelu:  # GELU in fp32 may land one bf16 step away from the fp64 GELU
         bound = bound + 4.0 * 2.0 ** -8 * np.max(np.abs(xin), axis=1) * np.max(inv_s) / np.sqrt(K) * 7.0 / np.maximum(amax, 1e-300)
     # the method as defined (fp64 decision), then the binary32 decision
@@ -71,6 +71,7 @@ def test_every_code_of_a_large_batch(w4, frames, K, gelu):
         want_q, want_d = oracle.quantize_rows(hat, 4, decision)
         np.testing.assert_allclose(st, want_d, rtol=2e-5, atol=0)
         flips = compare_codes(got, want_q, ratio, bound, 1e-4)
-        print(f"M={M} K={K} gelu={gelu}: {flips} flips of {got.size} against the {decision} decision")
+        print(f"M={M} K={K} gelu={gelu} ({act_transform(flags)}): {flips} flips of {got.size} "
+              f"against the {decision} decision")
         del want_q
     assert w4.w4a4_get_device_status() == 0

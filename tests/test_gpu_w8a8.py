@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from w4a4_post_quantized_b200 import synth
-from parity import compare_codes, rel_fro, tie_bound
+from parity import act_transform, compare_codes, rel_fro, tie_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -124,7 +124,7 @@ def test_quantize_act_int8_parity(w4, M, K, plain):
         ratio = np.where(amax[:, None] > 0, hat * 127.0 / amax[:, None], 0.0)
     xin = oracle.bf16_to_f64(X)
     mult = np.ones(K) if plain else 1.0 / s
-    bound = tie_bound(xin, mult, ratio, amax, K, qmax=127.0)
+    bound = tie_bound(xin, mult, ratio, amax, K, qmax=127.0, transform=act_transform(flags))
     compare_codes(got, want_q, ratio, bound, 1e-4 if M * K >= 10 ** 5 else None)
 
 

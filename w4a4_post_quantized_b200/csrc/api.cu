@@ -11,10 +11,11 @@
 
 namespace {
 
-constexpr uint32_t kKnownFlags =
-    W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED | W4A4_FLAG_GELU_OUT;
+constexpr uint32_t kKnownFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 |
+                                 W4A4_FLAG_UNPACKED | W4A4_FLAG_GELU_OUT | W4A4_FLAG_FWHT;
 // flags of the activation quantizer (w4a4_quantize_act and the workspace sizes)
-constexpr uint32_t kActFlags = W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED;
+constexpr uint32_t kActFlags =
+    W4A4_FLAG_GELU | W4A4_FLAG_PLAIN | W4A4_FLAG_INT8 | W4A4_FLAG_UNPACKED | W4A4_FLAG_FWHT;
 constexpr uint32_t kWeightFlags = W4A4_FLAG_PLAIN | W4A4_FLAG_INT8;  // fixed at preparation
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -53,6 +54,18 @@ bool one_per_byte(uint32_t flags) { return (flags & (W4A4_FLAG_INT8 | W4A4_FLAG_
 size_t code_bytes(int64_t M, int32_t K, uint32_t flags) {
   return static_cast<size_t>(M) * (one_per_byte(flags) ? K : K / 2);
 }
+// The activation quantizer for these flags: the rotation on the tensor cores
+// (quant_tc.cu) for DSFQ without GELU, unless W4A4_FLAG_FWHT asks for the
+// CUDA-core transform; the CUDA-core kernel (quant.cu) otherwise.
+cudaError_t quantize_rows(const uint16_t *X, int64_t M, int32_t K, const float *inv_smooth,
+                          uint8_t *qx, float *scale_tok, uint32_t flags, w4a4::CodeFormat fmt,
+                          cudaStream_t st) {
+  const bool rot = !(flags & W4A4_FLAG_PLAIN), gelu = (flags & W4A4_FLAG_GELU) != 0;
+  if (rot && !gelu && !(flags & W4A4_FLAG_FWHT))
+    return w4a4::launch_quantize_rows_tc(X, M, K, inv_smooth, qx, scale_tok, fmt, st);
+  return w4a4::launch_quantize_rows(X, M, K, inv_smooth, qx, scale_tok, rot, gelu, fmt, st);
+}
+
 w4a4::CodeFormat code_format(uint32_t flags) {
   if (flags & W4A4_FLAG_INT8) return w4a4::kCodeBytes8;
   return (flags & W4A4_FLAG_UNPACKED) ? w4a4::kCodeBytes4 : w4a4::kCodePacked4;
@@ -212,10 +225,8 @@ w4a4_status w4a4_quantize_act(const uint16_t *X, int64_t M, int32_t K, const flo
   if ((flags & W4A4_FLAG_INT8) && (flags & W4A4_FLAG_UNPACKED)) return W4A4_ERR_UNSUPPORTED;
   w4a4_status s = check_act(X, M, K, inv_smooth, qx, scale_tok, flags);
   if (s != W4A4_OK) return s;
-  return cuda_status(w4a4::launch_quantize_rows(X, M, K, inv_smooth, qx, scale_tok,
-                                                !(flags & W4A4_FLAG_PLAIN),
-                                                (flags & W4A4_FLAG_GELU) != 0, code_format(flags),
-                                                as_stream(stream)));
+  return cuda_status(quantize_rows(X, M, K, inv_smooth, qx, scale_tok, flags, code_format(flags),
+                                   as_stream(stream)));
 }
 
 w4a4_status w4a4_linear_ex(const uint8_t *qx, const float *scale_tok, int64_t M,
@@ -263,9 +274,7 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
   uint8_t *qx = static_cast<uint8_t *>(workspace);
   float *st = reinterpret_cast<float *>(qx + round256(code_bytes(M, w->K, cf)));
   cudaStream_t cs = as_stream(stream);
-  cudaError_t e = w4a4::launch_quantize_rows(X, M, w->K, w->inv_smooth, qx, st,
-                                             !(flags & W4A4_FLAG_PLAIN),
-                                             (flags & W4A4_FLAG_GELU) != 0, code_format(cf), cs);
+  cudaError_t e = quantize_rows(X, M, w->K, w->inv_smooth, qx, st, flags, code_format(cf), cs);
   if (e != cudaSuccess) return cuda_status(e);
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, st, w->scale_ch, w->bias, Y, nullptr,
                    M, w->N, w->K, one_per_byte(cf), (flags & W4A4_FLAG_GELU_OUT) != 0};

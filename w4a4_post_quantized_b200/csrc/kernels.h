@@ -2,6 +2,7 @@
 // kernel translation units.  Not part of the public interface.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap types (the encode function is fetched at run time)
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -47,6 +48,19 @@ struct GemmArgs {
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,
                                   cudaStream_t st);
+
+// A 2-D TMA tensor map (cuTensorMapEncodeTiled through the runtime's driver
+// entry point): `outer` rows of `inner` elements, rows `row_bytes` apart, box
+// box_inner x box_outer, no interleave, 256-byte L2 promotion, zero fill.
+bool encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                          uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                          CUtensorMapSwizzle swz);
+
+// quant_tc.cu: the activation quantizer with the rotation on the tensor cores
+// (DSFQ: rotation and smoothing on; no GELU).  Same arguments and outputs as
+// launch_quantize_rows with rot = true, gelu = false.
+cudaError_t launch_quantize_rows_tc(const uint16_t *X, int64_t M, int K, const float *mult,
+                                    uint8_t *q, float *scale, CodeFormat code, cudaStream_t st);
 
 // status word: *out = its device address in the current context (for kernel
 // arguments); an error when the lookup fails (nothing may then be launched)

@@ -290,6 +290,59 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of a swizzled operand tile in any of the
+// canonical layouts (K-major or MN-major; the instruction descriptor says
+// which): start address, leading and stride byte offsets (multiples of 16),
+// descriptor version 1 (sm_100) and the swizzle mode, 2 = 128-byte, 4 = 64-byte.
+//   K-major:  rows of the swizzle width along K; 8-row groups `sbo` apart
+//             (lbo unused).
+//   MN-major: atoms of the swizzle width along M (or N) by 8 rows along K;
+//             atoms `lbo` apart along M (N), 8-row K groups `sbo` apart.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (static_cast<uint64_t>(1u) << 46) |
+         (static_cast<uint64_t>(layout & 7u) << 61);
+}
+constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4;
+
+// D[tmem] (+)= A[smem desc] x B[smem desc]^T with 16-bit floating-point
+// inputs (kind::f16; A and B of the same type, given by the instruction
+// descriptor) and fp32 accumulators.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same with tf32 inputs (kind::tf32), fp32 accumulators.
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of kind::f16 (bf16 A and B) or kind::tf32, fp32
+// accumulators, A MN-major when A_MN (else K-major), B K-major, M x N tile.
+template <int M, int N, bool TF32, bool A_MN>
+__host__ __device__ constexpr uint32_t idesc_f32acc() {
+  return (1u << 4)                                    // D format: f32
+         | ((TF32 ? 2u : 1u) << 7)                    // A format: tf32 / bf16
+         | ((TF32 ? 2u : 1u) << 10)                   // B format: tf32 / bf16
+         | ((A_MN ? 1u : 0u) << 15)                   // A major-ness
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
 // Instruction descriptor of tcgen05.mma kind::i8: s32 accumulators, signed
 // 8-bit A and B, both K-major, M x N tile.
 template <int M, int N>

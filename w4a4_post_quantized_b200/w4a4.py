@@ -31,6 +31,7 @@ W4A4_FLAG_INT8 = 0x4
 W4A4_FLAG_UNPACKED = 0x8
 W4A4_FLAG_GELU_OUT = 0x10
 W4A4_FLAG_X_DEVICE = 0x20
+W4A4_FLAG_FWHT = 0x100
 W4A4_FLAG_Y_DEVICE = 0x40
 W4A4_DEBUG_STALL = 0x80000000
 
