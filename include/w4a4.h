@@ -116,11 +116,11 @@ typedef enum {
                                  fp32 rounding, so codes may differ at rounding ties.
                                  By default the DSFQ path (no W4A4_FLAG_PLAIN, no
                                  W4A4_FLAG_GELU) uses the tensor cores, via
-                                 H_K = H_R (x) H_R with R = sqrt(K): a bf16 product
-                                 (exact inputs, fp32 sums) then a tf32 product of the
-                                 fp32 intermediate split into two tf32 terms;
-                                 W4A4_FLAG_PLAIN has no rotation and W4A4_FLAG_GELU
-                                 inputs use the CUDA-core transform. */
+                                 H_K = H_128 (x) H_(K/128): the 128-point factor as a
+                                 bf16 product (exact inputs, fp32 sums), the small
+                                 factor in fp32 registers; W4A4_FLAG_PLAIN has no
+                                 rotation and W4A4_FLAG_GELU inputs use the CUDA-core
+                                 transform. */
 
 /* Prepared weights of one linear layer.  The caller allocates every array
  * (device memory) with the sizes given and keeps ownership. */

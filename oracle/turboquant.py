@@ -14,10 +14,17 @@ Models" (gist.science), technical summary:
              times" the information-theoretic 4^-b (section 2.1).
   [TQ-KV]    section 4.2: the DUSt3R KV cache, d = 1024, b = 4, 7.9x smaller.
 
-Readings (the page prints no codebook, no rotation recipe beyond "QR of a
-Gaussian matrix", and no storage format):
-  * Pi = H diag(s) / sqrt(d), H the Sylvester Hadamard matrix, s a seeded random
-    sign vector: an orthogonal matrix applied in O(d log d); s is an input.
+Readings (the page prints no codebook, no storage format, and of the
+rotation only that it is a random orthogonal matrix obtained by QR of a
+Gaussian matrix):
+  * Pi = Q diag(sign(diag(R))) for the QR factorisation G = Q R of a d x d
+    matrix G of independent standard normal entries (an input, seeded): the
+    sign fix makes the factorisation unique (R with a positive diagonal), and
+    Pi is then Haar-distributed (rotation_qr).
+  * a fast variant, not the page's matrix: Pi = H diag(s) / sqrt(d), H the
+    Sylvester Hadamard matrix, s a seeded random sign vector -- orthogonal and
+    applied in O(d log d) (rotation); the codec kernels offer it beside the
+    dense Pi, and it is judged only on the MSE bound and the distortion.
   * the coordinate density of a uniformly random unit vector:
     f(x) = Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2)) (1 - x^2)^((d-3)/2) on [-1, 1]
     ((x + 1)/2 ~ Beta((d-1)/2, (d-1)/2)).
@@ -116,31 +123,49 @@ def distortion(d: int, centroids, boundaries) -> float:
     return total
 
 
+def rotation_qr(G) -> np.ndarray:
+    """[TQ-FLOW] the page's random orthogonal matrix: Pi = Q diag(sign(diag R))
+    for G = Q R (numpy's Householder QR, LAPACK), G a d x d Gaussian matrix."""
+    G = np.asarray(G, dtype=np.float64)
+    Q, R = np.linalg.qr(G)
+    sg = np.sign(np.diag(R))
+    sg[sg == 0] = 1.0
+    return Q * sg[None, :]
+
+
 def rotation(signs) -> np.ndarray:
-    """[TQ-FLOW] Pi = H diag(s) / sqrt(d) (reading: a seeded random orthogonal matrix)."""
+    """The fast variant's orthogonal matrix Pi = H diag(s) / sqrt(d) (not the
+    page's: see the module docstring)."""
     s = np.asarray(signs, dtype=np.float64)
     d = s.shape[0]
     return hadamard(d) * s[None, :] / math.sqrt(d)
 
 
-def encode(X, signs, boundaries):
+def _as_rotation(Pi_or_signs) -> np.ndarray:
+    a = np.asarray(Pi_or_signs, dtype=np.float64)
+    return rotation(a) if a.ndim == 1 else a
+
+
+def encode(X, Pi, boundaries):
     """[TQ-FLOW] gamma = ||x||, y = Pi x / gamma, code = #{boundaries < y}.
+    Pi: the rotation matrix [d, d] (rotation_qr), or a sign vector [d] for the
+    fast variant's H diag(s) / sqrt(d).
     Returns (codes uint8 [n, d], gamma [n], y [n, d])."""
     X = np.asarray(X, dtype=np.float64)
     gamma = np.sqrt(np.sum(X * X, axis=1))
-    Pi = rotation(signs)
+    P = _as_rotation(Pi)
     with np.errstate(divide="ignore", invalid="ignore"):
         U = np.where(gamma[:, None] > 0, X / gamma[:, None], 0.0)
-    Y = U @ Pi.T
+    Y = U @ P.T
     codes = np.searchsorted(np.asarray(boundaries, np.float64), Y, side="left").astype(np.uint8)
     return codes, gamma, Y
 
 
-def decode(codes, gamma, signs, centroids):
-    """[TQ-FLOW] theta~ = gamma * Pi^T * centroids[codes]."""
-    Pi = rotation(signs)
+def decode(codes, gamma, Pi, centroids):
+    """[TQ-FLOW] theta~ = gamma * Pi^T * centroids[codes] (Pi as for encode)."""
+    P = _as_rotation(Pi)
     Yq = np.asarray(centroids, np.float64)[np.asarray(codes, np.int64)]
-    return np.asarray(gamma, np.float64)[:, None] * (Yq @ Pi)
+    return np.asarray(gamma, np.float64)[:, None] * (Yq @ P)
 
 
 def pack4(codes) -> np.ndarray:

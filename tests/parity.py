@@ -23,15 +23,14 @@ tie_bound, the bound on |ratio_gpu - ratio_oracle| (u = 2^-24):
     multiplier, with c fixed by the transform that formed it:
       - "fwht", the CUDA-core fast Walsh-Hadamard transform: a +-sum of K
         inputs formed through log2(K) round-to-nearest levels, c = log2(K) u;
-      - "tc", the tensor-core product through H_K = H_R (x) H_R (R = sqrt K):
-        stage 1 sums R exact products in fp32 on the tensor cores, stage 2
-        sums 2R products of the two tf32 terms of each intermediate value,
-        whose sum is within 2^-22 of it.  The summation order and rounding
-        inside the tensor core are not specified, so each sum of n terms is
-        bounded as n sequential additions that may each lose a full unit in
-        the last place (2u) of the running sum: c = (R + 2R) 2u + 2^-22, i.e.
-        (3R + 1/2) 2^-23 (stage-1 errors pass through stage 2 unchanged in
-        size: its coefficients are +-1);
+      - "tc", the tensor-core kernel through H_K = H_128 (x) H_S
+        (S = K / 128): the tensor cores sum 128 exact +-products in fp32,
+        then log2(S) round-to-nearest butterfly levels finish in registers.
+        The summation order and rounding inside the tensor core are not
+        specified, so its sum of 128 terms is bounded as 128 sequential
+        additions that may each lose a full unit in the last place (2u) of
+        the running sum; its errors pass through the +-1 butterflies
+        unchanged in size: c = (256 + log2 S) u;
     in the ratio that is e_ratio = qmax e_val / absmax;
   * the absmax is one of those values, so it carries the same absolute error
     e_val; through the reciprocal step it moves every ratio of the row by at
@@ -52,8 +51,7 @@ def transform_error_coefficient(K: int, transform: str) -> float:
     if transform == "fwht":
         return np.log2(K) * U
     if transform == "tc":
-        R = int(round(np.sqrt(K)))
-        return (3 * R + 0.5) * 2.0 ** -23
+        return (256 + np.log2(K // 128)) * U
     raise ValueError(transform)
 
 

@@ -122,3 +122,68 @@ def test_mse_of_random_directions_matches_the_quantizer_and_the_bound(b):
     assert rel.mean() <= tq.mse_bound(b)
     # fewer bits, more error: the bound and the distortion both fall by about 4 per bit
     assert 3.0 < (tq.distortion(d, *tq.lloyd_max(d, b - 1)) * d) / D < 4.5
+
+
+def test_qr_rotation_is_the_sign_fixed_q_factor():
+    """rotation_qr(G) is orthogonal and is the Q of the unique QR
+    factorisation of G with a positive diagonal in R: Pi^T G is upper
+    triangular with a positive diagonal, and Pi (Pi^T G) = G."""
+    from w4a4_post_quantized_b200 import synth
+    d = 256
+    G = synth.gaussian_matrix(d, seed=5)
+    P = tq.rotation_qr(G)
+    np.testing.assert_allclose(P @ P.T, np.eye(d), atol=1e-12)
+    R = P.T @ G
+    assert np.max(np.abs(np.tril(R, -1))) < 1e-11 * np.max(np.abs(R))
+    assert np.all(np.diag(R) > 0)
+    np.testing.assert_allclose(P @ np.triu(R), G, atol=1e-11)
+    # a Householder QR written out here (not LAPACK's) gives the same matrix
+    A = G.copy()
+    Q = np.eye(d)
+    for k in range(d - 1):
+        x = A[k:, k].copy()
+        v = x.copy()
+        v[0] += math.copysign(np.linalg.norm(x), x[0])
+        v /= np.linalg.norm(v)
+        A[k:, :] -= 2.0 * np.outer(v, v @ A[k:, :])
+        Q[:, k:] -= 2.0 * np.outer(Q[:, k:] @ v, v)
+    Q = Q * np.sign(np.diag(A))[None, :]
+    np.testing.assert_allclose(Q, P, atol=1e-10)
+
+
+def test_qr_rotation_spreads_a_basis_vector_like_a_uniform_direction():
+    """Haar-distributed Pi: the image of a fixed unit vector is a uniform
+    direction, whose coordinates follow the Beta coordinate density (a
+    Kolmogorov-Smirnov test over the d coordinates of one column, and the
+    fourth moment 3 / (d (d + 2)) within sampling error).  An identity or a
+    signed permutation would fail both."""
+    from w4a4_post_quantized_b200 import synth
+    d = 1024
+    P = tq.rotation_qr(synth.gaussian_matrix(d, seed=9))
+    a = (d - 1) / 2.0
+    for col in (0, 517):
+        y = P[:, col]
+        assert abs(np.sum(y * y) - 1.0) < 1e-12
+        p = scipy.stats.kstest((y + 1) / 2, scipy.stats.beta(a, a).cdf).pvalue
+        assert p > 1e-3, p
+        m4 = np.mean(y ** 4)
+        # Var(y^4) ~ 105/d^4 - (3/d^2)^2 = 96/d^4: 6 standard errors
+        assert abs(m4 - 3.0 / (d * (d + 2))) < 6 * math.sqrt(96.0 / d ** 4 / d)
+
+
+@pytest.mark.parametrize("b", [3, 4])
+def test_mse_with_the_qr_rotation_matches_the_quantizer_and_the_bound(b):
+    """The page's pipeline with its rotation: for isotropic inputs the
+    normalised error is d * D(b) within sampling error, under the bound."""
+    from w4a4_post_quantized_b200 import synth
+    d, n = 1024, 300
+    rng = np.random.default_rng(21 + b)
+    X = rng.standard_normal((n, d)) * rng.uniform(0.5, 3.0, (n, 1))
+    P = tq.rotation_qr(synth.gaussian_matrix(d, seed=3))
+    c, t = tq.lloyd_max(d, b)
+    codes, gamma, _ = tq.encode(X, P, t)
+    Xr = tq.decode(codes, gamma, P, c)
+    rel = np.sum((X - Xr) ** 2, axis=1) / gamma ** 2
+    D = tq.distortion(d, c, t) * d
+    assert abs(rel.mean() - D) < 4 * rel.std() / math.sqrt(n) + 1e-4 * D
+    assert rel.mean() <= tq.mse_bound(b)

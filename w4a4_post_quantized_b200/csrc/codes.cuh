@@ -56,10 +56,30 @@ constexpr int code_bytes_of(int elems) {
 }
 
 // Codes of V consecutive elements whose row absmax is amax, stored at dst
-// (16-byte aligned).  code = round-half-even(v * kQmax / amax); |v * inv| <=
+// (16-byte aligned, or aligned to the codes' size when that is 4 or 8 bytes).  code = round-half-even(v * kQmax / amax); |v * inv| <=
 // kQmax (1 + 2^-24), so no clamp can ever act.  Adding 1.5 * 2^23 in the same
 // fused operation rounds the exact product to an integer whose low 8 bits are
 // the two's-complement code.
+// Stores W 32-bit words at dst with the widest accesses their count allows
+// (dst aligned to 16 bytes, or to 4 W bytes when W < 4).
+template <int W>
+__device__ __forceinline__ void store_words(const uint32_t (&words)[W], uint8_t *__restrict__ dst) {
+  if constexpr (W % 4 == 0) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int c = 0; c < W / 4; ++c)
+      d4[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+  } else if constexpr (W == 2) {
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(words[0], words[1]);
+  } else {
+    static_assert(W == 1, "word count");
+    *reinterpret_cast<uint32_t *>(dst) = words[0];
+  }
+}
+
+template <int V, int CODE>
+__device__ __forceinline__ void store_code_words(const float (&v)[V], uint8_t *__restrict__ dst);
+
 template <int V, int CODE>
 __device__ __forceinline__ void store_codes(float (&v)[V], float amax, uint8_t *__restrict__ dst) {
   constexpr float kQmax = CODE == kCodeBytes8 ? 127.0f : 7.0f;
@@ -72,7 +92,14 @@ __device__ __forceinline__ void store_codes(float (&v)[V], float amax, uint8_t *
   const unsigned long long inv2 = pack2(inv, inv), magic2 = pack2(12582912.0f, 12582912.0f);
 #pragma unroll
   for (int k = 0; k < V; k += 2) fma_x2(v[k], v[k + 1], inv2, magic2);
-  uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+  store_code_words<V, CODE>(v, dst);
+}
+
+// The codes of V values already rounded by the fused multiply-add with
+// 1.5 * 2^23 (their low bytes are the two's-complement codes), packed in the
+// code format and stored at dst.
+template <int V, int CODE>
+__device__ __forceinline__ void store_code_words(const float (&v)[V], uint8_t *__restrict__ dst) {
   if constexpr (CODE != kCodePacked4) {
     // one byte per code.  Natural order: word w holds elements 4w .. 4w + 3.
     // Operand order: the word pair (2g, 2g + 1) holds elements 8g + 0, 2, 4, 6
@@ -85,9 +112,7 @@ __device__ __forceinline__ void store_codes(float (&v)[V], float amax, uint8_t *
       words[w] = low_bytes(__float_as_uint(v[e0]), __float_as_uint(v[e0 + d]),
                            __float_as_uint(v[e0 + 2 * d]), __float_as_uint(v[e0 + 3 * d]));
     }
-#pragma unroll
-    for (int c = 0; c < V / 16; ++c)
-      d4[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+    store_words<V / 4>(words, dst);
   } else {
     // word w: codes of elements 8w .. 8w + 7, element 2i in the low nibble of byte i
     uint32_t words[V / 8];
@@ -100,9 +125,7 @@ __device__ __forceinline__ void store_codes(float (&v)[V], float amax, uint8_t *
       const uint32_t odd = low_bytes(b[1], b[3], b[5], b[7]);
       words[w] = (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
     }
-#pragma unroll
-    for (int c = 0; c < V / 32; ++c)
-      d4[c] = make_uint4(words[4 * c + 0], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+    store_words<V / 8>(words, dst);
   }
 }
 

@@ -296,8 +296,9 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
 // descriptor version 1 (sm_100) and the swizzle mode, 2 = 128-byte, 4 = 64-byte.
 //   K-major:  rows of the swizzle width along K; 8-row groups `sbo` apart
 //             (lbo unused).
-//   MN-major: atoms of the swizzle width along M (or N) by 8 rows along K;
-//             atoms `lbo` apart along M (N), 8-row K groups `sbo` apart.
+//   MN-major: atoms of the swizzle width along M (or N) by 8 rows along K
+//             (4 rows for kLayoutSw128Base32); atoms `lbo` apart along M (N),
+//             K groups `sbo` apart.
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
                                               uint32_t layout) {
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
@@ -305,7 +306,11 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (static_cast<uint64_t>(1u) << 46) |
          (static_cast<uint64_t>(layout & 7u) << 61);
 }
-constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4;
+// 128-byte swizzle (16-byte chunks XOR row % 8), 64-byte swizzle (16-byte
+// chunks XOR (row / 2) % 4), and the 32-bit MN-major layout: 128-byte rows in
+// groups of 4, 32-byte chunks XOR row % 4 (the one layout tcgen05 reads
+// MN-major tf32 operands from).
+constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw128Base32 = 1;
 
 // D[tmem] (+)= A[smem desc] x B[smem desc]^T with 16-bit floating-point
 // inputs (kind::f16; A and B of the same type, given by the instruction

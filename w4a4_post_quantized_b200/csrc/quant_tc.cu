@@ -1,43 +1,47 @@
-// quant_tc.cu -- the DSFQ activation quantizer with the Hadamard rotation on
-// the tensor cores (sm_100a tcgen05).
+// quant_tc.cu -- the DSFQ activation quantizer with most of the Hadamard
+// rotation on the tensor cores (sm_100a tcgen05).
 //
 // What it computes is the rotate -> smooth -> per-token int4 step of page
 // "十亿参数的三维重建模型，能塞进手机吗？" (sections 预全局旋转, 后局部平滑,
 // 训练后量化（PTQ）, 细粒度量化粒度): for each token row x of K values,
 // y = x H_K (Sylvester Hadamard, natural order; the 1/sqrt(K) goes into the
 // stored step), y_j *= mult_j, step = max|y| / sqrt(K) / 7, codes
-// round-half-even(7 y / max|y|).  The CUDA-core version (quant.cu) spends most
-// of its instructions on the butterflies; here the rotation is two small
-// matrix products on the tensor cores, using the Kronecker structure of the
-// Sylvester matrix: with K = R^2 (R = 32 for K = 1024, R = 64 for K = 4096)
-// and a token row folded as X[a][b] = x[R a + b],
-//     y[R a' + b'] = sum_{a, b} H_R[a][a'] X[a][b] H_R[b][b'].
+// round-half-even(7 y / max|y|).
 //
-//   stage 1 (kind::f16, bf16 inputs, exact products, fp32 accumulators):
-//     Z[b][a'] = sum_a X[a][b] H_R[a][a'].  The MMA's A operand is the bf16
-//     token tile exactly as TMA loads it (rows a, columns b), read MN-major
-//     (M = b, contiguous; K = a); 128 / R tokens form one 128-row MMA.
-//   stage 2 (kind::tf32, fp32 accumulators):
-//     Y[a'][b'] = sum_b Z[b][a'] H_R[b][b'].  Z leaves tensor memory one row
-//     (one b, all a') per thread, which is one K-row of the MN-major A
-//     operand (M = a'); each value goes in as two tf32 terms, hi = Z with the
-//     low 13 mantissa bits cleared and lo = tf32-round(Z - hi), whose sum
-//     carries Z to a relative 2^-22.
-//   finish: thread (token, a') reads Y[a'][0..R) = y[R a' .. R a' + R) from
-//     tensor memory: R consecutive outputs, multiplied by mult, absmax over
-//     the token (warp shuffles, plus one exchange between the two warps of a
-//     token when R = 64), codes formed and stored as the CUDA-core kernel
-//     does (codes.cuh).
+// The Sylvester matrix factors as H_K = H_128 (x) H_S with S = K / 128 (8 at
+// K = 1024, 32 at K = 4096).  Folding a token row as X[a][b] = x[S a + b]
+// (a < 128, b < S),
+//     y[S a' + b'] = sum_b H_S[b][b'] Z[b][a'],   Z[b][a'] = sum_a H_128[a'][a] X[a][b].
+//   * Z on the tensor cores (kind::f16: bf16 inputs, exact +-1 products, fp32
+//     accumulators): D[a'][n] = sum_a H_128[a'][a] B[n][a] with A = H_128
+//     (128 x 128, K-major) and B the bf16 token tile read MN-major: column
+//     n = S t + b of token t of the tile, contiguous in b, exactly as the
+//     tokens lie in memory.  One 128 x 128 x 16 MMA covers 128 / S tokens;
+//     eight cover the 128 values of a.  (Few large MMAs: a tcgen05.mma takes
+//     about 100 cycles to issue whatever its size, so a factorisation into
+//     small products -- H_32 (x) H_32 as two N = 32 stages -- is bound by the
+//     issuing thread.)
+//   * H_S in registers: thread a' (tensor-memory lane a') holds Z[b][a'] for
+//     every b of each token, so the remaining log2(S) butterfly stages run on
+//     values the thread already has, and the thread ends with S consecutive
+//     outputs y[S a' .. S a' + S) -- their codes go out as one contiguous
+//     store, with no transpose.
+//   * absmax: a token's outputs are spread over the 128 lanes (4 warps), so
+//     each tile goes through tensor memory twice: pass 1 applies H_S and the
+//     multipliers, writes the values back in place (tcgen05.st) and forms the
+//     per-token maxima (warp shuffles, then one exchange between the 4 warps
+//     through shared memory); pass 2 reads the values again and forms the
+//     codes with each token's reciprocal step, computed once by one lane.
 //
-// Warp roles (one persistent CTA of 384 threads per SM, 128-row groups
-// round-robin over the CTAs):
-//   warp 0      TMA producer: one 128 x R bf16 box per group (TOK tokens)
-//   warp 1      MMA issuer (one thread): stage 1 of group i, then stage 2 of i-1
-//   warp 2      tensor-memory allocator
-//   warps 4..7  split: stage-1 accumulators -> hi / lo tf32 operand tiles
-//   warps 8..11 finish: stage-2 accumulators -> smoothing, absmax, codes
-// warp % 4 selects the 32 tensor-memory lanes a warp may access: lane
-// 32 q + l holds row (token t, index rho) with t = (32 q + l) / R.
+// Warp roles (one persistent CTA of 384 threads per SM; tiles of 128 / S
+// tokens round-robin over the CTAs):
+//   warp 0        producer: one bulk copy (K = 1024) or two TMA boxes (K = 4096)
+//                 per tile into a ring of stages
+//   warp 1        MMA issuer (one thread): 8 MMAs per tile into one of four
+//                 128-column accumulator slots of tensor memory
+//   warp 2        tensor-memory allocator
+//   warps 4..11   two finishing sets of 4 warps (one per lane quadrant);
+//                 successive tiles go to alternate sets
 //
 // Every wait is bounded (ptx.cuh): a stuck pipeline sets the device status
 // word, the CTA lets its copies land and its MMAs finish, frees its tensor
@@ -49,6 +53,7 @@
 
 #include "codes.cuh"
 #include "ctxcache.h"
+#include "fwht.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -56,91 +61,60 @@ namespace w4a4 {
 namespace {
 
 constexpr int kTcThreads = 384;
-constexpr int W_PROD = 0, W_MMA = 1, W_ALLOC = 2, W_SPLIT0 = 4, W_FIN0 = 8;
+constexpr int W_PROD = 0, W_MMA = 1, W_ALLOC = 2, W_FIN0 = 4;
+constexpr int kFinSets = 2;
+constexpr int kSlots = 4;        // accumulator slots (128 columns each)
+constexpr int kHBytes = 128 * 128 * 2;
 
 template <int K>
 struct TcPlan {
-  static constexpr int R = K == 1024 ? 32 : 64;      // H_K = H_R (x) H_R
-  static constexpr int TOK = 128 / R;                // tokens per 128-row MMA group
-  static constexpr int Q = R / 32;                   // lane quadrants (warps) per token
-  static constexpr int XST = K == 1024 ? 6 : 3;      // token-tile stages
-  static constexpr int D1S = K == 1024 ? 4 : 2;      // stage-1 accumulator slots (R columns)
-  static constexpr int D2S = K == 1024 ? 4 : 2;      // stage-2 accumulator slots (R columns)
-  static constexpr int A2B = 2;                      // stage-2 operand buffers
-  static constexpr int NT = 2;                       // tf32 terms per value (hi, lo)
-  static constexpr int X_BYTES = 128 * R * 2;        // one group's bf16 tile
-  static constexpr uint32_t LAYOUT1 = R == 32 ? kLayoutSw64 : kLayoutSw128;  // 2R-byte rows
-  static constexpr int SW1 = 2 * R;                  // swizzle width of the bf16 tiles (bytes)
-  static constexpr int A1_LBO = 2 * K;               // tokens (MN atoms) apart in the tile
-  static constexpr int A1_SBO = 8 * 2 * R;           // 8 rows a apart
-  static constexpr int B1_BYTES = R * R * 2;
-  static constexpr int B1_SBO = 8 * 2 * R;
-  static constexpr int TERM = 128 * R * 4;           // one tf32 term of the stage-2 A operand
-  static constexpr int A2_BYTES = NT * TERM;
-  static constexpr int A2_LBO = (R / 8) * 1024;      // MN atoms (32 values of a') apart
-  static constexpr int B2_BYTES = R * R * 4;
+  static constexpr int S = K / 128;                  // H_K = H_128 (x) H_S
+  static constexpr int LOGS = S == 8 ? 3 : 5;
+  static constexpr int TOKT = 128 / S;               // tokens per tile (N = 128 columns)
+  static constexpr int X_BYTES = TOKT * K * 2;       // one tile of bf16 tokens (32 KB)
+  static constexpr int XST = 4;                      // tile stages
+  // B operand (the token tile, MN-major): K = 1024: no swizzle, 8-row groups
+  // of 16-byte rows, tokens (MN atoms of 8 values) 2 KB apart; K = 4096:
+  // 64-byte swizzle (the TMA boxes' layout), atoms of 32 values, tokens 8 KB
+  // apart, 8-row groups 512 bytes apart.
+  static constexpr uint32_t B_LAYOUT = S == 8 ? 0u : kLayoutSw64;
+  static constexpr uint32_t B_LBO = S == 8 ? 128u : static_cast<uint32_t>(2 * K);
+  static constexpr uint32_t B_SBO = S == 8 ? static_cast<uint32_t>(2 * K) : 512u;
+  static constexpr uint32_t B_KSTEP = S == 8 ? 256u : 1024u;  // 16 rows of a
   static constexpr int OFF_X = 0;
-  static constexpr int OFF_A2 = OFF_X + XST * X_BYTES;
-  static constexpr int OFF_B1 = OFF_A2 + A2B * A2_BYTES;
-  static constexpr int OFF_B2 = OFF_B1 + (B1_BYTES + 1023) / 1024 * 1024;
-  static constexpr int OFF_TAB = OFF_B2 + B2_BYTES;  // multipliers, K floats
-  static constexpr int OFF_PAIR = OFF_TAB + 4 * K;   // [D2S][4] per-warp absmax (R = 64)
-  static constexpr int OFF_BAR = OFF_PAIR + D2S * 4 * 4;
-  static constexpr int NUM_BARS = 2 * XST + 2 * D1S + 2 * A2B + 2 * D2S + D2S * TOK + 1;
+  static constexpr int OFF_H = OFF_X + XST * X_BYTES;
+  static constexpr int OFF_TM = OFF_H + kHBytes;     // [kSlots][TOKT][4] warp maxima
+  static constexpr int OFF_BAR = OFF_TM + kSlots * TOKT * 4 * 4;
+  static constexpr int NUM_BARS = 2 * XST + 3 * kSlots + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024
-  static constexpr uint32_t TMEM_COLS = 256;
-  static_assert(D1S * R + D2S * R <= static_cast<int>(TMEM_COLS), "tensor-memory budget");
   static_assert(SMEM <= 232448, "shared-memory budget");
-  static_assert(OFF_A2 % 1024 == 0 && OFF_B1 % 1024 == 0 && OFF_B2 % 1024 == 0 && X_BYTES % 1024 == 0,
-                "swizzled tiles need 1024-byte alignment");
-  static constexpr uint32_t IDESC1 = idesc_f32acc<128, R, false, true>();
-  static constexpr uint32_t IDESC2 = idesc_f32acc<128, R, true, true>();
+  static_assert(OFF_H % 1024 == 0 && X_BYTES % 1024 == 0, "tile alignment");
+  // kind::f16, bf16 A and B, fp32 D, A K-major, B MN-major, M = N = 128
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                                    ((128u >> 3) << 17) | ((128u >> 4) << 24);
 };
-
-// Physical offset of a logical byte offset inside a tile whose 16-byte chunks
-// are XOR-swizzled by address bits 7.. (64-byte: 2 bits, 128-byte: 3 bits).
-__device__ __forceinline__ uint32_t swz(uint32_t off, int width) {
-  const uint32_t mask = width == 64 ? 3u : 7u;
-  return off ^ (((off >> 7) & mask) << 4);
-}
-
-__device__ __forceinline__ uint32_t tf32_rna(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
 
 template <int K, int CODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, const float *__restrict__ mult,
-                    uint8_t *__restrict__ q, float *__restrict__ scale, unsigned int *__restrict__ status,
-                    int num_groups) {
+    quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, const uint16_t *__restrict__ X, int64_t M,
+                    const float *__restrict__ mult, uint8_t *__restrict__ q, float *__restrict__ scale,
+                    unsigned int *__restrict__ status, int num_tiles) {
   using P = TcPlan<K>;
-  constexpr int R = P::R;
+  constexpr int S = P::S, TOKT = P::TOKT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + P::OFF_BAR);
-  uint64_t *x_full = bars;                      // a group's token tile landed
-  uint64_t *x_free = x_full + P::XST;           // stage-1 MMAs reading it completed
-  uint64_t *d1_full = x_free + P::XST;          // stage-1 accumulators complete
-  uint64_t *d1_free = d1_full + P::D1S;         // split warps read them (4 arrivals)
-  uint64_t *a2_full = d1_free + P::D1S;         // stage-2 operand written (4 arrivals)
-  uint64_t *a2_free = a2_full + P::A2B;         // stage-2 MMAs reading it completed
-  uint64_t *d2_full = a2_free + P::A2B;         // stage-2 accumulators complete
-  uint64_t *d2_free = d2_full + P::D2S;         // finish warps read them (4 arrivals)
-  uint64_t *pair_bar = d2_free + P::D2S;        // [D2S][TOK]: the two warps of a token (R = 64)
-  uint64_t *mma_done = pair_bar + P::D2S * P::TOK;
+  uint64_t *x_full = bars;                 // a tile's tokens landed
+  uint64_t *x_free = x_full + P::XST;      // the MMAs reading it completed
+  uint64_t *d_full = x_free + P::XST;      // an accumulator slot complete
+  uint64_t *d_free = d_full + kSlots;      // its 4 finishing warps are done with it
+  uint64_t *tm_bar = d_free + kSlots;      // its 4 finishing warps wrote their maxima
+  uint64_t *mma_done = tm_bar + kSlots;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + P::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + P::OFF_MISC + 4);
-  float *pairmax = reinterpret_cast<float *>(smem + P::OFF_PAIR);
+  float *tmax = reinterpret_cast<float *>(smem + P::OFF_TM);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -150,40 +124,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&x_full[s], 1);
       mbar_init(&x_free[s], 1);
     }
-    for (int s = 0; s < P::D1S; ++s) {
-      mbar_init(&d1_full[s], 1);
-      mbar_init(&d1_free[s], 4);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&d_full[s], 1);
+      mbar_init(&d_free[s], 4);
+      mbar_init(&tm_bar[s], 4);
     }
-    for (int s = 0; s < P::A2B; ++s) {
-      mbar_init(&a2_full[s], 4);
-      mbar_init(&a2_free[s], 1);
-    }
-    for (int s = 0; s < P::D2S; ++s) {
-      mbar_init(&d2_full[s], 1);
-      mbar_init(&d2_free[s], 4);
-    }
-    for (int s = 0; s < P::D2S * P::TOK; ++s) mbar_init(&pair_bar[s], 2);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == W_PROD && lane == 0) tma_prefetch_desc(&tmX);
+  if (warp == W_PROD && lane == 0 && S != 8) tma_prefetch_desc(&tmX);
   if (warp == W_ALLOC) {
-    tmem_alloc(tmem_slot, P::TMEM_COLS);
+    tmem_alloc(tmem_slot, kSlots * 128);
     tmem_relinquish();
   }
-  // The two Hadamard operands, +-1 in bf16 (stage 1) and tf32 (stage 2),
-  // K-major: row n holds H_R[k][n] over k (H_R is symmetric).
   {
-    uint8_t *b1 = smem + P::OFF_B1;
-    uint8_t *b2 = smem + P::OFF_B2;
-    for (int idx = threadIdx.x; idx < R * R; idx += kTcThreads) {
-      const int n = idx / R, k = idx % R;
-      const bool neg = (__popc(n & k) & 1) != 0;
-      *reinterpret_cast<uint16_t *>(b1 + swz(n * 2 * R + 2 * k, P::SW1)) = neg ? 0xBF80u : 0x3F80u;
-      // tf32 rows are 4R bytes: K halves of 32 values, each a 128-byte swizzled tile
-      const uint32_t off2 = (k / 32) * (R * 128) + n * 128 + (k % 32) * 4;
-      *reinterpret_cast<uint32_t *>(b2 + swz(off2, 128)) = neg ? 0xBF800000u : 0x3F800000u;
+    // H_128 in bf16, K-major with the 128-byte swizzle: row a' holds
+    // H[a'][a] over a, in two 64-value halves of 16 KB (row a' at 128 a',
+    // 16-byte chunk c at c ^ (a' % 8))
+    uint8_t *h = smem + P::OFF_H;
+    for (int idx = threadIdx.x; idx < 128 * 128; idx += kTcThreads) {
+      const int ap = idx >> 7, a = idx & 127;
+      const uint32_t off = (a >> 6) * 16384 + ap * 128 + ((((a & 63) >> 3) ^ (ap & 7)) << 4) + (a & 7) * 2;
+      *reinterpret_cast<uint16_t *>(h + off) = (__popc(ap & a) & 1) ? 0xBF80u : 0x3F80u;
     }
     fence_proxy_async_smem();
   }
@@ -195,27 +158,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // stream; X and mult are read only after it has completed.
   griddep_launch_dependents();
   griddep_wait();
-  {
-    // multiplier table: float4 (c, rho) at c * R + rho holds mult[R rho + 4c .. + 3]
-    // (the finishing thread rho reads its R consecutive multipliers; a warp's
-    // 16-byte reads of one c are consecutive: conflict-free)
-    float4 *tab = reinterpret_cast<float4 *>(smem + P::OFF_TAB);
-    for (int idx = threadIdx.x; idx < K / 4; idx += kTcThreads) {
-      const int c = idx / R, rho = idx % R;
-      tab[idx] = __ldg(reinterpret_cast<const float4 *>(mult + R * rho + 4 * c));
-    }
-  }
-  __syncthreads();
 
   if (warp == W_PROD) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       uint32_t it = 0;
-      for (int g = blockIdx.x; g < num_groups; g += gridDim.x, ++it) {
+      for (int g = blockIdx.x; g < num_tiles; g += gridDim.x, ++it) {
         const uint32_t s = it % P::XST;
         if (!mbar_wait(&x_free[s], ((it / P::XST) & 1u) ^ 1u, abort_flag, status)) break;
-        mbar_arrive_expect_tx(&x_full[s], P::X_BYTES);
-        tma_load_2d(smem + P::OFF_X + s * P::X_BYTES, &tmX, 0, g * 128, &x_full[s]);
+        uint8_t *dst = smem + P::OFF_X + s * P::X_BYTES;
+        const int64_t tok0 = static_cast<int64_t>(g) * TOKT;
+        if constexpr (S == 8) {
+          // the tile's tokens are contiguous: one bulk copy of the valid ones
+          // (the rest of the stage keeps old bytes; their columns are not stored)
+          const int64_t valid = (M - tok0 < TOKT) ? M - tok0 : TOKT;
+          const uint32_t bytes = static_cast<uint32_t>(valid) * 2 * K;
+          mbar_arrive_expect_tx(&x_full[s], bytes);
+          bulk_load(dst, X + tok0 * K, bytes, &x_full[s]);
+        } else {
+          // rows (token, a) of S values through the 64-byte swizzle, 256 rows
+          // (two tokens) per box; rows past the end are filled with zeros
+          mbar_arrive_expect_tx(&x_full[s], P::X_BYTES);
+          tma_load_2d(dst, &tmX, 0, static_cast<int>(g * 512), &x_full[s]);
+          tma_load_2d(dst + P::X_BYTES / 2, &tmX, 0, static_cast<int>(g * 512 + 256), &x_full[s]);
+        }
       }
       // let every issued copy land before the CTA can exit
       for (uint32_t u = (it > P::XST ? it - P::XST : 0); u < it; ++u)
@@ -225,156 +191,159 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t x0 = smem_u32(smem + P::OFF_X);
-      const uint32_t a20 = smem_u32(smem + P::OFF_A2);
-      const uint32_t b1 = smem_u32(smem + P::OFF_B1);
-      const uint32_t b2 = smem_u32(smem + P::OFF_B2);
-      // stage 2 of the i-th group of this CTA
-      auto stage2 = [&](uint32_t i) -> bool {
-        const uint32_t ab = i % P::A2B, d2 = i % P::D2S;
-        if (!mbar_wait(&a2_full[ab], (i / P::A2B) & 1u, abort_flag, status)) return false;
-        if (!mbar_wait(&d2_free[d2], ((i / P::D2S) & 1u) ^ 1u, abort_flag, status)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem_base + P::D1S * R + d2 * R;
-#pragma unroll
-        for (int term = 0; term < P::NT; ++term)
-#pragma unroll
-          for (int j = 0; j < R / 8; ++j)
-            mma_tf32(d,
-                     umma_desc(a20 + ab * P::A2_BYTES + term * P::TERM + j * 1024, P::A2_LBO, 1024,
-                               kLayoutSw128),
-                     umma_desc(b2 + (j / 4) * (R * 128) + (j % 4) * 32, 16, 1024, kLayoutSw128),
-                     P::IDESC2, (term | j) != 0 ? 1u : 0u);
-        tc_commit(&a2_free[ab]);
-        tc_commit(&d2_full[d2]);
-        return true;
-      };
+      const uint32_t h0 = smem_u32(smem + P::OFF_H);
       uint32_t it = 0;
-      bool ok = true;
-      for (int g = blockIdx.x; g < num_groups; g += gridDim.x, ++it) {
-        const uint32_t s = it % P::XST, d1 = it % P::D1S;
+      for (int g = blockIdx.x; g < num_tiles; g += gridDim.x, ++it) {
+        const uint32_t s = it % P::XST, d = it % kSlots;
         if (!mbar_wait(&x_full[s], (it / P::XST) & 1u, abort_flag, status) ||
-            !mbar_wait(&d1_free[d1], ((it / P::D1S) & 1u) ^ 1u, abort_flag, status)) {
-          ok = false;
+            !mbar_wait(&d_free[d], ((it / kSlots) & 1u) ^ 1u, abort_flag, status))
           break;
-        }
         tc_fence_after();
-        const uint32_t d = tmem_base + d1 * R;
 #pragma unroll
-        for (int j = 0; j < R / 16; ++j)
-          mma_f16(d, umma_desc(x0 + s * P::X_BYTES + j * 2 * P::A1_SBO, P::A1_LBO, P::A1_SBO, P::LAYOUT1),
-                  umma_desc(b1 + j * 32, 16, P::B1_SBO, P::LAYOUT1), P::IDESC1, j != 0 ? 1u : 0u);
+        for (int j = 0; j < 8; ++j)
+          mma_f16(tmem_base + d * 128,
+                  umma_desc(h0 + (j >> 2) * 16384 + (j & 3) * 32, 16, 1024, kLayoutSw128),
+                  umma_desc(x0 + s * P::X_BYTES + j * P::B_KSTEP, P::B_LBO, P::B_SBO, P::B_LAYOUT),
+                  P::IDESC, j != 0 ? 1u : 0u);
         tc_commit(&x_free[s]);
-        tc_commit(&d1_full[d1]);
-        if (it > 0 && !stage2(it - 1)) {
-          ok = false;
-          break;
-        }
+        tc_commit(&d_full[d]);
       }
-      if (ok && it > 0) stage2(it - 1);
       // every MMA issued must finish before tensor memory is freed
       tc_commit(mma_done);
       mbar_wait_drain(mma_done, 0, status);
     }
-  } else if (warp >= W_SPLIT0 && warp < W_SPLIT0 + 4) {
-    // ------------------------------------------------------------------ split
-    const int qd = warp & 3;
-    const int t = qd / P::Q;                 // token of the group
-    const int rho = (qd % P::Q) * 32 + lane; // b: one K-row of the stage-2 operand
-    const uint32_t taddr0 = tmem_base + (static_cast<uint32_t>(qd * 32) << 16);
-    const uint32_t a2base = smem_u32(smem + P::OFF_A2);
-    uint32_t it = 0;
-    for (int g = blockIdx.x; g < num_groups; g += gridDim.x, ++it) {
-      const uint32_t d1 = it % P::D1S, ab = it % P::A2B;
-      if (!mbar_wait(&d1_full[d1], (it / P::D1S) & 1u, abort_flag, status)) break;
-      tc_fence_after();
-      uint32_t z[R];
-      tmem_ld_32x32b_x32(taddr0 + d1 * R, *reinterpret_cast<uint32_t(*)[32]>(&z[0]));
-      if constexpr (R == 64)
-        tmem_ld_32x32b_x32(taddr0 + d1 * R + 32, *reinterpret_cast<uint32_t(*)[32]>(&z[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&d1_free[d1]);
-      if (!mbar_wait(&a2_free[ab], ((it / P::A2B) & 1u) ^ 1u, abort_flag, status)) break;
-      // row rho of atom (t, ah): logical offset atom * LBO + (rho / 8) * 1024 + (rho % 8) * 128,
-      // 16-byte chunk c (values a' = 32 ah + 4c .. + 3) at c ^ (rho % 8)
-      const uint32_t rowb = a2base + ab * P::A2_BYTES + (rho >> 3) * 1024 + (rho & 7) * 128;
-#pragma unroll
-      for (int ah = 0; ah < P::Q; ++ah) {
-        const uint32_t atom = rowb + (t * P::Q + ah) * P::A2_LBO;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t x = z[32 * ah + 4 * c + e];
-            hi[e] = x & 0xFFFFE000u;
-            lo[e] = tf32_rna(__uint_as_float(x) - __uint_as_float(hi[e]));
-          }
-          const uint32_t a = atom + ((c ^ (rho & 7)) << 4);
-          st_shared_v4(a, hi[0], hi[1], hi[2], hi[3]);
-          st_shared_v4(a + P::TERM, lo[0], lo[1], lo[2], lo[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a2_full[ab]);
-    }
-  } else if (warp >= W_FIN0) {
+  } else if (warp >= W_FIN0 && warp < W_FIN0 + 4 * kFinSets) {
     // ----------------------------------------------------------------- finish
     const int qd = warp & 3;
-    const int t = qd / P::Q;
-    const int rho = (qd % P::Q) * 32 + lane;  // a': outputs R rho .. R rho + R - 1
-    const uint32_t taddr0 = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + P::D1S * R;
-    const float4 *tab = reinterpret_cast<const float4 *>(smem + P::OFF_TAB);
+    const int set = (warp - W_FIN0) >> 2;
+    const int ap = 32 * qd + lane;               // a': outputs S a' .. S a' + S - 1
+    const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * qd) << 16);
     constexpr float kQmax = CODE == kCodeBytes8 ? 127.0f : 7.0f;
     constexpr float kInvSqrtK = K == 1024 ? 0.03125f : 0.015625f;
-    uint32_t it = 0;
-    for (int g = blockIdx.x; g < num_groups; g += gridDim.x, ++it) {
-      const uint32_t d2 = it % P::D2S;
-      if (!mbar_wait(&d2_full[d2], (it / P::D2S) & 1u, abort_flag, status)) break;
+    float m[S];                                  // this thread's multipliers
+#pragma unroll
+    for (int c = 0; c < S / 4; ++c) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(mult + S * ap) + c);
+      m[4 * c] = v.x;
+      m[4 * c + 1] = v.y;
+      m[4 * c + 2] = v.z;
+      m[4 * c + 3] = v.w;
+    }
+    // token u of a 32-column load: its S values for this lane, transformed
+    // by H_S and smoothed
+    auto token_values = [&](const uint32_t (&r)[32], int j0, float (&y)[S]) {
+#pragma unroll
+      for (int b = 0; b < S; ++b) y[b] = __uint_as_float(r[j0 + b]);
+      butterflies<S, 0, P::LOGS>(y);
+#pragma unroll
+      for (int b = 0; b < S; b += 2) mul_x2(y[b], y[b + 1], m[b], m[b + 1]);
+    };
+    auto local_max = [&](const float (&y)[S]) {
+      float am = 0.0f;
+#pragma unroll
+      for (int b = 0; b < S; b += 2) am = fmax3(am, fabsf(y[b]), fabsf(y[b + 1]));
+      return am;
+    };
+    for (uint32_t it = set; blockIdx.x + it * gridDim.x < static_cast<uint32_t>(num_tiles);
+         it += kFinSets) {
+      const int g = static_cast<int>(blockIdx.x + it * gridDim.x);
+      const uint32_t d = it % kSlots;
+      if (!mbar_wait(&d_full[d], (it / kSlots) & 1u, abort_flag, status)) break;
       tc_fence_after();
-      uint32_t yb[R];
-      tmem_ld_32x32b_x32(taddr0 + d2 * R, *reinterpret_cast<uint32_t(*)[32]>(&yb[0]));
-      if constexpr (R == 64)
-        tmem_ld_32x32b_x32(taddr0 + d2 * R + 32, *reinterpret_cast<uint32_t(*)[32]>(&yb[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&d2_free[d2]);
-      float y[R];
+      const uint32_t taddr = tq + d * 128;
+      // pass 1: H_S and the multipliers, written back in place (tcgen05.st),
+      // and the per-token maxima over this warp's 32 lanes
+      float tok_max[TOKT];
 #pragma unroll
-      for (int c = 0; c < R / 4; ++c) {
-        const float4 m = tab[c * R + rho];
-        y[4 * c + 0] = __uint_as_float(yb[4 * c + 0]);
-        y[4 * c + 1] = __uint_as_float(yb[4 * c + 1]);
-        y[4 * c + 2] = __uint_as_float(yb[4 * c + 2]);
-        y[4 * c + 3] = __uint_as_float(yb[4 * c + 3]);
-        mul_x2(y[4 * c + 0], y[4 * c + 1], m.x, m.y);
-        mul_x2(y[4 * c + 2], y[4 * c + 3], m.z, m.w);
-      }
-      float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int c = 0; c < 4; ++c) {              // 32 columns = 32 / S tokens
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int r = 0; r < R; r += 8)
+        for (int u = 0; u < 32 / S; ++u) {
+          float y[S];
+          token_values(r, u * S, y);
+          tok_max[c * (32 / S) + u] = local_max(y);
 #pragma unroll
-        for (int a = 0; a < 4; ++a) am[a] = fmax3(am[a], fabsf(y[r + 2 * a]), fabsf(y[r + 2 * a + 1]));
-      float amax = fmax3(am[0], am[1], fmaxf(am[2], am[3]));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      if constexpr (P::Q == 2) {
-        // the other warp of this token holds the other half of its outputs
-        uint64_t *pb = &pair_bar[d2 * P::TOK + t];
-        if (lane == 0) {
-          pairmax[d2 * 4 + qd] = amax;
-          mbar_arrive(pb);
+          for (int b = 0; b < S; ++b) r[u * S + b] = __float_as_uint(y[b]);
         }
-        if (!mbar_wait(pb, (it / P::D2S) & 1u, abort_flag, status)) break;
-        amax = fmaxf(amax, pairmax[d2 * 4 + (qd ^ 1)]);
+        tmem_st_32x32b_x32(taddr + 32 * c, r);
       }
-      const int64_t tok = static_cast<int64_t>(g) * P::TOK + t;
-      if (tok < M) {
-        if (lane == 0 && (qd % P::Q) == 0) scale[tok] = amax * kInvSqrtK / kQmax;
-        store_codes<R, CODE>(y, amax, q + tok * code_bytes_of<CODE>(K) + rho * code_bytes_of<CODE>(R));
+      // maxima over the warp, reduce-scattered: at the step with lane offset
+      // o a lane keeps the half of its remaining tokens that its lane bit
+      // selects and sends the other half, so lane l ends with the warp's
+      // maximum of token l / (32 / TOKT)
+#pragma unroll
+      for (int step = 0; step < 5; ++step) {
+        const int o = 16 >> step;
+        const int half = (TOKT >> step) / 2;     // tokens sent at this step (0: plain reduce)
+        const bool upper = (lane & o) != 0;
+        if (half > 0) {
+#pragma unroll
+          for (int j = 0; j < (half > 0 ? half : 1); ++j) {
+            const float keep = upper ? tok_max[j + half] : tok_max[j];
+            const float send = upper ? tok_max[j] : tok_max[j + half];
+            tok_max[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+          }
+        } else {
+          tok_max[0] = fmaxf(tok_max[0], __shfl_xor_sync(0xffffffffu, tok_max[0], o));
+        }
+      }
+      // exchange with the other three warps of the set
+      float *tm = tmax + d * TOKT * 4;
+      constexpr int kLanesPerTok = 32 / TOKT;
+      if (lane % kLanesPerTok == 0) tm[(lane / kLanesPerTok) * 4 + qd] = tok_max[0];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tm_bar[d]);
+      if (!mbar_wait(&tm_bar[d], (it / kSlots) & 1u, abort_flag, status)) break;
+      // lane t < TOKT: token t's maximum, step and reciprocal step (the same
+      // binary32 arithmetic as store_codes: a maximum below 2^-100 is first
+      // scaled by 2^64, exactly, to keep kQmax / amax finite)
+      const int64_t tok0 = static_cast<int64_t>(g) * TOKT;
+      float inv_l = 0.0f, pre_l = 1.0f;
+      if (lane < TOKT) {
+        const float4 w = reinterpret_cast<const float4 *>(tm)[lane];
+        float amax = fmaxf(fmaxf(w.x, w.y), fmaxf(w.z, w.w));
+        if (qd == 0 && tok0 + lane < M) scale[tok0 + lane] = amax * kInvSqrtK / kQmax;
+        if (amax < 0x1p-100f) {
+          amax *= 0x1p+64f;
+          pre_l = 0x1p+64f;
+        }
+        inv_l = amax > 0.0f ? kQmax / amax : 0.0f;
+      }
+      tmem_wait_st();
+      // pass 2: codes
+      const unsigned long long magic2 = pack2(12582912.0f, 12582912.0f);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        tmem_wait_ld();
+        if (c == 3) {                            // the slot is no longer read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&d_free[d]);
+        }
+#pragma unroll
+        for (int u = 0; u < 32 / S; ++u) {
+          const int t = c * (32 / S) + u;
+          const float inv = __shfl_sync(0xffffffffu, inv_l, t);
+          const float pre = __shfl_sync(0xffffffffu, pre_l, t);
+          const int64_t tok = tok0 + t;
+          if (tok < M) {
+            float y[S];
+#pragma unroll
+            for (int b = 0; b < S; ++b) y[b] = __uint_as_float(r[u * S + b]);
+            if (pre != 1.0f) {
+#pragma unroll
+              for (int b = 0; b < S; ++b) y[b] *= pre;
+            }
+            const unsigned long long inv2 = pack2(inv, inv);
+#pragma unroll
+            for (int b = 0; b < S; b += 2) fma_x2(y[b], y[b + 1], inv2, magic2);
+            store_code_words<S, CODE>(y, q + tok * code_bytes_of<CODE>(K) + ap * code_bytes_of<CODE>(S));
+          }
+        }
       }
     }
   }
@@ -382,11 +351,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == W_ALLOC) tmem_dealloc(tmem_base, P::TMEM_COLS);
+  if (warp == W_ALLOC) tmem_dealloc(tmem_base, kSlots * 128);
 }
 
-// Tokens per launch: the TMA row coordinate (token * R) must stay below 2^31.
-constexpr int64_t kTcMaxTokens = int64_t(1) << 24;
+// Tokens per launch: the TMA row coordinate (token * 128) must stay below 2^31.
+constexpr int64_t kTcMaxTokens = int64_t(1) << 23;
 
 template <int K, int CODE>
 cudaError_t launch_tc_k(const uint16_t *X, int64_t M, const float *mult, uint8_t *q, float *scale,
@@ -404,16 +373,17 @@ cudaError_t launch_tc_k(const uint16_t *X, int64_t M, const float *mult, uint8_t
   if ((e = status_word(&status)) != cudaSuccess) return e;
   for (int64_t m0 = 0; m0 < M; m0 += kTcMaxTokens) {
     const int64_t m = (M - m0 < kTcMaxTokens) ? M - m0 : kTcMaxTokens;
-    // the token rows as m R rows of R bf16 values (row a of every token)
-    CUtensorMap tm;
-    if (!encode_tensor_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X + m0 * K, P::R,
-                              static_cast<uint64_t>(m) * P::R, 2 * P::R, P::R, 128,
-                              P::R == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+    CUtensorMap tm = {};
+    // K = 4096: the tokens as rows (token, a) of 32 bf16 values
+    if (P::S != 8 &&
+        !encode_tensor_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X + m0 * K, P::S,
+                              static_cast<uint64_t>(m) * 128, 2 * P::S, P::S, 256,
+                              CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
-    const int groups = static_cast<int>((m + P::TOK - 1) / P::TOK);
+    const int tiles = static_cast<int>((m + P::TOKT - 1) / P::TOKT);
     const int sms = device_sm_count();
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(groups < sms ? groups : sms, 1, 1);
+    cfg.gridDim = dim3(tiles < sms ? tiles : sms, 1, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = P::SMEM;
     cfg.stream = st;
@@ -422,8 +392,8 @@ cudaError_t launch_tc_k(const uint16_t *X, int64_t M, const float *mult, uint8_t
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, tm, m, mult, q + m0 * code_bytes_of<CODE>(K), scale + m0, status,
-                           groups);
+    e = cudaLaunchKernelEx(&cfg, kern, tm, X + m0 * K, m, mult, q + m0 * code_bytes_of<CODE>(K),
+                           scale + m0, status, tiles);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();

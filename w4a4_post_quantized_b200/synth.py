@@ -154,6 +154,13 @@ def kv_vectors(n: int, d: int, seed: int) -> np.ndarray:
     return x
 
 
+def gaussian_matrix(d: int, seed: int) -> np.ndarray:
+    """fp64 [d, d] of independent standard normal entries (the Gaussian matrix
+    whose QR factor is a random rotation)."""
+    rng = np.random.Generator(np.random.PCG64([seed, 0x6A55]))
+    return rng.standard_normal((d, d))
+
+
 def random_signs(d: int, seed: int) -> np.ndarray:
     """fp32 [d] of independent +-1 (the random sign vector of a rotation)."""
     rng = np.random.Generator(np.random.PCG64([seed, 0x516E]))
