@@ -286,8 +286,10 @@ def run_ours(args, wl, world, rank, local):
         barrier(world)
         torch.cuda.synchronize()
         t0.record(stream)
+        torch.cuda.nvtx.range_push("timed")
         for i in range(args.steps):
             step(i)
+        torch.cuda.nvtx.range_pop()
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -481,9 +483,11 @@ def run_ours(args, wl, world, rank, local):
                 "ms_per_launch_in_step": g_step_ms,
                 "timing": f"CUDA events around {n_iso} back-to-back launches of this kernel alone; "
                           "ms_per_launch_in_step: events between the two kernels of a step"}
-    roofline_q = {"bound": "hbm", "kernel": "quantize_rows_kernel", "achieved": q_gbs,
+    q_kernel = "quant_tc_kernel" if not gelu else "quantize_rows_kernel"
+    roofline_q = {"bound": "hbm", "kernel": q_kernel, "achieved": q_gbs,
                   "peak": peaks["hbm"], "unit": "GB/s", "frac": q_gbs / peaks["hbm"],
-                  "traffic": profile_traffic("quant.cu", f"quant_{args.workload}"),
+                  "traffic": profile_traffic("quant_tc.cu" if not gelu else "quant.cu",
+                                             f"quant_{args.workload}"),
                   "ms_per_launch": q_ms, "algorithmic_bytes_per_launch": q_bytes,
                   "ms_per_launch_in_step": q_step_ms}
 
@@ -705,8 +709,10 @@ def run_stack(args, st, world, rank, local):
         barrier(world)
         torch.cuda.synchronize()
         t0.record(stream)
+        torch.cuda.nvtx.range_push("timed")
         for _ in range(args.steps):
             step()
+        torch.cuda.nvtx.range_pop()
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -732,7 +738,11 @@ def run_stack(args, st, world, rank, local):
     value = world * ops_step * args.steps / (elapsed_ms * 1e-3) / 1e12
     q_ms = [e[0].elapsed_time(e[1]) for e in ev]
     g_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    q_bytes = [2.0 * M * K + M * K + 4.0 * M for (_, _, K, _) in layers]   # X in, one-per-byte codes, steps
+    # algorithmic bytes of the quantizer: X in, 4-bit codes out (half a byte
+    # each), the steps; the fused call's route stores the codes one per byte
+    # (M K bytes instead of M K / 2: the GEMM then reads them without widening)
+    q_bytes = [2.5 * M * K + 4.0 * M for (_, _, K, _) in layers]
+    q_moved = [3.0 * M * K + 4.0 * M for (_, _, K, _) in layers]
     g_ops = [2.0 * M * N * K for (_, _, K, N) in layers]
     peaks = load_peaks()
     int8_peak_burst = peaks["bf16"] * INT8_PER_BF16
@@ -771,7 +781,8 @@ def run_stack(args, st, world, rank, local):
             "K": K, "N": N, "layers": c,
             "in_step_quantize_us": per[name]["quantize_ms"] / c * 1e3,
             "in_step_gemm_us": per[name]["gemm_ms"] / c * 1e3,
-            "alone_quantize_us": tq_ms * 1e3, "alone_quantize_gbs": (3.0 * M * K + 4 * M) / (tq_ms * 1e-3) / 1e9,
+            "alone_quantize_us": tq_ms * 1e3, "alone_quantize_gbs": (2.5 * M * K + 4 * M) / (tq_ms * 1e-3) / 1e9,
+            "alone_quantize_gbs_moved": (3.0 * M * K + 4 * M) / (tq_ms * 1e-3) / 1e9,
             "alone_gemm_us": tg_ms * 1e3, "alone_gemm_tops": gtops,
             "alone_gemm_frac_burst": gtops / int8_peak_burst}
     # M7 (the pages' +0.2 % for DSFQ over plain quantization): the fused call per
@@ -858,10 +869,14 @@ def run_stack(args, st, world, rank, local):
         "timing": "CUDA events on the launching stream around each GEMM launch of one step "
                   "(time-weighted: sum of ops / sum of launch durations)"}
     roofline_q = {
-        "bound": "hbm", "kernel": "quantize_rows_kernel", "achieved": q_ach, "peak": peaks["hbm"],
+        "bound": "hbm", "kernel": "quant_tc_kernel", "achieved": q_ach, "peak": peaks["hbm"],
         "unit": "GB/s", "frac": q_ach / peaks["hbm"],
-        "traffic": profile_traffic("quant.cu", f"quant_{args.workload}"),
-        "ms_per_launch": q_total_ms / len(layers), "algorithmic_bytes_per_launch": sum(q_bytes) / len(layers)}
+        "traffic": profile_traffic("quant_tc.cu", f"quant_{args.workload}"),
+        "ms_per_launch": q_total_ms / len(layers), "algorithmic_bytes_per_launch": sum(q_bytes) / len(layers),
+        "bytes_moved_per_launch": sum(q_moved) / len(layers),
+        "achieved_moved": sum(q_moved) / (q_total_ms * 1e-3) / 1e9,
+        "bytes_note": "algorithmic = 2 M K (X) + M K / 2 (4-bit codes) + 4 M (steps); moved: the codes "
+                      "go one per byte on the fused call's route (3 M K + 4 M)"}
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -956,8 +971,10 @@ def run_tq(args, world, rank, local):
         barrier(world)
         torch.cuda.synchronize()
         t0.record(stream)
+        torch.cuda.nvtx.range_push("timed")
         for i in range(args.steps):
             step(i)
+        torch.cuda.nvtx.range_pop()
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
