@@ -74,6 +74,7 @@ STACKS = {
 METRIC = "W4A4 linear TOPS & tokens/s on VGGT shapes, % of INT8 TC peak / HBM BW"
 NSETS = 4          # input/output buffer sets rotated so no step finds its inputs in L2
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput ratio (4.5 / 2.25 POPS)
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 : bf16 tensor throughput ratio
 
 
 def load_peaks():
@@ -925,24 +926,31 @@ def tq_bytes(n: int, d: int):
     return n * 4 * d + packed, packed + n * 4 * d
 
 
+TQ_PI_SEED = 77   # seed of the Gaussian matrix whose QR factor is the rotation
+
+
 def tq_oracle_sample(rows: int, seed: int = 0):
-    """The oracle's encode + decode on `rows` KV vectors (untimed setup)."""
+    """The oracle's encode + decode with the page's rotation (Q of a Gaussian
+    matrix) on `rows` KV vectors (untimed setup)."""
     from oracle import turboquant as tq
     d = synth.KV_DIM
     X = synth.kv_vectors(rows, d, seed=seed + 10)
-    s = synth.random_signs(d, seed=seed + 2)
+    P = tq.rotation_qr(synth.gaussian_matrix(d, seed=TQ_PI_SEED))
     c, t = tq.lloyd_max(d, 4)
 
     def run():
-        codes, gamma, _ = tq.encode(X, s, t)
-        return tq.decode(codes, gamma, s, c)
+        codes, gamma, _ = tq.encode(X, P, t)
+        return tq.decode(codes, gamma, P, c)
     import oracle
     return run, rows, oracle.max_threads()
 
 
 def run_tq(args, world, rank, local):
     """The 3DTurboQuant KV-cache codec on the page's DUSt3R case: 24576 vectors
-    of d = 1024 (100.7 MB of fp32), b = 4; a step encodes and decodes one batch."""
+    of d = 1024 (100.7 MB of fp32), b = 4; a step encodes and decodes one batch
+    with the page's rotation (the Q factor of a Gaussian matrix, a dense
+    product on the tensor cores).  The signed-Hadamard fast variant is timed
+    beside it."""
     import torch
     from w4a4_post_quantized_b200 import w4a4
     n, d = synth.KV_VECTORS, synth.KV_DIM
@@ -951,13 +959,18 @@ def run_tq(args, world, rank, local):
     c, t = w4a4.tq_codebook(d, 4)
     cd, td = torch.from_numpy(c).to(dev), torch.from_numpy(t).to(dev)
     seed = 1000 * rank
+    # the rotation: QR on the host, once (untimed, like weight preparation)
+    hi, lo, thi, tlo = [torch.from_numpy(a).to(dev)
+                        for a in w4a4.tq_rotation_qr(synth.gaussian_matrix(d, seed=TQ_PI_SEED))]
     sg = torch.from_numpy(synth.random_signs(d, seed=seed + 2)).to(dev)
     Xs = [torch.from_numpy(synth.kv_vectors(n, d, seed=seed + 10 + i)).to(dev) for i in range(NSETS)]
     Cs = [torch.empty((n, d // 2), dtype=torch.uint8, device=dev) for _ in range(NSETS)]
     Ns = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(NSETS)]
     Ys = [torch.empty((n, d), dtype=torch.float32, device=dev) for _ in range(NSETS)]
-    enc = lambda j: w4a4.tq_encode(Xs[j], sg, td, codes=Cs[j], norms=Ns[j])
-    dec = lambda j: w4a4.tq_decode(Cs[j], Ns[j], sg, cd, Y=Ys[j])
+    enc = lambda j: w4a4.tq_encode_dense(Xs[j], hi, lo, td, codes=Cs[j], norms=Ns[j])
+    dec = lambda j: w4a4.tq_decode_dense(Cs[j], Ns[j], thi, tlo, cd, Y=Ys[j])
+    fenc = lambda j: w4a4.tq_encode(Xs[j], sg, td, codes=Cs[j], norms=Ns[j])
+    fdec = lambda j: w4a4.tq_decode(Cs[j], Ns[j], sg, cd, Y=Ys[j])
 
     def step(i):
         enc(i % NSETS)
@@ -980,7 +993,7 @@ def run_tq(args, world, rank, local):
         barrier(world)
         iso = {}
         n_iso = max(3, min(args.steps, 200))
-        for name, fn in (("encode", enc), ("decode", dec)):
+        for name, fn in (("encode", enc), ("decode", dec), ("fast_encode", fenc), ("fast_decode", fdec)):
             for i in range(3):
                 fn(i % NSETS)
             k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -995,12 +1008,17 @@ def run_tq(args, world, rank, local):
     ms_step = elapsed_ms / args.steps
     be, bd = tq_bytes(n, d)
     value = world * (be + bd) * args.steps / (elapsed_ms * 1e-3) / 1e9
-    # reconstruction quality of the timed batch 0 against the page's bound
-    step(0)
-    torch.cuda.synchronize()
-    X64 = Xs[0].double()
-    rel = (((X64 - Ys[0].double()) ** 2).sum(1) / (X64 ** 2).sum(1))
+    # reconstruction quality of batch 0 against the page's bound, both variants
     bound = math.sqrt(3.0) * math.pi / 2.0 * 4.0 ** -4
+    X64 = Xs[0].double()
+    quality = {}
+    for name, (e_, d_) in (("page_rotation", (enc, dec)), ("fast_variant", (fenc, fdec))):
+        e_(0)
+        d_(0)
+        torch.cuda.synchronize()
+        rel = (((X64 - Ys[0].double()) ** 2).sum(1) / (X64 ** 2).sum(1))
+        quality[name] = {"mse_rel_mean": float(rel.mean()), "mse_rel_max": float(rel.max())}
+    quality.update({"page_bound": bound, "compression_vs_fp32": (4 * n * d) / (n * (d // 2) + 4 * n)})
     # end to end: X from pinned host memory, encode + decode, Y back to pinned host memory
     Xh = Xs[0].cpu().pin_memory()
     Yh = torch.empty((n, d), dtype=torch.float32, pin_memory=True)
@@ -1008,8 +1026,8 @@ def run_tq(args, world, rank, local):
 
     def host_step():
         Xd.copy_(Xh, non_blocking=True)
-        w4a4.tq_encode(Xd, sg, td, codes=Cs[0], norms=Ns[0])
-        w4a4.tq_decode(Cs[0], Ns[0], sg, cd, Y=Yd)
+        w4a4.tq_encode_dense(Xd, hi, lo, td, codes=Cs[0], norms=Ns[0])
+        w4a4.tq_decode_dense(Cs[0], Ns[0], thi, tlo, cd, Y=Yd)
         Yh.copy_(Yd, non_blocking=True)
     for _ in range(3):
         host_step()
@@ -1024,34 +1042,45 @@ def run_tq(args, world, rank, local):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(world, a0.elapsed_time(a1)) / e2e_steps
     peaks = load_peaks()
-    kern = "tq_encode_kernel" if iso["encode"] >= iso["decode"] else "tq_decode_kernel"
-    kb = be if kern == "tq_encode_kernel" else bd
-    kms = max(iso["encode"], iso["decode"])
-    ach = kb / (kms * 1e-3) / 1e9
+    # the dense codec is a contraction: 2 n d^2 flops per kernel (the method's
+    # product), run as three tf32 products for fp32-level accuracy; its peak is
+    # the tf32 rate = the measured bf16 burst x the nominal tf32 : bf16 ratio
+    tf32_peak = peaks["bf16"] * TF32_PER_BF16
+    kern = "encode" if iso["encode"] >= iso["decode"] else "decode"
+    kms = iso[kern]
+    flops = 2.0 * n * d * d
+    ach = flops / (kms * 1e-3) / 1e12
     line = {
         "metric": TQ_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32 in/out, u4 codes", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32 in/out, u4 codes, tf32x3 products", "data": "synthetic",
         "vectors_per_s": world * n * args.steps / (elapsed_ms * 1e-3),
-        "config": {"workload": "3DTurboQuant DUSt3R KV cache: 24576 x 1024 fp32 (100.7 MB), b = 4",
+        "config": {"workload": "3DTurboQuant DUSt3R KV cache: 24576 x 1024 fp32 (100.7 MB), b = 4, "
+                               "the page's rotation (Q of a seeded Gaussian matrix)",
                    "n": n, "d": d, "bits": 4, "per_rank_batch": n,
                    "parallelism": f"dp{world} (independent replicas)",
                    "l2": f"inputs/outputs rotated over {NSETS} buffer sets (~{(8 * n * d + n * d // 2) * NSETS / 1e6:.0f} MB > L2)"},
         "clocks": clk.summary(),
         "e2e": {"value": world * (be + bd) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 4 * n * d, "d2h_bytes_per_step": 4 * n * d,
-                "api": "tq_encode + tq_decode (C ABI) with X copied from and Y copied to pinned host memory"},
+                "api": "tq_encode_dense + tq_decode_dense (C ABI) with X copied from and Y copied to pinned host memory"},
         "gpu_launches": 2 * args.steps,
-        "roofline": {"bound": "hbm", "kernel": kern, "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": ach / peaks["hbm"],
-                     "traffic": profile_traffic("tq.cu", f"{kern.split('_kernel')[0]}_kv_turboquant"),
-                     "ms_per_launch": kms, "algorithmic_bytes_per_launch": kb,
+        "roofline": {"bound": "tensor", "kernel": f"tq_dense_kernel ({kern})", "achieved": ach,
+                     "peak": tf32_peak, "unit": "TFLOP/s", "frac": ach / tf32_peak,
+                     "traffic": None, "ms_per_launch": kms, "algorithmic_flops_per_launch": flops,
+                     "executed_tflops_3_terms": 3 * ach,
+                     "peak_note": f"tf32 = {TF32_PER_BF16:.3f} x {peaks['src']} bf16 burst {peaks['bf16']} TFLOP/s "
+                                  "(nominal 1.1 : 2.25 PFLOP/s)",
                      "encode_ms": iso["encode"], "decode_ms": iso["decode"],
-                     "encode_gbs": be / (iso["encode"] * 1e-3) / 1e9,
-                     "decode_gbs": bd / (iso["decode"] * 1e-3) / 1e9,
                      "timing": f"CUDA events around {n_iso} back-to-back launches of each kernel alone"},
-        "quality": {"mse_rel_mean": float(rel.mean()), "mse_rel_max": float(rel.max()),
-                    "page_bound": bound, "compression_vs_fp32": (4 * n * d) / (n * (d // 2) + 4 * n)},
+        "fast_variant": {
+            "what": "tq_encode / tq_decode: Pi = H diag(s) / sqrt(d) (signed Hadamard, not the page's matrix), "
+                    "HBM-bound", "encode_ms": iso["fast_encode"], "decode_ms": iso["fast_decode"],
+            "encode_gbs": be / (iso["fast_encode"] * 1e-3) / 1e9,
+            "decode_gbs": bd / (iso["fast_decode"] * 1e-3) / 1e9,
+            "encode_frac_hbm": be / (iso["fast_encode"] * 1e-3) / 1e9 / peaks["hbm"],
+            "decode_frac_hbm": bd / (iso["fast_decode"] * 1e-3) / 1e9 / peaks["hbm"]},
+        "quality": quality,
         "device_status": status,
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -1092,7 +1121,9 @@ def run_tq_reference(args, world, rank):
     line = {"impl": "reference", "metric": TQ_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "3DTurboQuant DUSt3R KV cache, d = 1024, b = 4", "n_sampled": r},
+            "config": {"workload": "3DTurboQuant DUSt3R KV cache: 24576 x 1024 fp32 (100.7 MB), b = 4, "
+                                   "the page's rotation (Q of a seeded Gaussian matrix)",
+                       "n": synth.KV_VECTORS, "d": d, "bits": 4, "n_sampled": r},
             "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": f"{r} of {synth.KV_VECTORS} vectors per step"},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

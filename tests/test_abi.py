@@ -404,3 +404,27 @@ def test_noalloc_argument_order(lib):
     assert f(A, 4089, ctypes.byref(_weights(K=4096)), A, 0, None) == 2
     assert f(A, -1, ctypes.byref(w), A, 0, None) == 2
     assert f(A, 10, None, A, 0, None) == 1
+
+
+def test_tq_rotation_qr_on_the_host(lib):
+    """tq_rotation_qr (host code, no GPU): the library's Householder QR gives
+    the oracle's sign-fixed Q factor (numpy's QR) of the same Gaussian matrix;
+    its tf32 terms carry Pi to 2^-21 relative, the hi terms have the 13 low
+    mantissa bits clear, and the Pi^T terms are the transposes."""
+    import numpy as np
+    from oracle import turboquant as tq
+    from w4a4_post_quantized_b200 import synth
+    vp = ctypes.c_void_p
+    lib.tq_rotation_qr.argtypes = [vp, ctypes.c_int32, vp, vp, vp, vp]
+    lib.tq_rotation_qr.restype = ctypes.c_int
+    d = 1024
+    G = synth.gaussian_matrix(d, seed=5)
+    out = [np.empty((d, d), np.float32) for _ in range(4)]
+    assert lib.tq_rotation_qr(G.ctypes.data_as(vp), d, *[o.ctypes.data_as(vp) for o in out]) == 0
+    P = tq.rotation_qr(G)
+    hi, lo = out[0].astype(np.float64), out[1].astype(np.float64)
+    assert np.max(np.abs(hi + lo - P) / np.abs(P)) < 2.0 ** -21
+    assert np.all((out[0].view(np.uint32) & 0x1FFF) == 0) and np.all((out[1].view(np.uint32) & 0x1FFF) == 0)
+    assert np.array_equal(out[2], out[0].T) and np.array_equal(out[3], out[1].T)
+    assert lib.tq_rotation_qr(G.ctypes.data_as(vp), 512, *[o.ctypes.data_as(vp) for o in out]) == 4
+    assert lib.tq_rotation_qr(None, d, *[o.ctypes.data_as(vp) for o in out]) == 1

@@ -80,6 +80,9 @@ _clear_status = _sig("w4a4_clear_device_status", ctypes.c_int, [_vp])
 _tq_codebook = _sig("tq_codebook", ctypes.c_int, [_i32, _i32, _vp, _vp])
 _tq_encode = _sig("tq_encode", ctypes.c_int, [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp])
 _tq_decode = _sig("tq_decode", ctypes.c_int, [_vp, _vp, _i64, _i32, _vp, _vp, _vp, _vp])
+_tq_rotation_qr = _sig("tq_rotation_qr", ctypes.c_int, [_vp, _i32, _vp, _vp, _vp, _vp])
+_tq_encode_dense = _sig("tq_encode_dense", ctypes.c_int, [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp])
+_tq_decode_dense = _sig("tq_decode_dense", ctypes.c_int, [_vp, _vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp])
 _status_string = _sig("w4a4_status_string", ctypes.c_char_p, [ctypes.c_int])
 _version = _sig("w4a4_version", ctypes.c_char_p, [])
 
@@ -340,4 +343,39 @@ def tq_decode(codes: torch.Tensor, norms: torch.Tensor, signs: torch.Tensor, cen
     Y = Y if Y is not None else torch.empty((n, d), dtype=torch.float32, device=codes.device)
     _check(_tq_decode(_ptr(codes), _ptr(norms), n, d, _ptr(signs), _ptr(centroids), _ptr(Y),
                       _stream(stream)), "tq_decode")
+    return Y
+
+
+# ---------------------------------- the page's dense rotation (QR of a Gaussian)
+def tq_rotation_qr(G):
+    """Host: Pi = the sign-fixed Q factor of the d x d Gaussian matrix G (numpy
+    float64), as tf32 hi / lo terms of Pi and of Pi^T: returns
+    (pi_hi, pi_lo, pit_hi, pit_lo), numpy float32 [d, d] each."""
+    import numpy as np
+    G = np.ascontiguousarray(G, dtype=np.float64)
+    d = G.shape[0]
+    out = [np.empty((d, d), np.float32) for _ in range(4)]
+    _check(_tq_rotation_qr(G.ctypes.data_as(_vp), d, *[o.ctypes.data_as(_vp) for o in out]),
+           "tq_rotation_qr")
+    return tuple(out)
+
+
+def tq_encode_dense(X: torch.Tensor, pi_hi: torch.Tensor, pi_lo: torch.Tensor, boundaries: torch.Tensor,
+                    codes=None, norms=None, stream=None):
+    """X [n, d] fp32 -> (codes uint8 [n, d/2], norms fp32 [n]) with the dense Pi."""
+    n, d = X.shape
+    codes = codes if codes is not None else torch.empty((n, d // 2), dtype=torch.uint8, device=X.device)
+    norms = norms if norms is not None else torch.empty(n, dtype=torch.float32, device=X.device)
+    _check(_tq_encode_dense(_ptr(X), n, d, _ptr(pi_hi), _ptr(pi_lo), _ptr(boundaries), _ptr(codes),
+                            _ptr(norms), _stream(stream)), "tq_encode_dense")
+    return codes, norms
+
+
+def tq_decode_dense(codes: torch.Tensor, norms: torch.Tensor, pit_hi: torch.Tensor, pit_lo: torch.Tensor,
+                    centroids: torch.Tensor, Y=None, stream=None):
+    """(codes [n, d/2], norms [n]) -> Y [n, d] fp32 with the dense Pi."""
+    n, d = codes.shape[0], codes.shape[1] * 2
+    Y = Y if Y is not None else torch.empty((n, d), dtype=torch.float32, device=codes.device)
+    _check(_tq_decode_dense(_ptr(codes), _ptr(norms), n, d, _ptr(pit_hi), _ptr(pit_lo), _ptr(centroids),
+                            _ptr(Y), _stream(stream)), "tq_decode_dense")
     return Y
