@@ -369,8 +369,8 @@ def test_gelu_on_output(w4, route):
     erf in fp64, rounded to bf16) of the same call's output without the flag,
     on an fc1-shaped layer (K = 1024, N = 4096), through every GEMM route and
     the W8A8 setting.
-    Below -5.9 the kernel's GELU returns -0 (or the exact value): the exact
-    GELU there is below 1e-8 of the input in magnitude."""
+    Below -5.9375 the kernel's GELU is the constant -5.9375 Phi(-5.9375)
+    (-8.6e-9): the exact GELU there lies between it and 0."""
     M, N, K = 300, 4096, 1024
     X = synth.activations(M, K, seed=820)
     W, b = synth.weights(N, K, seed=821), synth.bias(N, seed=822)
@@ -390,11 +390,12 @@ def test_gelu_on_output(w4, route):
     y1 = host(Y1.view(torch.int16)).view(np.uint16)
     want = oracle.gelu_bf16(y0)
     f0 = synth.bf16_bits_to_f32(y0).astype(np.float64)
-    far = f0 < -5.9
+    far = f0 < -5.9375
     assert far.sum() > 0 and (~far).sum() > 0.9 * f0.size   # both branches exercised
     assert np.array_equal(y1[~far], want[~far])
     f1 = synth.bf16_bits_to_f32(y1[far]).astype(np.float64)
-    assert np.all((y1[far] == 0x8000) | (y1[far] == want[far]))
+    assert len(set(y1[far].tolist())) == 1
+    assert np.all(f1 <= oracle.bf16_to_f64(want[far]))
     assert np.all(np.abs(f1) <= 1e-8 * np.abs(f0[far]))
     assert w4.w4a4_get_device_status() == 0
 

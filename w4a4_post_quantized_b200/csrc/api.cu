@@ -243,6 +243,7 @@ w4a4_status w4a4_linear_ex(const uint8_t *qx, const float *scale_tok, int64_t M,
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, scale_tok, w->scale_ch, w->bias, Y, nullptr,
                    M, w->N, w->K, int8_weights(w) || (flags & W4A4_FLAG_UNPACKED) != 0,
                    (flags & W4A4_FLAG_GELU_OUT) != 0};
+  a.acc22 = !int8_weights(w);
   return cuda_status(w4a4::launch_gemm(a, as_stream(stream)));
 }
 
@@ -278,6 +279,7 @@ w4a4_status w4a4_linear_fused(const uint16_t *X, int64_t M, const w4a4_weights_t
   if (e != cudaSuccess) return cuda_status(e);
   w4a4::GemmArgs a{qx, w->qw, w->qw8, w->colsum, st, w->scale_ch, w->bias, Y, nullptr,
                    M, w->N, w->K, one_per_byte(cf), (flags & W4A4_FLAG_GELU_OUT) != 0};
+  a.acc22 = !int8_weights(w);
   return cuda_status(w4a4::launch_gemm(a, cs));
 }
 

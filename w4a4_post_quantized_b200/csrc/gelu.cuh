@@ -8,15 +8,18 @@
 namespace w4a4 {
 namespace {
 
-// GELU(x) = x Phi(x) of two bf16 inputs, rounded to bf16 (the activation an
-// MLP's second linear receives).  Phi(-|x|) = erfc(z) / 2, z = |x| / sqrt 2,
-// is evaluated as exp2(-log2(e) z^2 + c(u)), u = z / 2.1 - 1, for z <= 4.2: the
-// exp(-z^2 + polynomial) form of Numerical Recipes' erfcc (section 6.2), with
-// c a degree-11 fit in z by w4a4_post_quantized_b200/gelu_fit.py (relative
-// error of erfc 6.5e-8 in fp64; factor 1/2 folded in).  For z > 4.2,
-// Phi(-|x|) < 1.4e-9 is taken as 0.  Then GELU = x - x Phi(-x) for x >= 0 and
-// x Phi(-|x|) for x < 0, with no cancellation on either side.  Pairs of inputs
-// share packed fp32x2 arithmetic.
+// GELU(x) = x Phi(x) of a bf16 pair, rounded to bf16 (the activation an MLP's
+// second linear receives), as
+//     GELU(x) = max(x, 0) - a Phi(-a),   a = min(|x|, 5.9375)  (one fma),
+// with no cancellation on either side, and Phi(-a) = exp2(c(u)),
+// u = a / 2.96875 - 1, c the degree-10 fit of log2 Phi(-a) on [0, 5.9375]
+// made by w4a4_post_quantized_b200/gelu_fit.py (the Gaussian's -a^2 / (2 ln 2)
+// is part of the polynomial).  For every bf16 input with |x| <= 5.9375 the
+// result is the exact GELU rounded to bf16 (checked exhaustively on the host
+// with room for ex2.approx's error); above, it rounds to x as the exact GELU
+// does, and below -5.9375 it is the constant -5.9375 Phi(-5.9375) = -8.6e-9
+// (the exact values lie in (-8.6e-9, 0)).  Pairs share packed fp32x2
+// arithmetic: 21 instructions per pair.
 __device__ __forceinline__ unsigned long long f2(float a, float b) {
   unsigned long long r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
@@ -31,42 +34,42 @@ __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigne
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-__device__ __forceinline__ void gelu2_bf16(float &x0, float &x1) {
-  constexpr float kZ = 4.2f;
-  constexpr float kC[12] = {-3.02844500541687f,     -1.222137451171875f,   0.4550056755542755f,
-                            -0.20184531807899475f,  0.09051182866096497f,  -0.03863636031746864f,
-                            0.0148030836135149f,    -0.004897787235677242f, 0.0015472964150831103f,
-                            -5.184028486837633e-05f, -0.0006587805110029876f, 0.0003328344027977437f};
-  const float z0 = fabsf(x0) * 0.70710678118654752f, z1 = fabsf(x1) * 0.70710678118654752f;
-  const unsigned long long z = f2(z0, z1);
-  const unsigned long long u = fma2(z, f2(2.0f / kZ, 2.0f / kZ), f2(-1.0f, -1.0f));
-  unsigned long long p = f2(kC[11], kC[11]);
+// GELU of the two bf16 values of a packed pair (element 0 in the low half),
+// bf16 pair out.
+__device__ __forceinline__ uint32_t gelu_pair_bf16(uint32_t w) {
+  constexpr float kA = 5.9375f;
+  constexpr float kC[11] = {-9.38557243347168f,     -13.937177658081055f,   -5.902686595916748f,
+                            -0.20182649791240692f,  0.0904492437839508f,    -0.038198795169591904f,
+                            0.014783327467739582f,  -0.0058014956302940845f, 0.001542369951494038f,
+                            0.0008624561014585197f, -0.0006574652506969869f};
+  const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xFFFF0000u);
+  // na = -a = max(-|x|, -A)
+  const unsigned long long na = f2(fmaxf(-fabsf(x0), -kA), fmaxf(-fabsf(x1), -kA));
+  const unsigned long long u = fma2(na, f2(-2.0f / kA, -2.0f / kA), f2(-1.0f, -1.0f));
+  unsigned long long p = f2(kC[10], kC[10]);
 #pragma unroll
-  for (int i = 10; i >= 0; --i) p = fma2(p, u, f2(kC[i], kC[i]));
-  const float nl2e = -1.4426950408889634f;
-  float a0, a1;
-  f2_split(fma2(mul2(z, z), f2(nl2e, nl2e), p), a0, a1);
-  const float ph0 = z0 <= kZ ? ex2_approx(a0) : 0.0f;  // Phi(-|x|)
-  const float ph1 = z1 <= kZ ? ex2_approx(a1) : 0.0f;
-  const unsigned long long ph = f2(ph0, ph1), x = f2(x0, x1);
-  float pos0, pos1, neg0, neg1;
-  f2_split(fma2(f2(-x0, -x1), ph, x), pos0, pos1);  // x - x Phi(-x)
-  f2_split(mul2(x, ph), neg0, neg1);                 // x Phi(x), x < 0
-  const float g0 = x0 >= 0.0f ? pos0 : neg0, g1 = x1 >= 0.0f ? pos1 : neg1;
+  for (int i = 9; i >= 0; --i) p = fma2(p, u, f2(kC[i], kC[i]));
+  float e0, e1;
+  f2_split(p, e0, e1);
+  // max(x, 0) - a Phi(-a), one rounding
+  float g0, g1;
+  f2_split(fma2(na, f2(ex2_approx(e0), ex2_approx(e1)), f2(fmaxf(x0, 0.0f), fmaxf(x1, 0.0f))), g0, g1);
   const __nv_bfloat162 h = __floats2bfloat162_rn(g0, g1);
-  x0 = __low2float(h);
-  x1 = __high2float(h);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// The same on two floats holding bf16 values; the results are bf16 values.
+__device__ __forceinline__ void gelu2_bf16(float &x0, float &x1) {
+  const uint32_t w = (__float_as_uint(x1) & 0xFFFF0000u) | (__float_as_uint(x0) >> 16);
+  const uint32_t g = gelu_pair_bf16(w);
+  x0 = __uint_as_float(g << 16);
+  x1 = __uint_as_float(g & 0xFFFF0000u);
 }
 
 }  // namespace

@@ -239,14 +239,7 @@ __device__ __forceinline__ uint32_t dequant2_bf16_cvt(int32_t a0, int32_t a1, fl
   return pack_bf16x2(y0, y1);
 }
 
-// GELU of the two bf16 values of a packed pair (bf16 in, bf16 out).
-__device__ __forceinline__ uint32_t gelu_pair_bf16(uint32_t w) {
-  float a = __uint_as_float(w << 16), b = __uint_as_float(w & 0xFFFF0000u);
-  gelu2_bf16(a, b);
-  return (__float_as_uint(b) & 0xFFFF0000u) | (__float_as_uint(a) >> 16);
-}
-
-template <int MODE, bool OUT_S32, bool GELU_OUT = false>
+template <int MODE, bool OUT_S32, bool GELU_OUT = false, bool ACC22 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmY, const float *__restrict__ scale_tok,
@@ -574,7 +567,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int u = 0; u < 2; ++u)
                 pk[h][u][j] =
-                    P::A8 ? dequant2_bf16_cvt(static_cast<int32_t>(r[h][4 * j + 2 * u]),
+                    (P::A8 && !ACC22) ? dequant2_bf16_cvt(static_cast<int32_t>(r[h][4 * j + 2 * u]),
                                               static_cast<int32_t>(r[h][4 * j + 2 * u + 1]),
                                               st4[2 * h + u], scl.x, scl.y, bi.x, bi.y)
                           : dequant2_bf16(static_cast<int32_t>(r[h][4 * j + 2 * u]) + o.x,
@@ -743,10 +736,10 @@ bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uin
   return encode_tensor_map_2d(map, dt, base, inner, outer, row_bytes, box_inner, box_outer, swz);
 }
 
-template <int MODE, bool OUT_S32, bool GELU_OUT = false>
+template <int MODE, bool OUT_S32, bool GELU_OUT = false, bool ACC22 = false>
 cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   using P = Plan<MODE>;
-  auto kern = w4a4_gemm_kernel<MODE, OUT_S32, GELU_OUT>;
+  auto kern = w4a4_gemm_kernel<MODE, OUT_S32, GELU_OUT, ACC22>;
   static ContextCache<bool> attr_set;  // the shared-memory attribute, per context
   bool done = false;
   cudaError_t e = attr_set.get(&done, [&](bool *v) {
@@ -819,12 +812,20 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st) {
   // byte operands: 128 x 128 tiles when 128 x 256 ones would fill at most half of the SMs
   const int64_t wide_tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
   const bool narrow = a.a8 && 2 * wide_tiles <= device_sm_count();
+  // byte operands with small accumulators (4-bit weight codes): exact integer-add conversion
+  const bool acc22 = a.acc22 && a.K <= 4096;
   if (a.gelu_out) {
     if (a.acc) return cudaErrorInvalidValue;
+    if (a.a8 && acc22)
+      return narrow ? launch_t<kInt8Narrow, false, true, true>(a, st)
+                    : launch_t<kInt8, false, true, true>(a, st);
     if (a.a8)
       return narrow ? launch_t<kInt8Narrow, false, true>(a, st) : launch_t<kInt8, false, true>(a, st);
     return a.qw8 ? launch_t<kExpanded, false, true>(a, st) : launch_t<kPacked, false, true>(a, st);
   }
+  if (!a.acc && a.a8 && acc22)
+    return narrow ? launch_t<kInt8Narrow, false, false, true>(a, st)
+                  : launch_t<kInt8, false, false, true>(a, st);
   if (narrow) return a.acc ? launch_t<kInt8Narrow, true>(a, st) : launch_t<kInt8Narrow, false>(a, st);
   if (a.a8) return a.acc ? launch_t<kInt8, true>(a, st) : launch_t<kInt8, false>(a, st);
   const bool packed = (a.qw8 == nullptr);

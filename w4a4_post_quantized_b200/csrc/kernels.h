@@ -44,6 +44,10 @@ struct GemmArgs {
   bool gelu_out = false;    // y = bf16(GELU(bf16 result)) (an MLP's first linear)
   bool stall = false;       // failure-path test: the TMA producer issues nothing and every
                             // bounded wait gives up after 1 ms (sets the status word)
+  bool acc22 = false;       // every accumulator is below 2^22 in magnitude (4-bit weight codes
+                            // in [-7, 7], activation bytes in [-128, 127], K <= 4096): with
+                            // byte operands the epilogue converts them with the exact
+                            // integer-add bias instead of the int -> float conversion
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st);
 cudaError_t launch_expand_weights(const uint8_t *qw, int N, int K, int8_t *qw8, int32_t *colsum,
