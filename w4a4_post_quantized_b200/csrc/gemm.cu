@@ -105,23 +105,33 @@ constexpr uint32_t TMEM_COLS = 512;     // the whole tensor memory of the SM
 //     256-column accumulators.  The narrow variant (128 x 128 tiles, 6 stages
 //     of 32 KB) serves shapes whose 128 x 256 tiles would leave more than
 //     half of the SMs idle (a single frame: 44 tiles), doubling the tiles.
-enum : int { kExpanded = 0, kPacked = 1, kInt8 = 2, kInt8Narrow = 3 };
+//   int8 pair: the same operands for a CTA pair (a cluster of 2) sharing a
+//     256 x 256 tile: each CTA loads its 128 rows of A and 128 rows of B
+//     (6 stages of 32 KB), the leader issues cta_group::2 MMAs that read both
+//     CTAs' halves, and each CTA's tensor memory holds its 128 rows x 256
+//     columns (two buffers), drained by its own epilogue.  Per multiply-add a
+//     CTA loads and the tensor cores read a third less shared memory than a
+//     128 x 256 tile of one CTA, and the same stage bytes cover 1.5x the time.
+enum : int { kExpanded = 0, kPacked = 1, kInt8 = 2, kInt8Narrow = 3, kInt8Pair = 4 };
 
 template <int MODE>
 struct Plan {
   static constexpr bool B_PACKED = MODE == kPacked;
   static constexpr bool A_TMEM = MODE == kExpanded;
   static constexpr bool NARROW = MODE == kInt8Narrow;
-  static constexpr bool A8 = MODE == kInt8 || NARROW;  // both operands one code per byte
+  static constexpr bool PAIR = MODE == kInt8Pair;
+  static constexpr bool A8 = MODE == kInt8 || NARROW || PAIR;  // both operands one code per byte
   static constexpr bool EPI16 = !B_PACKED;           // 16x256b epilogue fragments
   static constexpr int TN = A_TMEM ? 192 : (NARROW ? 128 : BN);  // tile columns
-  static constexpr int STAGES = B_PACKED ? 3 : (NARROW ? 6 : (A8 ? 4 : 5));  // TMA stages
+  static constexpr int TNL = PAIR ? TN / 2 : TN;     // B rows a CTA loads
+  static constexpr int TM = PAIR ? 2 * BM : BM;      // tile rows (of the pair)
+  static constexpr int STAGES = B_PACKED ? 3 : ((NARROW || PAIR) ? 6 : (A8 ? 4 : 5));  // TMA stages
   static constexpr int KG = A_TMEM ? 2 : 1;          // k-blocks per widen -> MMA handshake
   static constexpr int WSLOTS = A8 ? 0 : 2;          // widened operand slots
   static constexpr int A_ST = A8 ? A_UN : A_PK;      // A bytes of a stage
   static constexpr int OFF_ST_A = 0;                 // A: packed [BM x 64 B] or int8 [BM x 128 B] (swizzled)
   static constexpr int OFF_ST_B = A_ST;              // B: int8 [TN x 128 B] (swizzled) or packed
-  static constexpr int STAGE_BYTES = A_ST + (B_PACKED ? B_PK : TN * BK);
+  static constexpr int STAGE_BYTES = A_ST + (B_PACKED ? B_PK : TNL * BK);
   static constexpr int OFF_W = STAGES * STAGE_BYTES;
   static constexpr int OFF_W_A = 0;                  // widened A [BM x 128 B] (swizzled)
   static constexpr int OFF_W_B = A_UN;               // widened B (B_PACKED only)
@@ -140,10 +150,10 @@ struct Plan {
                     WSLOT_BYTES % 1024 == 0 && OFF_EPI % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
   // tcgen05.mma kind::i8 instruction descriptor: s32 D; A unsigned (code + 8)
-  // with expanded B, signed otherwise; B signed; both K-major; 128 x TN.
+  // with expanded B, signed otherwise; B signed; both K-major; TM x TN.
   static constexpr uint32_t IDESC = (2u << 4) | ((A_TMEM ? 0u : 1u) << 7) | (1u << 10) |
                                     (static_cast<uint32_t>(TN >> 3) << 17) |
-                                    (static_cast<uint32_t>(BM >> 4) << 24);
+                                    (static_cast<uint32_t>(TM >> 4) << 24);
 };
 
 constexpr int W_TMA = 0, W_MMA = 1, W_TMEM = 2;
@@ -267,6 +277,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // a CTA pair works on the pair's tiles; rank 0 (the leader) issues the MMAs
+  constexpr bool PAIR = P::PAIR;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(nclusters_x()) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -279,7 +294,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], (GELU_OUT && P::A8 ? 2 : 1) * NUM_EPI_WARPS);
+      // (a pair's leader counts the epilogue warps of both CTAs)
+      mbar_init(&acc_empty[b], (GELU_OUT && P::A8 ? 2 : 1) * NUM_EPI_WARPS * (PAIR ? 2 : 1));
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -291,11 +307,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (!OUT_S32) tma_prefetch_desc(&tmY);
   }
   if (warp == W_TMEM) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // Everything above (barriers, tensor memory, descriptor prefetch) may overlap
@@ -311,34 +333,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       // stall (a test of the failure path, w4a4_gemm_s32_ex with W4A4_DEBUG_STALL):
       // no copy is ever issued, so the consumers' first waits run out
-      for (int tile = blockIdx.x; tile < num_tiles && ok && !stall; tile += gridDim.x) {
+      for (int tile = unit0; tile < num_tiles && ok && !stall; tile += units) {
         const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
         for (int kb = 0; kb < num_kb; ++kb) {
           const uint32_t s = issued % ST, ph = (issued / ST) & 1u;
-          if (!mbar_wait(&freed[s], ph ^ 1u, abort_flag, &g_status, wait_ns)) {
+          if (!mbar_wait<PAIR>(&freed[s], ph ^ 1u, abort_flag, &g_status, wait_ns)) {
             ok = false;
             break;
           }
           uint8_t *stage = smem + s * P::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], P::STAGE_BYTES);
-          tma_load_2d(stage + P::OFF_ST_A, &tmA, P::A8 ? kb * BK : kb * BKP, mb * BM, &full[s]);
-          tma_load_2d(stage + P::OFF_ST_B, &tmB, B_PACKED ? kb * BKP : kb * BK, nb * P::TN, &full[s]);
+          if constexpr (PAIR) {
+            // both CTAs' bytes land on the leader's barrier, which the leader arms
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * P::STAGE_BYTES);
+            const uint32_t bar0 = cluster_addr(&full[s], 0);
+            tma_load_2d_pair(stage + P::OFF_ST_A, &tmA, kb * BK, mb * P::TM + static_cast<int>(rank) * BM,
+                             bar0);
+            tma_load_2d_pair(stage + P::OFF_ST_B, &tmB, kb * BK,
+                             nb * P::TN + static_cast<int>(rank) * P::TNL, bar0);
+          } else {
+            mbar_arrive_expect_tx(&full[s], P::STAGE_BYTES);
+            tma_load_2d(stage + P::OFF_ST_A, &tmA, P::A8 ? kb * BK : kb * BKP, mb * BM, &full[s]);
+            tma_load_2d(stage + P::OFF_ST_B, &tmB, B_PACKED ? kb * BKP : kb * BK, nb * P::TN, &full[s]);
+          }
           ++issued;
         }
       }
-      // let every issued copy land before the CTA can exit
-      for (uint32_t t = (issued > ST ? issued - ST : 0); t < issued; ++t)
-        mbar_wait_drain(&full[t % ST], (t / ST) & 1u, &g_status, wait_ns);
+      // let every issued copy land before the CTA can exit (a pair's copies
+      // complete on the leader's barriers: the leader waits for both CTAs',
+      // and the closing cluster barrier holds the other CTA until then)
+      if (!PAIR || rank == 0)
+        for (uint32_t t = (issued > ST ? issued - ST : 0); t < issued; ++t)
+          mbar_wait_drain<PAIR>(&full[t % ST], (t / ST) & 1u, &g_status, wait_ns);
     }
   } else if (warp == W_MMA) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------- MMA issuer
       uint32_t consumed = 0, group = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      for (int tile = unit0; tile < num_tiles && ok; tile += units, ++it) {
         const uint32_t b = it & 1, pb = (it >> 1) & 1;
-        if (!mbar_wait(&acc_empty[b], pb ^ 1u, abort_flag, &g_status, wait_ns)) break;
+        if (!mbar_wait<PAIR>(&acc_empty[b], pb ^ 1u, abort_flag, &g_status, wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * P::TN;
         if constexpr (P::A_TMEM) {
@@ -369,7 +404,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // both operands straight from the TMA stage
           for (int kb = 0; kb < num_kb; ++kb) {
             const uint32_t s = consumed % ST, ps = (consumed / ST) & 1u;
-            if (!mbar_wait(&full[s], ps, abort_flag, &g_status, wait_ns)) {
+            if (!mbar_wait<PAIR>(&full[s], ps, abort_flag, &g_status, wait_ns)) {
               ok = false;
               break;
             }
@@ -377,10 +412,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t a0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_ST_A);
             const uint32_t b0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_ST_B);
 #pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk)
-              mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), P::IDESC,
-                     (kb | kk) != 0 ? 1u : 0u);
-            tc_commit(&freed[s]);
+            for (int kk = 0; kk < BK / 32; ++kk) {
+              if constexpr (PAIR)
+                mma_i8_pair(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
+                            P::IDESC, (kb | kk) != 0 ? 1u : 0u);
+              else
+                mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), P::IDESC,
+                       (kb | kk) != 0 ? 1u : 0u);
+            }
+            if constexpr (PAIR)
+              tc_commit_pair(&freed[s], 0x3);  // frees the stage in both CTAs
+            else
+              tc_commit(&freed[s]);
             ++consumed;
           }
         } else {
@@ -405,11 +448,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ++consumed;
           }
         }
-        if (ok) tc_commit(&acc_full[b]);
+        if (ok) {
+          if constexpr (PAIR)
+            tc_commit_pair(&acc_full[b], 0x3);
+          else
+            tc_commit(&acc_full[b]);
+        }
       }
-      // every MMA issued must finish before tensor memory is freed
-      tc_commit(mma_done);
-      mbar_wait_drain(mma_done, 0, &g_status, wait_ns);
+      // every MMA issued must finish before tensor memory is freed (a pair's
+      // commit is only issued after pair MMAs: with none, nothing is pending)
+      if constexpr (PAIR) {
+        if (consumed > 0) {
+          tc_commit_pair(mma_done, 0x1);
+          mbar_wait_drain<PAIR>(mma_done, 0, &g_status, wait_ns);
+        }
+      } else {
+        tc_commit(mma_done);
+        mbar_wait_drain(mma_done, 0, &g_status, wait_ns);
+      }
     }
   } else if (!P::A8 && warp >= W_UNPACK0 && warp < W_UNPACK0 + 4) {
     // ------------------------------------------------------------------ widen
@@ -504,7 +560,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float *csc = reinterpret_cast<float *>(coff + TN);
     float *cbi = csc + TN;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int tile = unit0; tile < num_tiles; tile += units, ++it) {
       const uint32_t b = it & 1, pb = (it >> 1) & 1;
       const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
       __syncwarp();  // every lane is done reading the previous tile's constants
@@ -519,9 +575,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       __syncwarp();
-      if (!mbar_wait(&acc_full[b], pb, abort_flag, &g_status, wait_ns)) break;
+      if (!mbar_wait<PAIR>(&acc_full[b], pb, abort_flag, &g_status, wait_ns)) break;
       tc_fence_after();
-      const int row0 = mb * BM + ew * 32;
+      const int row0 = mb * P::TM + static_cast<int>(rank) * BM + ew * 32;
       if constexpr (!OUT_S32 && P::EPI16) {
         // 16x256b fragments: thread t holds rows q = t/4 + 8 i (i < 4) of the
         // warp's 32 rows and, per 8-column group j, columns 8j + 2(t%4) + {0,1};
@@ -544,7 +600,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (sc == (half + 1) * SC_PER - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[b]);
+            if (lane == 0) {
+              if constexpr (PAIR)
+                mbar_arrive_cluster(&acc_empty[b], 0);  // the leader's barrier
+              else
+                mbar_arrive(&acc_empty[b]);
+            }
           }
           const int c0 = sc * EPI_COLS;
           const int n0 = nb * TN + c0;
@@ -625,7 +686,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (sc == TN / EPI_COLS - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[b]);
+          if (lane == 0) {
+            if constexpr (PAIR)
+              mbar_arrive_cluster(&acc_empty[b], 0);
+            else
+              mbar_arrive(&acc_empty[b]);
+          }
         }
         const int c0 = sc * EPI_COLS;
         const int n0 = nb * TN + c0;
@@ -683,8 +749,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the leader's MMAs and the other CTA's reads are done
   tc_fence_after();
-  if (warp == W_TMEM) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == W_TMEM) {
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
+  }
 }
 
 // Expand packed weight codes to the int8 operand order the kernel above
@@ -758,7 +830,7 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   const bool okB = P::B_PACKED ? make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw, kp, a.N, kp,
                                           BKP, BN, CU_TENSOR_MAP_SWIZZLE_NONE)
                             : make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qw8, a.K, a.N,
-                                          a.K, BK, P::TN, CU_TENSOR_MAP_SWIZZLE_128B);
+                                          a.K, BK, P::TNL, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!okB) return cudaErrorInvalidValue;
   if (OUT_S32) {
     tmY = tmA;  // unused
@@ -766,22 +838,44 @@ cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
                           static_cast<uint64_t>(a.N) * 2, EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_128B)) {
     return cudaErrorInvalidValue;
   }
-  const int num_m = static_cast<int>((a.M + BM - 1) / BM);
+  const int num_m = static_cast<int>((a.M + P::TM - 1) / P::TM);
   const int num_n = (a.N + P::TN - 1) / P::TN;
   const int tiles = num_m * num_n;
-  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
   // programmatic stream serialization: the prologue may overlap the previous
   // kernel's tail (the kernel waits for it before reading any input)
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = P::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  int grid;
+  if constexpr (P::PAIR) {
+    // persistent CTA pairs: as many clusters of 2 as can be resident at once
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    static ContextCache<int> clusters;
+    int max_clusters = 0;
+    e = clusters.get(&max_clusters, [&](int *v) {
+      cudaLaunchConfig_t q = cfg;
+      q.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+      q.attrs = &attr[1];
+      q.numAttrs = 1;
+      return cudaOccupancyMaxActiveClusters(v, kern, &q);
+    });
+    if (e != cudaSuccess) return e;
+    if (max_clusters <= 0) return cudaErrorInvalidConfiguration;
+    grid = 2 * (tiles < max_clusters ? tiles : max_clusters);
+  } else {
+    grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  }
+  cfg.gridDim = dim3(grid, 1, 1);
   // a stalled launch (failure-path test) gives every bounded wait 1 ms
   const unsigned long long wait_ns = a.stall ? 1000000ull : kWaitLimitNs;
   e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmY, a.scale_tok, a.scale_ch, a.bias, a.colsum, a.acc,
@@ -814,19 +908,30 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st) {
   const bool narrow = a.a8 && 2 * wide_tiles <= device_sm_count();
   // byte operands with small accumulators (4-bit weight codes): exact integer-add conversion
   const bool acc22 = a.acc22 && a.K <= 4096;
+  // byte operands, enough tiles, a long main loop per tile (K >= 2048, where
+  // the tensor pipe rather than the writes of Y bounds the kernel): CTA pairs
+  // on 256 x 256 tiles (fc2 of the stack 253 -> 227 us); with K = 1024 the
+  // pairs' coupled epilogues lose more than the main loop gains (frame QKV
+  // 30.8 -> 35.5 us), so those keep one CTA per 128 x 256 tile
+  const bool pair = a.a8 && !narrow && a.K >= 2048;
   if (a.gelu_out) {
     if (a.acc) return cudaErrorInvalidValue;
-    if (a.a8 && acc22)
-      return narrow ? launch_t<kInt8Narrow, false, true, true>(a, st)
-                    : launch_t<kInt8, false, true, true>(a, st);
-    if (a.a8)
-      return narrow ? launch_t<kInt8Narrow, false, true>(a, st) : launch_t<kInt8, false, true>(a, st);
+    if (a.a8 && acc22) {
+      if (narrow) return launch_t<kInt8Narrow, false, true, true>(a, st);
+      return pair ? launch_t<kInt8Pair, false, true, true>(a, st) : launch_t<kInt8, false, true, true>(a, st);
+    }
+    if (a.a8) {
+      if (narrow) return launch_t<kInt8Narrow, false, true>(a, st);
+      return pair ? launch_t<kInt8Pair, false, true>(a, st) : launch_t<kInt8, false, true>(a, st);
+    }
     return a.qw8 ? launch_t<kExpanded, false, true>(a, st) : launch_t<kPacked, false, true>(a, st);
   }
-  if (!a.acc && a.a8 && acc22)
-    return narrow ? launch_t<kInt8Narrow, false, false, true>(a, st)
-                  : launch_t<kInt8, false, false, true>(a, st);
+  if (!a.acc && a.a8 && acc22) {
+    if (narrow) return launch_t<kInt8Narrow, false, false, true>(a, st);
+    return pair ? launch_t<kInt8Pair, false, false, true>(a, st) : launch_t<kInt8, false, false, true>(a, st);
+  }
   if (narrow) return a.acc ? launch_t<kInt8Narrow, true>(a, st) : launch_t<kInt8Narrow, false>(a, st);
+  if (pair) return a.acc ? launch_t<kInt8Pair, true>(a, st) : launch_t<kInt8Pair, false>(a, st);
   if (a.a8) return a.acc ? launch_t<kInt8, true>(a, st) : launch_t<kInt8, false>(a, st);
   const bool packed = (a.qw8 == nullptr);
   if (a.acc) return packed ? launch_t<kPacked, true>(a, st) : launch_t<kExpanded, true>(a, st);
