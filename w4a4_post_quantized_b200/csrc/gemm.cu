@@ -112,6 +112,11 @@ constexpr uint32_t TMEM_COLS = 512;     // the whole tensor memory of the SM
 //     columns (two buffers), drained by its own epilogue.  Per multiply-add a
 //     CTA loads and the tensor cores read a third less shared memory than a
 //     128 x 256 tile of one CTA, and the same stage bytes cover 1.5x the time.
+//     The pair synchronises through barriers at CTA scope (the other CTA's
+//     arrivals publish completed tensor-memory reads, the copies and MMAs
+//     complete through their own mechanisms): cluster-scope release /
+//     acquire on those waits and arrivals made the pair slower than one CTA
+//     per tile wherever the epilogue bounds the kernel (K = 1024).
 enum : int { kExpanded = 0, kPacked = 1, kInt8 = 2, kInt8Narrow = 3, kInt8Pair = 4 };
 
 template <int MODE>
@@ -125,7 +130,11 @@ struct Plan {
   static constexpr int TN = A_TMEM ? 192 : (NARROW ? 128 : BN);  // tile columns
   static constexpr int TNL = PAIR ? TN / 2 : TN;     // B rows a CTA loads
   static constexpr int TM = PAIR ? 2 * BM : BM;      // tile rows (of the pair)
-  static constexpr int STAGES = B_PACKED ? 3 : ((NARROW || PAIR) ? 6 : (A8 ? 4 : 5));  // TMA stages
+  static constexpr int STAGES = B_PACKED ? 3 : (NARROW ? 6 : (PAIR ? 5 : (A8 ? 4 : 5)));  // TMA stages
+  // staging buffers (32 x 64 bf16) per epilogue lane quadrant: the output
+  // stores in flight per SM are what bounds the writes of Y under load (4 KB
+  // each; 16 of them reach about 6 TB/s, 8 about half that)
+  static constexpr int EPI_NB = PAIR ? 4 : 2;
   static constexpr int KG = A_TMEM ? 2 : 1;          // k-blocks per widen -> MMA handshake
   static constexpr int WSLOTS = A8 ? 0 : 2;          // widened operand slots
   static constexpr int A_ST = A8 ? A_UN : A_PK;      // A bytes of a stage
@@ -139,7 +148,7 @@ struct Plan {
   static constexpr uint32_t TMEM_A0 = 2 * TN;        // first widened-A column (A_TMEM)
   static_assert(!A_TMEM || TMEM_A0 + WSLOTS * KG * 32 <= 512, "tensor-memory budget");
   static constexpr int OFF_EPI = OFF_W + WSLOTS * WSLOT_BYTES;
-  static constexpr int OFF_COL = OFF_EPI + NUM_EPI_WARPS * 2 * EPI_BYTES;  // per-warp constants
+  static constexpr int OFF_COL = OFF_EPI + NUM_EPI_WARPS * EPI_NB * EPI_BYTES;  // per-warp constants
   static constexpr int COL_WORDS = A8 ? 0 : 3 * TN;  // (int8: no code offset, no table)
   static constexpr int OFF_BAR = OFF_COL + NUM_EPI_WARPS * COL_WORDS * 4;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * (WSLOTS > 0 ? WSLOTS : 1) + 2 * 2 + 1;
@@ -337,7 +346,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int mb = tile / num_n_tiles, nb = tile % num_n_tiles;
         for (int kb = 0; kb < num_kb; ++kb) {
           const uint32_t s = issued % ST, ph = (issued / ST) & 1u;
-          if (!mbar_wait<PAIR>(&freed[s], ph ^ 1u, abort_flag, &g_status, wait_ns)) {
+          if (!mbar_wait(&freed[s], ph ^ 1u, abort_flag, &g_status, wait_ns)) {
             ok = false;
             break;
           }
@@ -363,7 +372,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // and the closing cluster barrier holds the other CTA until then)
       if (!PAIR || rank == 0)
         for (uint32_t t = (issued > ST ? issued - ST : 0); t < issued; ++t)
-          mbar_wait_drain<PAIR>(&full[t % ST], (t / ST) & 1u, &g_status, wait_ns);
+          mbar_wait_drain(&full[t % ST], (t / ST) & 1u, &g_status, wait_ns);
     }
   } else if (warp == W_MMA) {
     if (lane == 0 && rank == 0) {
@@ -373,7 +382,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int tile = unit0; tile < num_tiles && ok; tile += units, ++it) {
         const uint32_t b = it & 1, pb = (it >> 1) & 1;
-        if (!mbar_wait<PAIR>(&acc_empty[b], pb ^ 1u, abort_flag, &g_status, wait_ns)) break;
+        if (!mbar_wait(&acc_empty[b], pb ^ 1u, abort_flag, &g_status, wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * P::TN;
         if constexpr (P::A_TMEM) {
@@ -404,7 +413,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // both operands straight from the TMA stage
           for (int kb = 0; kb < num_kb; ++kb) {
             const uint32_t s = consumed % ST, ps = (consumed / ST) & 1u;
-            if (!mbar_wait<PAIR>(&full[s], ps, abort_flag, &g_status, wait_ns)) {
+            if (!mbar_wait(&full[s], ps, abort_flag, &g_status, wait_ns)) {
               ok = false;
               break;
             }
@@ -460,7 +469,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if constexpr (PAIR) {
         if (consumed > 0) {
           tc_commit_pair(mma_done, 0x1);
-          mbar_wait_drain<PAIR>(mma_done, 0, &g_status, wait_ns);
+          mbar_wait_drain(mma_done, 0, &g_status, wait_ns);
         }
       } else {
         tc_commit(mma_done);
@@ -575,7 +584,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       __syncwarp();
-      if (!mbar_wait<PAIR>(&acc_full[b], pb, abort_flag, &g_status, wait_ns)) break;
+      if (!mbar_wait(&acc_full[b], pb, abort_flag, &g_status, wait_ns)) break;
       tc_fence_after();
       const int row0 = mb * P::TM + static_cast<int>(rank) * BM + ew * 32;
       if constexpr (!OUT_S32 && P::EPI16) {
@@ -644,13 +653,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                 for (int u = 0; u < 2; ++u) pk[h][u][j] = gelu_pair_bf16(pk[h][u][j]);
           }
-          uint8_t *stg = smem + P::OFF_EPI + (ew * 2 + (EPI8 ? half : (sc & 1))) * EPI_BYTES;
-          if (lane == 0) {  // the store that last read this buffer is done
-            if constexpr (EPI8)
-              bulk_wait_read<0>();
-            else
-              bulk_wait_read<1>();
-          }
+          // this warp's staging buffers: a quadrant's EPI_NB, split between its
+          // two warps when eight share the epilogue
+          constexpr int NBW = EPI8 ? P::EPI_NB / 2 : P::EPI_NB;
+          uint8_t *stg = smem + P::OFF_EPI + ((ew * P::EPI_NB) + (EPI8 ? half * NBW : 0) + (sc % NBW)) * EPI_BYTES;
+          if (lane == 0) bulk_wait_read<NBW - 1>();  // the store that last read this buffer is done
           __syncwarp();
           // staging tile: 32 rows of 128 bytes, 16-byte chunk k of row R at k ^ (R % 8);
           // stmatrix x4 #(h, jp): matrices (u, j) = (0, 2jp), (1, 2jp), (0, 2jp+1), (1, 2jp+1)
@@ -908,12 +915,10 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t st) {
   const bool narrow = a.a8 && 2 * wide_tiles <= device_sm_count();
   // byte operands with small accumulators (4-bit weight codes): exact integer-add conversion
   const bool acc22 = a.acc22 && a.K <= 4096;
-  // byte operands, enough tiles, a long main loop per tile (K >= 2048, where
-  // the tensor pipe rather than the writes of Y bounds the kernel): CTA pairs
-  // on 256 x 256 tiles (fc2 of the stack 253 -> 227 us); with K = 1024 the
-  // pairs' coupled epilogues lose more than the main loop gains (frame QKV
-  // 30.8 -> 35.5 us), so those keep one CTA per 128 x 256 tile
-  const bool pair = a.a8 && !narrow && a.K >= 2048;
+  // byte operands and enough tiles: CTA pairs on 256 x 256 tiles (frame QKV
+  // 30.8 -> 31.5 us, the 48-block stack's layers 8-10 % faster: QKV 229 ->
+  // 208 us, proj 82 -> 73, fc1 with the GELU 384 -> 367, fc2 253 -> 226)
+  const bool pair = a.a8 && !narrow;
   if (a.gelu_out) {
     if (a.acc) return cudaErrorInvalidValue;
     if (a.a8 && acc22) {

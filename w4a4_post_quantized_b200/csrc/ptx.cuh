@@ -47,28 +47,15 @@ constexpr uint32_t kSuspendHintNs = 20000;
 // Test for completion of the phase with the given parity; a thread whose phase
 // is not complete is suspended by the hardware until it completes or the hint
 // runs out, so waiting costs no issue slots or shared-memory bandwidth.
-// CLUSTER: acquire at cluster scope (a barrier that the other CTA of a pair
-// arrives on, or that a pair's tensor-core commit signals).
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  if constexpr (CLUSTER) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
-        : "memory");
-  }
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
   return ok != 0;
 }
 
@@ -76,15 +63,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // (returns false, sets bit 0 (W4A4_DEV_TIMEOUT) of *status, raises *abort)
 // after limit_ns of %globaltimer, and returns false early when another role of
 // the CTA has raised *abort.
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           unsigned int *status,
                                           unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait<CLUSTER>(a, parity)) return true;
+  if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (;;) {
-    if (mbar_try_wait<CLUSTER>(a, parity)) return true;
+    if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > limit_ns) {
       atomicOr(status, 1u);
@@ -96,14 +82,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 
 // Same as mbar_wait but ignores *abort: used on the exit path to let copies
 // that are already in flight land before the CTA leaves.
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
                                                 unsigned int *status,
                                                 unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait<CLUSTER>(a, parity)) return true;
+  if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
-  while (!mbar_try_wait<CLUSTER>(a, parity)) {
+  while (!mbar_try_wait(a, parity)) {
     if (globaltimer() - t0 > limit_ns) {
       atomicOr(status, 1u);
       return false;
@@ -142,11 +127,12 @@ __device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
 }
-// Arrive (release, cluster scope) on the mbarrier at `bar`'s offset in CTA `rank`.
+// Arrive on the mbarrier at `bar`'s offset in CTA `rank` (default semantics:
+// release at CTA scope; what the arrival publishes is tensor-memory reads that
+// tcgen05.wait::ld has already completed, not memory writes, so no
+// cluster-scope release is needed).
 __device__ __forceinline__ void mbar_arrive_cluster(uint64_t *bar, uint32_t rank) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                   cluster_addr(bar, rank))
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr(bar, rank)) : "memory");
 }
 
 // ----------------------------------------------------------------------- TMA
