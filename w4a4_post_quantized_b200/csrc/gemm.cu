@@ -130,11 +130,11 @@ struct Plan {
   static constexpr int TN = A_TMEM ? 192 : (NARROW ? 128 : BN);  // tile columns
   static constexpr int TNL = PAIR ? TN / 2 : TN;     // B rows a CTA loads
   static constexpr int TM = PAIR ? 2 * BM : BM;      // tile rows (of the pair)
-  static constexpr int STAGES = B_PACKED ? 3 : (NARROW ? 6 : (PAIR ? 5 : (A8 ? 4 : 5)));  // TMA stages
-  // staging buffers (32 x 64 bf16) per epilogue lane quadrant: the output
-  // stores in flight per SM are what bounds the writes of Y under load (4 KB
-  // each; 16 of them reach about 6 TB/s, 8 about half that)
-  static constexpr int EPI_NB = PAIR ? 4 : 2;
+  static constexpr int STAGES = B_PACKED ? 3 : ((NARROW || PAIR) ? 6 : (A8 ? 4 : 5));  // TMA stages
+  // staging buffers (32 x 64 bf16) per epilogue lane quadrant (a CTA pair's
+  // eight epilogue warps take one each: 6 stages and 2 buffers measured 3 %
+  // faster on the K = 1024 layers than 5 and 4)
+  static constexpr int EPI_NB = 2;
   static constexpr int KG = A_TMEM ? 2 : 1;          // k-blocks per widen -> MMA handshake
   static constexpr int WSLOTS = A8 ? 0 : 2;          // widened operand slots
   static constexpr int A_ST = A8 ? A_UN : A_PK;      // A bytes of a stage
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       // (a pair's leader counts the epilogue warps of both CTAs)
-      mbar_init(&acc_empty[b], (GELU_OUT && P::A8 ? 2 : 1) * NUM_EPI_WARPS * (PAIR ? 2 : 1));
+      mbar_init(&acc_empty[b], ((GELU_OUT || PAIR) && P::A8 ? 2 : 1) * NUM_EPI_WARPS * (PAIR ? 2 : 1));
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -551,14 +551,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (warp >= W_EPI0 || (GELU_OUT && P::A8 && warp >= W_UNPACK0 && warp < W_UNPACK0 + 4)) {
+  } else if (warp >= W_EPI0 || ((GELU_OUT || P::PAIR) && P::A8 && warp >= W_UNPACK0 && warp < W_UNPACK0 + 4)) {
     // ---------------------------------------------------------------- epilogue
     const int ew = warp & 3;  // owns TMEM lanes 32 ew .. 32 ew + 31
     // With the GELU on the output (the epilogue's ALU work then exceeds the
-    // main loop's time) the byte-operand mode's idle warps 4..7 join in: the
-    // two warps of a lane quadrant take half of the tile's columns each, with
-    // one staging buffer each.
-    constexpr bool EPI8 = GELU_OUT && P::A8;
+    // main loop's time), and in a CTA pair, the byte-operand mode's idle warps
+    // 4..7 join in: the two warps of a lane quadrant take half of the tile's
+    // columns each, with one staging buffer each.
+    constexpr bool EPI8 = (GELU_OUT || P::PAIR) && P::A8;
     const int half = (EPI8 && warp < W_EPI0) ? 1 : 0;
     constexpr int SC_PER = EPI8 ? P::TN / EPI_COLS / 2 : P::TN / EPI_COLS;
     // this warp's copy of the tile's per-column constants:
