@@ -33,15 +33,17 @@
 //     through shared memory); pass 2 reads the values again and forms the
 //     codes with each token's reciprocal step, computed once by one lane.
 //
-// Warp roles (one persistent CTA of 384 threads per SM; tiles of 128 / S
+// Warp roles (one persistent CTA of 512 threads per SM; tiles of 128 / S
 // tokens round-robin over the CTAs):
 //   warp 0        producer: one bulk copy (K = 1024) or two TMA boxes (K = 4096)
 //                 per tile into a ring of stages
 //   warp 1        MMA issuer (one thread): 8 MMAs per tile into one of four
 //                 128-column accumulator slots of tensor memory
 //   warp 2        tensor-memory allocator
-//   warps 4..11   two finishing sets of 4 warps (one per lane quadrant);
-//                 successive tiles go to alternate sets
+//   warps 4..15   three finishing sets of 4 warps (one per lane quadrant);
+//                 successive tiles go to the sets in turn (a set's passes
+//                 wait on tensor-memory loads, so several tiles in flight
+//                 hide that latency)
 //
 // Every wait is bounded (ptx.cuh): a stuck pipeline sets the device status
 // word, the CTA lets its copies land and its MMAs finish, frees its tensor
@@ -60,9 +62,9 @@
 namespace w4a4 {
 namespace {
 
-constexpr int kTcThreads = 384;
+constexpr int kTcThreads = 512;
 constexpr int W_PROD = 0, W_MMA = 1, W_ALLOC = 2, W_FIN0 = 4;
-constexpr int kFinSets = 2;
+constexpr int kFinSets = 3;  // (with two, the 32-frame K = 1024 layers ran 8 % slower)
 constexpr int kSlots = 4;        // accumulator slots (128 columns each)
 constexpr int kHBytes = 128 * 128 * 2;
 
@@ -141,12 +143,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   {
     // H_128 in bf16, K-major with the 128-byte swizzle: row a' holds
     // H[a'][a] over a, in two 64-value halves of 16 KB (row a' at 128 a',
-    // 16-byte chunk c at c ^ (a' % 8))
+    // 16-byte chunk c at c ^ (a' % 8)).  One 16-byte store per chunk of 8
+    // values a = 8c + i: H[a'][a] = (-1)^(popc(a' & 8c) + popc(a' & i)), the
+    // row of H_8 selected by a' % 8, negated when a' & 8c has odd parity.
     uint8_t *h = smem + P::OFF_H;
-    for (int idx = threadIdx.x; idx < 128 * 128; idx += kTcThreads) {
-      const int ap = idx >> 7, a = idx & 127;
-      const uint32_t off = (a >> 6) * 16384 + ap * 128 + ((((a & 63) >> 3) ^ (ap & 7)) << 4) + (a & 7) * 2;
-      *reinterpret_cast<uint16_t *>(h + off) = (__popc(ap & a) & 1) ? 0xBF80u : 0x3F80u;
+    for (int q = threadIdx.x; q < 128 * 16; q += kTcThreads) {
+      const int ap = q >> 4, c = q & 15;
+      const uint32_t flip = (__popc(ap & (8 * c)) & 1) ? 0x80008000u : 0u;
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = (__popc(ap & 7 & (2 * k)) & 1) ? 0xBF80u : 0x3F80u;
+        const uint32_t hi = (__popc(ap & 7 & (2 * k + 1)) & 1) ? 0xBF80u : 0x3F80u;
+        w[k] = (lo | (hi << 16)) ^ flip;
+      }
+      *reinterpret_cast<uint4 *>(h + (c >> 3) * 16384 + ap * 128 + (((c & 7) ^ (ap & 7)) << 4)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
     }
     fence_proxy_async_smem();
   }
