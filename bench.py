@@ -878,6 +878,16 @@ def run_stack(args, st, world, rank, local):
         "achieved_moved": sum(q_moved) / (q_total_ms * 1e-3) / 1e9,
         "bytes_note": "algorithmic = 2 M K (X) + M K / 2 (4-bit codes) + 4 M (steps); moved: the codes "
                       "go one per byte on the fused call's route (3 M K + 4 M)"}
+    # the same kernel launched alone (per layer shape, back to back), weighted
+    # by the step's layers: in the step each launch also pays for the write-back
+    # of the GEMM output that the previous launch left dirty in L2
+    q_alone_ms = sum(per_layer[name]["alone_quantize_us"] * 1e-3 for (_, name, _, _) in layers)
+    roofline_q.update({
+        "achieved_alone": sum(q_bytes) / (q_alone_ms * 1e-3) / 1e9,
+        "frac_alone": sum(q_bytes) / (q_alone_ms * 1e-3) / 1e9 / peaks["hbm"],
+        "frac_alone_moved": sum(q_moved) / (q_alone_ms * 1e-3) / 1e9 / peaks["hbm"],
+        "timing": "frac: CUDA events around each quantize launch of one step (time-weighted); "
+                  "frac_alone: each layer shape's kernel alone, 10 back-to-back launches"})
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
