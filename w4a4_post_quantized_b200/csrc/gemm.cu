@@ -31,14 +31,19 @@
 //     qw8's operand order (the fused call's default route), or the W8A8
 //     setting's 8-bit codes in natural order.  TMA loads both straight into
 //     the 128-byte swizzled operand layout and the MMA reads them there
-//     (signed x signed); no widening at all; tiles 128 x 256.
+//     (signed x signed); no widening at all.  With enough tiles a cluster of
+//     two CTAs shares a 256 x 256 tile (cta_group::2: each CTA loads its 128
+//     rows of A and of B, the leader issues the MMAs, each CTA drains its own
+//     128 rows); small shapes take 128 x 128 tiles of one CTA.
 //
-// Warp roles (one persistent CTA per SM, tiles round-robin, M-major):
+// Warp roles (one persistent CTA, or CTA pair, per SM, tiles round-robin, M-major):
 //   warp 0      TMA producer (one thread)
 //   warp 1      tcgen05.mma issuer (one thread)
 //   warp 2      tensor-memory allocator
 //   warps 4..7  widen packed int4 -> int8 (into tensor memory, or into the
-//               swizzled shared-memory operand tiles of the packed-B path)
+//               swizzled shared-memory operand tiles of the packed-B path);
+//               with byte operands, a second epilogue warp per lane quadrant
+//               when the GELU is on the output or the CTAs work in pairs
 //   warps 8..11 epilogue: tcgen05.ld accumulators (64 columns at a time),
 //               subtract the code-offset term, scale by scale_tok[m] *
 //               scale_ch[n], add bias in fp32, round to bf16, TMA-store
