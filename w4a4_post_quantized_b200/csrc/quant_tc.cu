@@ -52,6 +52,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "codes.cuh"
 #include "ctxcache.h"
@@ -324,39 +325,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         inv_l = amax > 0.0f ? kQmax / amax : 0.0f;
       }
       tmem_wait_st();
-      // pass 2: codes
+      // pass 2: codes.  The common tile (every token present, no step so
+      // small that it needs the 2^64 rescale) runs without the per-token
+      // rescale and bounds tests.
       const unsigned long long magic2 = pack2(12582912.0f, 12582912.0f);
+      const bool plain_tile = !__any_sync(0xffffffffu, pre_l != 1.0f) && tok0 + TOKT <= M;
+      auto pass2 = [&](auto plain) {
+        constexpr bool PLAIN = decltype(plain)::value;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + 32 * c, r);
-        tmem_wait_ld();
-        if (c == 3) {                            // the slot is no longer read
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&d_free[d]);
-        }
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + 32 * c, r);
+          tmem_wait_ld();
+          if (c == 3) {                            // the slot is no longer read
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_free[d]);
+          }
 #pragma unroll
-        for (int u = 0; u < 32 / S; ++u) {
-          const int t = c * (32 / S) + u;
-          const float inv = __shfl_sync(0xffffffffu, inv_l, t);
-          const float pre = __shfl_sync(0xffffffffu, pre_l, t);
-          const int64_t tok = tok0 + t;
-          if (tok < M) {
-            float y[S];
+          for (int u = 0; u < 32 / S; ++u) {
+            const int t = c * (32 / S) + u;
+            const float inv = __shfl_sync(0xffffffffu, inv_l, t);
+            const int64_t tok = tok0 + t;
+            if (PLAIN || tok < M) {
+              float y[S];
 #pragma unroll
-            for (int b = 0; b < S; ++b) y[b] = __uint_as_float(r[u * S + b]);
-            if (pre != 1.0f) {
+              for (int b = 0; b < S; ++b) y[b] = __uint_as_float(r[u * S + b]);
+              if constexpr (!PLAIN) {
+                const float pre = __shfl_sync(0xffffffffu, pre_l, t);
+                if (pre != 1.0f) {
 #pragma unroll
-              for (int b = 0; b < S; ++b) y[b] *= pre;
+                  for (int b = 0; b < S; ++b) y[b] *= pre;
+                }
+              }
+              const unsigned long long inv2 = pack2(inv, inv);
+#pragma unroll
+              for (int b = 0; b < S; b += 2) fma_x2(y[b], y[b + 1], inv2, magic2);
+              store_code_words<S, CODE>(y, q + tok * code_bytes_of<CODE>(K) + ap * code_bytes_of<CODE>(S));
             }
-            const unsigned long long inv2 = pack2(inv, inv);
-#pragma unroll
-            for (int b = 0; b < S; b += 2) fma_x2(y[b], y[b + 1], inv2, magic2);
-            store_code_words<S, CODE>(y, q + tok * code_bytes_of<CODE>(K) + ap * code_bytes_of<CODE>(S));
           }
         }
-      }
+      };
+      if (plain_tile)
+        pass2(std::true_type{});
+      else
+        pass2(std::false_type{});
     }
   }
 
