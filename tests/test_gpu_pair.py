@@ -1,6 +1,6 @@
-"""The CTA-pair GEMM (byte operands, K >= 2048, enough tiles): two CTAs of a
-cluster share a 256 x 256 tile, each loading its 128 rows of A and of B, the
-leader issuing cta_group::2 MMAs.
+"""The CTA-pair GEMM (byte operands, enough tiles): two CTAs of a cluster
+share a 256 x 256 tile, each loading its 128 rows of A and of B, the leader
+issuing cta_group::2 MMAs.
 
   * accumulators bit-exact against the oracle's int64 product, with a ragged
     last pair tile (the second CTA's half partly or wholly past M), several
@@ -73,10 +73,13 @@ def test_pair_gemm_s32_int8_bit_exact(w4):
 
 
 @pytest.mark.parametrize("gelu", [False, True])
-def test_pair_outputs_equal_the_widening_route(w4, gelu):
-    M, N = 2500, 1024
-    X = synth.activations(M, K, seed=904)
-    W, b = synth.weights(N, K, seed=905), synth.bias(N, seed=906)
+@pytest.mark.parametrize("k,N", [(K, 1024), (1024, 4096)])
+def test_pair_outputs_equal_the_widening_route(w4, gelu, k, N):
+    """fc2-shaped (K = 4096) and fc1-shaped (K = 1024, N = 4096: the stack's
+    GELU layer) pair launches against the widening route, bit for bit."""
+    M = 2500
+    X = synth.activations(M, k, seed=904)
+    W, b = synth.weights(N, k, seed=905), synth.bias(N, seed=906)
     bf = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
     pw = w4.w4a4_prepare_weights(bf(W), bf(b), bf(X[:synth.calibration_rows(M)]))
     fl = w4.W4A4_FLAG_GELU_OUT if gelu else 0
