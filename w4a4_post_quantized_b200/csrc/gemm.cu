@@ -331,9 +331,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // TPRE (byte operands, small accumulators): every accumulator starts at the
+  // bit pattern of the float 1.5 * 2^23 and the MMAs always accumulate, so an
+  // accumulator's bits are the float 1.5 * 2^23 + acc (exact below 2^22) and
+  // the epilogue needs no integer add; each epilogue warp refills what it
+  // has read before it frees the buffer.  Here the epilogue warps fill both
+  // buffers of their lane quadrant once.
+  constexpr bool TPRE = ACC22 && P::A8 && !OUT_S32;
+  if constexpr (TPRE) {
+    constexpr bool E8 = (GELU_OUT || PAIR) && P::A8;
+    if (warp >= W_EPI0 || (E8 && warp >= W_UNPACK0)) {
+      const int cols_per_warp = E8 ? P::TN : 2 * P::TN;          // E8: each warp one buffer
+      const uint32_t c0 = E8 ? (warp >= W_EPI0 ? 0u : static_cast<uint32_t>(P::TN)) : 0u;
+      const uint32_t lanes = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      for (int c = 0; c < cols_per_warp; c += 32) tmem_fill_32x32b_x32(tmem_base + lanes + c0 + c, 0x4B400000u);
+      tmem_wait_st();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  // (a pair: both CTAs' barriers exist, and both tensor memories are filled,
+  // before either CTA signals the other or the leader's MMAs write them)
+  if constexpr (PAIR) cluster_sync();
+  tc_fence_after();
   // Everything above (barriers, tensor memory, descriptor prefetch) may overlap
   // the tail of the kernel that produced qx and scale_tok; from here on this
   // CTA reads what earlier kernels wrote.
@@ -427,12 +449,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t b0 = smem_u32(smem + s * P::STAGE_BYTES + P::OFF_ST_B);
 #pragma unroll
             for (int kk = 0; kk < BK / 32; ++kk) {
+              // (TPRE: the accumulators start at the float bias, always accumulate)
               if constexpr (PAIR)
                 mma_i8_pair(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
-                            P::IDESC, (kb | kk) != 0 ? 1u : 0u);
+                            P::IDESC, (TPRE || (kb | kk) != 0) ? 1u : 0u);
               else
                 mma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), P::IDESC,
-                       (kb | kk) != 0 ? 1u : 0u);
+                       (TPRE || (kb | kk) != 0) ? 1u : 0u);
             }
             if constexpr (PAIR)
               tc_commit_pair(&freed[s], 0x3);  // frees the stage in both CTAs
@@ -611,7 +634,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld_16x256b_x8(tbase + sc * EPI_COLS, r[0]);
           tmem_ld_16x256b_x8(tbase + (16u << 16) + sc * EPI_COLS, r[1]);
           tmem_wait_ld();
+          if constexpr (TPRE) {  // the columns just read start the buffer's next tile at the bias
+            tmem_fill_32x32b_x32(tbase + sc * EPI_COLS, 0x4B400000u);
+            tmem_fill_32x32b_x32(tbase + sc * EPI_COLS + 32, 0x4B400000u);
+          }
           if (sc == (half + 1) * SC_PER - 1) {
+            if constexpr (TPRE) tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -627,7 +655,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int n = nb * TN + c0 + 8 * j + tc;  // N is even: the pair is all in or all out
-            int2 o = make_int2(0x4B400000, 0x4B400000);
+            int2 o = TPRE ? make_int2(0, 0) : make_int2(0x4B400000, 0x4B400000);
             float2 scl = make_float2(0.0f, 0.0f), bi = make_float2(0.0f, 0.0f);
             if (n < N) {
               if constexpr (P::A_TMEM) {
