@@ -32,6 +32,8 @@
 //     per-token maxima (warp shuffles, then one exchange between the 4 warps
 //     through shared memory); pass 2 reads the values again and forms the
 //     codes with each token's reciprocal step, computed once by one lane.
+//     Each pass reads its 128 columns in four 32-column loads; at K = 4096
+//     the next load is issued before the current chunk is worked on.
 //
 // Warp roles (one persistent CTA of 512 threads per SM; tiles of 128 / S
 // tokens round-robin over the CTAs):
@@ -267,11 +269,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // pass 1: H_S and the multipliers, written back in place (tcgen05.st),
       // and the per-token maxima over this warp's 32 lanes
       float tok_max[TOKT];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {              // 32 columns = 32 / S tokens
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + 32 * c, r);
-        tmem_wait_ld();
+      auto pass1_chunk = [&](int c, uint32_t(&r)[32]) {
 #pragma unroll
         for (int u = 0; u < 32 / S; ++u) {
           float y[S];
@@ -281,6 +279,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int b = 0; b < S; ++b) r[u * S + b] = __float_as_uint(y[b]);
         }
         tmem_st_32x32b_x32(taddr + 32 * c, r);
+      };
+      if constexpr (S == 32) {
+        // one token per chunk: chunk c + 1's load is in flight while chunk c
+        // is transformed (87936 tokens: 201 -> 199 us at K = 4096; at
+        // K = 1024 the second buffer cost more than the overlap gained,
+        // 44 -> 50 us, so S = 8 keeps one load at a time)
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(taddr, ra);
+        tmem_wait_ld();
+        tmem_ld_32x32b_x32(taddr + 32, rb);
+        pass1_chunk(0, ra);
+        tmem_wait_ld();
+        tmem_ld_32x32b_x32(taddr + 64, ra);
+        pass1_chunk(1, rb);
+        tmem_wait_ld();
+        tmem_ld_32x32b_x32(taddr + 96, rb);
+        pass1_chunk(2, ra);
+        tmem_wait_ld();
+        pass1_chunk(3, rb);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {              // 32 columns = 32 / S tokens
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + 32 * c, r);
+          tmem_wait_ld();
+          pass1_chunk(c, r);
+        }
       }
       // maxima over the warp, reduce-scattered: at the step with lane offset
       // o a lane keeps the half of its remaining tokens that its lane bit
@@ -330,18 +355,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // rescale and bounds tests.
       const unsigned long long magic2 = pack2(12582912.0f, 12582912.0f);
       const bool plain_tile = !__any_sync(0xffffffffu, pre_l != 1.0f) && tok0 + TOKT <= M;
+      auto release_slot = [&]() {                // the slot is no longer read
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_free[d]);
+      };
       auto pass2 = [&](auto plain) {
         constexpr bool PLAIN = decltype(plain)::value;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + 32 * c, r);
-          tmem_wait_ld();
-          if (c == 3) {                            // the slot is no longer read
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&d_free[d]);
-          }
+        auto codes_chunk = [&](int c, const uint32_t(&r)[32]) {
 #pragma unroll
           for (int u = 0; u < 32 / S; ++u) {
             const int t = c * (32 / S) + u;
@@ -363,6 +384,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               for (int b = 0; b < S; b += 2) fma_x2(y[b], y[b + 1], inv2, magic2);
               store_code_words<S, CODE>(y, q + tok * code_bytes_of<CODE>(K) + ap * code_bytes_of<CODE>(S));
             }
+          }
+        };
+        if constexpr (S == 32) {                 // loads overlapped as in pass 1
+          uint32_t ra[32], rb[32];
+          tmem_ld_32x32b_x32(taddr, ra);
+          tmem_wait_ld();
+          tmem_ld_32x32b_x32(taddr + 32, rb);
+          codes_chunk(0, ra);
+          tmem_wait_ld();
+          tmem_ld_32x32b_x32(taddr + 64, ra);
+          codes_chunk(1, rb);
+          tmem_wait_ld();
+          tmem_ld_32x32b_x32(taddr + 96, rb);
+          codes_chunk(2, ra);
+          tmem_wait_ld();
+          release_slot();
+          codes_chunk(3, rb);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(taddr + 32 * c, r);
+            tmem_wait_ld();
+            if (c == 3) release_slot();
+            codes_chunk(c, r);
           }
         }
       };
