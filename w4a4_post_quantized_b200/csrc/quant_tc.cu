@@ -177,6 +177,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == W_PROD) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
+      // K = 4096: X is read once, and its lines are made the first to go when
+      // L2 needs room (87936 tokens: 199 -> 195 us alone, 249 -> 241 us
+      // inside the stack step).  At K = 1024 the same hint made the kernel
+      // alone slower (44 -> 48 us) and left it unchanged in the step.
+      const uint64_t x_policy = S == 8 ? 0 : l2_policy_evict_first();
       uint32_t it = 0;
       for (int g = blockIdx.x; g < num_tiles; g += gridDim.x, ++it) {
         const uint32_t s = it % P::XST;
@@ -194,8 +199,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // rows (token, a) of S values through the 64-byte swizzle, 256 rows
           // (two tokens) per box; rows past the end are filled with zeros
           mbar_arrive_expect_tx(&x_full[s], P::X_BYTES);
-          tma_load_2d(dst, &tmX, 0, static_cast<int>(g * 512), &x_full[s]);
-          tma_load_2d(dst + P::X_BYTES / 2, &tmX, 0, static_cast<int>(g * 512 + 256), &x_full[s]);
+          tma_load_2d_hint(dst, &tmX, 0, static_cast<int>(g * 512), &x_full[s], x_policy);
+          tma_load_2d_hint(dst + P::X_BYTES / 2, &tmX, 0, static_cast<int>(g * 512 + 256), &x_full[s],
+                           x_policy);
         }
       }
       // let every issued copy land before the CTA can exit
