@@ -3,7 +3,8 @@ script and against the oracle's exact-erf GELU, on the CPU.
 
   * the coefficients compiled into gelu.cuh are the ones
     w4a4_post_quantized_b200/gelu_fit.py produces, and the fit describes
-    log2 Phi(-a) on [0, 5.9375] to within 1e-6;
+    log2 Phi(-a) on [0, 5.9375] to within 1e-5 (a relative error of Phi
+    under 7e-6, some 300 times finer than a bf16 step);
   * for every bf16 input x with 1e-30 <= |x| <= 5.9375, an emulation of the
     kernel's binary32 arithmetic gives the oracle's GELU rounded to bf16 bit
     for bit, whatever value within 3e-7 relative of 2^arg the hardware's
@@ -30,19 +31,21 @@ EX2_REL = 3e-7      # bound on ex2.approx.ftz.f32's relative error (2^-22 = 2.4e
 
 def _header_coefficients():
     text = open(HDR).read()
-    m = re.search(r"kC\[11\]\s*=\s*\{([^}]*)\}", text)
+    m = re.search(r"kC\[(\d+)\]\s*=\s*\{([^}]*)\}", text)
     assert m, "coefficient table not found in gelu.cuh"
-    return [float(v.strip().rstrip("f")) for v in m.group(1).split(",")]
+    c = [float(v.strip().rstrip("f")) for v in m.group(2).split(",")]
+    assert len(c) == int(m.group(1)) == gelu_fit.DEG + 1
+    return c
 
 
 def test_header_coefficients_are_the_fit():
     assert _header_coefficients() == gelu_fit.coefficients()
-    assert gelu_fit.max_fit_error() < 1e-6
+    assert gelu_fit.max_fit_error() < 1e-5
     # the fit is log2 Phi(-a): Phi(0) = 1/2 and Phi(-1) = 0.158655...
     c = np.array(gelu_fit.coefficients(), dtype=np.float64)
-    assert abs(np.polynomial.polynomial.polyval(-1.0, c) + 1.0) < 1e-6
+    assert abs(np.polynomial.polynomial.polyval(-1.0, c) + 1.0) < 1e-5
     u1 = 1.0 / (gelu_fit.A / 2) - 1.0
-    assert abs(2.0 ** np.polynomial.polynomial.polyval(u1, c) / (0.5 * math.erfc(1 / math.sqrt(2))) - 1) < 1e-6
+    assert abs(2.0 ** np.polynomial.polynomial.polyval(u1, c) / (0.5 * math.erfc(1 / math.sqrt(2))) - 1) < 1e-5
 
 
 def _f32(x):
@@ -66,8 +69,8 @@ def _kernel_gelu(x32, ex2_scale=1.0):
     c = [np.float32(v) for v in _header_coefficients()]
     na = np.maximum(-np.abs(x32), -A).astype(np.float32)
     u = _fma(na, np.full_like(na, -(np.float32(2.0) / A)), np.full_like(na, np.float32(-1.0)))
-    p = np.full_like(na, c[10])
-    for i in range(9, -1, -1):
+    p = np.full_like(na, c[-1])
+    for i in range(len(c) - 2, -1, -1):
         p = _fma(p, u, np.full_like(na, c[i]))
     ph = _f32(np.exp2(p.astype(np.float64)) * ex2_scale)
     relu = np.maximum(x32, np.float32(0.0)).astype(np.float32)
