@@ -861,7 +861,7 @@ def run_stack(args, st, world, rank, local):
         "unit": "TOPS", "frac": g_ach / int8_peak,
         "traffic": profile_traffic("gemm.cu", f"gemm_{args.workload}"),
         "peak_note": f"int8 = {INT8_PER_BF16:g} x {peaks['src']} sustained bf16 {peaks['bf16_sus']} TFLOP/s "
-                     "(the kernel runs inside an 80 ms step under the power cap)",
+                     "(the kernel runs inside a 66 ms step under the power cap)",
         "frac_of_nominal_4500": g_ach / nominal_int8,
         "frac_of_measured_int8_ceiling": (g_ach / ceiling["tops"]) if ceiling.get("tops") else None,
         "measured_int8_ceiling": ceiling,
