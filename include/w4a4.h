@@ -77,7 +77,12 @@ typedef enum {
 /* Flags. */
 #define W4A4_FLAG_GELU  0x1u  /* quantize_act / linear_fused: apply exact-erf GELU
                                  to X (rounded to bf16) before the rotation; the
-                                 input of an MLP's second linear */
+                                 input of an MLP's second linear.  The value is
+                                 the exact GELU rounded to bf16 for every bf16 x
+                                 with 1e-30 <= |x| <= 5.9375; x itself above
+                                 5.9375; -8.6e-9 below -5.9375 (the exact values
+                                 lie between it and 0); x/2 within one bf16 step
+                                 for |x| < 1e-30 */
 #define W4A4_FLAG_PLAIN 0x2u  /* no rotation and no smoothing: plain per-token /
                                  per-channel int4 quantization (the baseline that
                                  DSFQ is measured against); must match between
